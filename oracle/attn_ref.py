@@ -1,0 +1,133 @@
+"""Plain fp64 CPU oracle for the scaled-dot-product attention forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+and reference legs may call it.  It shares no code with the CUDA library.
+
+What it computes
+----------------
+The pages ("Making AMD GPUs go brrr", section "Real kernel example"; and
+"HipKittens: fast and furious AMD kernels", section "Performance results")
+name a tiled attention forward kernel -- causal and non-causal, over several
+head dims D and sequence lengths N -- whose hot loop is built from a score
+matmul, ``exp2`` and row sums, but print no formula.  The definition used
+here is the plain one that such a kernel reaches up to rounding order:
+
+    S   = scale * Q_h K_{kv(h)}^T                     (N x N)
+    S_ij = -inf        for j > i            (causal only, top-left aligned)
+    P   = row-softmax(S)
+    O_h = P V_{kv(h)}                                  (N x D)
+    LSE_i = ln sum_j exp(S_ij)             (natural log of the scaled scores)
+
+with kv(h) = h // (Hq / Hkv) (contiguous query-head groups share one KV head).
+Everything is evaluated in float64 on the bf16 input values upcast exactly;
+the full score matrix of one head is materialised, no blocking, no online
+softmax.  The readings of what the pages leave open (formula, LSE base,
+causal alignment, head mapping, layout) are listed in the design notes.
+
+Parity status: every function below is pinned by tests/test_oracle.py
+(closed forms, invariants, a scalar brute force and a library special case)
+and by tests/test_oracle_mutants.py (planted mistakes must fail a pin).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _as_f64(x) -> np.ndarray:
+    """Upcast a numpy array or a CPU torch tensor (bf16/fp32/fp64) to fp64."""
+    if hasattr(x, "detach"):  # torch tensor: go through float32, exact for bf16
+        import torch
+
+        x = x.detach().to("cpu")
+        if x.dtype != torch.float64:
+            x = x.to(torch.float32)
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def kv_head(h: int, Hq: int, Hkv: int) -> int:
+    """Query head h reads KV head h // (Hq/Hkv): contiguous groups of Hq/Hkv."""
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return h // (Hq // Hkv)
+
+
+def head_scores(qh: np.ndarray, kh: np.ndarray, causal: bool, scale: float) -> np.ndarray:
+    """Scaled, masked score matrix of one head: S = scale * q k^T, -inf above the diagonal if causal."""
+    S = scale * (qh @ kh.T)
+    if causal:
+        n_q, n_k = S.shape
+        i = np.arange(n_q)[:, None]
+        j = np.arange(n_k)[None, :]
+        S = np.where(j > i, -np.inf, S)
+    return S
+
+
+def head_probs(qh, kh, causal: bool, scale: float) -> np.ndarray:
+    """Row-softmax of the head's score matrix (each row sums to 1)."""
+    S = head_scores(_as_f64(qh), _as_f64(kh), causal, scale)
+    m = S.max(axis=1, keepdims=True)
+    E = np.exp(S - m)
+    return E / E.sum(axis=1, keepdims=True)
+
+
+def head_forward(qh, kh, vh, causal: bool, scale: float):
+    """One head: returns (O [N, D], LSE [N]) in fp64."""
+    qh, kh, vh = _as_f64(qh), _as_f64(kh), _as_f64(vh)
+    S = head_scores(qh, kh, causal, scale)
+    m = S.max(axis=1, keepdims=True)
+    E = np.exp(S - m)
+    l = E.sum(axis=1, keepdims=True)
+    O = (E / l) @ vh
+    lse = m[:, 0] + np.log(l[:, 0])
+    return O, lse
+
+
+def attention_forward(q, k, v, causal: bool, scale: float):
+    """Full forward: q [B,Hq,N,D], k/v [B,Hkv,N,D] -> (O [B,Hq,N,D], LSE [B,Hq,N]), fp64.
+
+    Computed one (b, h) head at a time, each with its full N x N score matrix.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    O = np.empty((B, Hq, N, v.shape[3]), dtype=np.float64)
+    lse = np.empty((B, Hq, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            kh = kv_head(h, Hq, Hkv)
+            O[b, h], lse[b, h] = head_forward(q[b, h], k[b, kh], v[b, kh], causal, scale)
+    return O, lse
+
+
+def attention_rows(q, k, v, rows, causal: bool, scale: float):
+    """Selected output rows, each from its own score row (for full-size sampled checks).
+
+    ``rows`` is a list of (b, h, i).  Row i of head (b, h) is the softmax of
+    scale * q[b,h,i] . k[b,kv(h),j] over the allowed keys j (all j, or j <= i
+    when causal), applied to V.  Returns (O [len(rows), D], LSE [len(rows)]).
+    Accepts torch tensors without converting them whole.
+    """
+    Hq = q.shape[1]
+    Hkv = k.shape[1]
+    out_o = []
+    out_l = []
+    cache_key = None
+    kh_arr = vh_arr = None
+    for (b, h, i) in rows:
+        kh = kv_head(h, Hq, Hkv)
+        if cache_key != (b, kh):
+            kh_arr = _as_f64(k[b, kh])
+            vh_arr = _as_f64(v[b, kh])
+            cache_key = (b, kh)
+        qi = _as_f64(q[b, h, i])
+        s = scale * (kh_arr @ qi)
+        if causal:
+            s = np.where(np.arange(s.shape[0]) > i, -np.inf, s)
+        m = s.max()
+        e = np.exp(s - m)
+        l = e.sum()
+        out_o.append((e / l) @ vh_arr)
+        out_l.append(m + np.log(l))
+    return np.stack(out_o), np.asarray(out_l)
