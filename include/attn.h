@@ -1,0 +1,114 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) bf16 attention forward library.
+ *
+ * The operation is the tiled attention forward pass named by "HipKittens:
+ * fast and furious AMD kernels" (section "Performance results": an attention
+ * forward kernel over several head dims D and sequence lengths N, causal and
+ * non-causal) and "Making AMD GPUs go brrr" (section "Real kernel example":
+ * a hot loop built from a score matmul, exp2 and row sums).  The pages print
+ * no formula; the library computes the plain definition
+ *
+ *     O[b,h]    = softmax(scale * Q[b,h] K[b,g(h)]^T  (+ causal mask)) V[b,g(h)]
+ *     LSE[b,h,i] = ln sum_j exp(scale * q_i . k_j)      (over the allowed keys j)
+ *
+ * with g(h) = h / (Hq / Hkv) (contiguous groups of query heads share one KV
+ * head) and, when causal, key j allowed for query i iff j <= i.
+ *
+ * Every entry point validates its arguments on the host before touching the
+ * GPU and returns an attn_status_t code; ATTN_OK is 0.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null pointer, negative size, Hq % Hkv != 0, non-finite scale */
+  ATTN_ERR_UNSUPPORTED = 2, /* head dim D other than 64 or 128, or a size beyond the limits below */
+  ATTN_ERR_MISALIGNED = 3,  /* a q/k/v/o pointer not 16-byte aligned, or lse not 4-byte aligned */
+  ATTN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
+  ATTN_ERR_TIMEOUT = 5      /* a kernel wait gave up (reported by attn_device_status) */
+} attn_status_t;
+
+/*
+ * attn_fwd -- enqueue one attention forward pass on `stream`.
+ *
+ * Arguments (all pointers are DEVICE pointers; the caller allocates, owns and
+ * frees every buffer; the library allocates nothing and keeps no pointer):
+ *   q     bf16 [B, Hq,  N, D], contiguous, row-major (D fastest).   read
+ *   k     bf16 [B, Hkv, N, D], contiguous.                          read
+ *   v     bf16 [B, Hkv, N, D], contiguous.                          read
+ *   o     bf16 [B, Hq,  N, D], contiguous.                          written (every element)
+ *   lse   fp32 [B, Hq,  N],    contiguous; natural-log log-sum-exp of the
+ *         scaled, masked scores of each query row.                  written (every element)
+ *   B, Hq, Hkv, N   batch, query heads, key/value heads, sequence length.
+ *         B >= 0, N >= 0, Hq >= 1, Hkv >= 1, Hq % Hkv == 0.  B == 0 or N == 0
+ *         is an empty problem: ATTN_OK is returned and nothing is launched
+ *         (pointers may then be null).  Limits: B*Hq <= 2^31-1 and N <= 2^31-1.
+ *   D     head dim of q, k, v and o: 64 or 128.
+ *   causal  0: every key is visible; non-zero: key j is visible to query i
+ *         iff j <= i (queries and keys share positions 0..N-1).
+ *   scale   finite float multiplying q.k before the softmax (1/sqrt(D) is
+ *         the usual choice; 0 and negative values are accepted).
+ *   stream  cudaStream_t (passed as void*) on which the kernel is enqueued;
+ *         null means the legacy default stream.  The call is asynchronous:
+ *         results are valid once the stream has reached this point.
+ *
+ * Errors: the host checks above are made before any CUDA call; on any error
+ * return nothing is launched and o/lse are untouched.  ATTN_ERR_CUDA means a
+ * CUDA call (tensor-map encode, attribute, launch) failed; the CUDA error
+ * string is available from attn_last_cuda_error().  The kernel's waits are
+ * bounded; if one gives up the kernel exits early and records the fact, which
+ * attn_device_status() reports after the caller synchronises.
+ *
+ * Numerics: fp32 accumulation of Q K^T and P V on the tensor cores, base-2
+ * online softmax in fp32, probabilities rounded to bf16 before P V, O rounded
+ * to bf16 (nearest-even).  The result is bitwise deterministic for a given
+ * input, device and build.
+ *
+ * Thread safety: calls are independent and may be made from several host
+ * threads and streams at once.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+             void* stream);
+
+/* Human-readable name of an attn_status_t value (static string, never null). */
+const char* attn_status_string(int status);
+
+/*
+ * Text of the last CUDA error seen by an entry point on the calling host
+ * thread ("" if none).  Static per-thread storage; valid until the next call
+ * on that thread.
+ */
+const char* attn_last_cuda_error(void);
+
+/*
+ * attn_device_status -- synchronise `stream` (void* cudaStream_t) and report
+ * whether any kernel of this library, on the current device, gave up on a
+ * bounded wait since the previous call.  Returns ATTN_OK or ATTN_ERR_TIMEOUT
+ * (and clears the record), or ATTN_ERR_CUDA if the synchronisation failed.
+ * If `site` is non-null it receives the code of the wait that gave up (0 if
+ * none).
+ */
+int attn_device_status(void* stream, int* site);
+
+/*
+ * attn_num_units -- number of work units (one unit = 256 query rows of one
+ * query head) a call with these sizes schedules; the persistent grid is
+ * min(units, SM count).  Host-only helper, no CUDA call.  Returns -1 on
+ * invalid sizes.
+ */
+long long attn_num_units(int B, int Hq, int N);
+
+/* Version string of the library build (static). */
+const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

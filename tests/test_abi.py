@@ -1,0 +1,91 @@
+"""The C ABI on the host: the library loads, exports what include/attn.h declares,
+and rejects bad arguments before any CUDA call (no GPU needed)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import tiled_attention_forward_03_b200 as attn
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED = (attn.ATTN_OK, attn.ATTN_ERR_INVALID_ARG,
+                                        attn.ATTN_ERR_UNSUPPORTED, attn.ATTN_ERR_MISALIGNED)
+P = 0x10000  # a 16-byte aligned fake device address; never dereferenced by a rejected call
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(HEADER, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(attn_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for required in ("attn_fwd", "attn_status_string", "attn_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(attn.lib_path)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_library_is_in_tree_and_built_for_sm100a():
+    assert os.path.dirname(attn.lib_path) == os.path.dirname(os.path.abspath(attn.__file__))
+    assert "sm_100a" in attn.attn_version()
+
+
+def test_status_strings():
+    assert attn.attn_status_string(OK) == "ATTN_OK"
+    assert attn.attn_status_string(attn.ATTN_ERR_TIMEOUT) == "ATTN_ERR_TIMEOUT"
+    assert attn.attn_status_string(12345) == "ATTN_ERR_UNKNOWN"
+
+
+def call(**kw):
+    args = dict(q=P, k=P, v=P, o=P, lse=P, B=1, Hq=2, Hkv=1, N=128, D=128, causal=0, scale=0.125, stream=None)
+    args.update(kw)
+    return attn.attn_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["Hq"],
+                         args["Hkv"], args["N"], args["D"], args["causal"], args["scale"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(q=None), INVALID), (dict(k=None), INVALID), (dict(v=None), INVALID),
+    (dict(o=None), INVALID), (dict(lse=None), INVALID),
+    (dict(B=-1), INVALID), (dict(N=-5), INVALID), (dict(Hq=0), INVALID), (dict(Hkv=0), INVALID),
+    (dict(Hq=3, Hkv=2), INVALID), (dict(scale=math.nan), INVALID), (dict(scale=math.inf), INVALID),
+    (dict(D=96), UNSUPPORTED), (dict(D=256), UNSUPPORTED), (dict(D=0), UNSUPPORTED),
+    (dict(q=P + 8), MISALIGNED), (dict(k=P + 2), MISALIGNED), (dict(v=P + 4), MISALIGNED),
+    (dict(o=P + 1), MISALIGNED), (dict(lse=P + 2), MISALIGNED),
+])
+def test_rejected_before_any_cuda_call(kw, expected):
+    assert call(**kw) == expected
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(N=0), dict(B=0, q=None, k=None, v=None, o=None, lse=None)])
+def test_empty_problem_is_ok_without_launch(kw):
+    assert call(**kw) == OK
+
+
+def test_lse_only_needs_4_byte_alignment():
+    # Misalignment is checked after null/size checks; a 4-byte aligned lse passes it,
+    # so the call only fails later, at the first CUDA call, when no GPU is present.
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("needs a machine without a GPU")
+    assert call(lse=P + 4) == attn.ATTN_ERR_CUDA
+
+
+def test_num_units():
+    assert attn.attn_num_units(4, 16, 2048) == 4 * 16 * 8
+    assert attn.attn_num_units(1, 2, 129) == 2 * 1
+    assert attn.attn_num_units(1, 1, 257) == 2
+    assert attn.attn_num_units(0, 1, 100) == 0
+    assert attn.attn_num_units(1, 0, 100) == -1

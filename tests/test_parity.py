@@ -1,0 +1,216 @@
+"""GPU parity: the CUDA attention forward against the fp64 oracle (needs a B200).
+
+Tolerances (stated for this path): over all compared O elements, max |dO| <= 2e-2
+and mean |dO| <= 2e-3; over all compared rows, max |dLSE| <= 1e-3.  Small cases
+are compared element by element in full; the full-size workloads are compared on
+seeded sampled rows (plus one whole head), each row computed by the oracle on its own.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention_forward, attention_rows, head_forward
+from tiled_attention_forward_03_b200.synth import (
+    CFG1, CFG2, CFG3, CFG4, make_qkv, make_workload_inputs, sample_rows, sweep_points)
+
+pytestmark = pytest.mark.gpu
+
+TOL_O_MAX = 2e-2
+TOL_O_MEAN = 2e-3
+TOL_LSE = 1e-3
+
+
+@pytest.fixture(scope="module")
+def attn():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import tiled_attention_forward_03_b200 as mod
+    return mod
+
+
+def gpu_forward(attn, q, k, v, causal, scale):
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    o, lse = attn.forward(qd, kd, vd, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    st, site = attn.device_status()
+    assert st == attn.ATTN_OK, f"kernel wait gave up at site {site}"
+    return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def assert_close(o, lse, o_ref, lse_ref, what=""):
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse)), f"{what}: non-finite output"
+    d = np.abs(o - o_ref)
+    dl = np.abs(lse - lse_ref)
+    msg = f"{what}: max|dO|={d.max():.3e} mean|dO|={d.mean():.3e} max|dLSE|={dl.max():.3e}"
+    assert d.max() <= TOL_O_MAX, msg
+    assert d.mean() <= TOL_O_MEAN, msg
+    assert dl.max() <= TOL_LSE, msg
+
+
+def check_full(attn, q, k, v, causal, scale, what=""):
+    o, lse = gpu_forward(attn, q, k, v, causal, scale)
+    o_ref, lse_ref = attention_forward(q, k, v, causal, scale)
+    assert_close(o, lse, o_ref, lse_ref, what)
+    return o, lse
+
+
+def check_sampled(attn, w, q, k, v, count=256, full_heads=((0, 0),)):
+    o, lse = gpu_forward(attn, q, k, v, w.causal, w.softmax_scale)
+    rows = sample_rows(w.B, w.Hq, w.N, count, seed=w.seed + 7)
+    o_ref, lse_ref = attention_rows(q, k, v, rows, w.causal, w.softmax_scale)
+    idx = tuple(np.array(x) for x in zip(*rows))
+    assert_close(o[idx], lse[idx], o_ref, lse_ref, w.name + " sampled rows")
+    g = w.Hq // w.Hkv
+    for (b, h) in full_heads:
+        oh, lh = head_forward(q[b, h], k[b, h // g], v[b, h // g], w.causal, w.softmax_scale)
+        assert_close(o[b, h], lse[b, h], oh, lh, f"{w.name} head {(b, h)}")
+    # properties at any size: finite everywhere, LSE >= the row's largest allowed score
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+
+
+# ------------------------------------------------------------------ the five workloads
+
+def test_cfg1_full(attn):
+    q, k, v = make_workload_inputs(CFG1)
+    check_full(attn, q, k, v, CFG1.causal, CFG1.softmax_scale, CFG1.name)
+
+
+def test_cfg2_full(attn):
+    q, k, v = make_workload_inputs(CFG2)
+    check_full(attn, q, k, v, CFG2.causal, CFG2.softmax_scale, CFG2.name)
+
+
+def test_cfg3_sampled(attn):
+    q, k, v = make_workload_inputs(CFG3)
+    check_sampled(attn, CFG3, q, k, v, full_heads=((0, 0), (15, 15)))
+
+
+def test_cfg4_sampled(attn):
+    q, k, v = make_workload_inputs(CFG4)
+    check_sampled(attn, CFG4, q, k, v, full_heads=((7, 31),))
+
+
+@pytest.mark.parametrize("w", sweep_points(), ids=lambda w: w.name)
+def test_sweep_point(attn, w):
+    q, k, v = make_workload_inputs(w)
+    if w.N <= 2048:
+        check_full(attn, q, k, v, w.causal, w.softmax_scale, w.name)
+    else:
+        check_sampled(attn, w, q, k, v, count=128, full_heads=())
+
+
+# ------------------------------------------------------------------ edge shapes
+
+EDGE = [
+    # (B, Hq, Hkv, N, D, causal)
+    (1, 1, 1, 1, 64, False), (1, 1, 1, 1, 128, True), (2, 2, 2, 7, 64, True), (1, 2, 1, 7, 128, False),
+    (1, 2, 2, 127, 128, True), (1, 2, 2, 127, 64, False), (1, 2, 2, 128, 128, True),
+    (1, 2, 2, 129, 128, True), (1, 2, 2, 129, 64, False), (1, 2, 2, 255, 64, True),
+    (1, 2, 2, 256, 128, False), (1, 2, 2, 257, 128, True), (2, 4, 2, 383, 64, True),
+    (1, 4, 1, 1000, 128, True), (1, 4, 1, 1000, 128, False), (1, 8, 1, 640, 64, True),
+    (3, 8, 4, 300, 128, False), (1, 16, 2, 513, 128, True),
+]
+
+
+@pytest.mark.parametrize("shape", EDGE, ids=lambda s: "B{}_Hq{}_Hkv{}_N{}_D{}_{}".format(*s[:5], "c" if s[5] else "nc"))
+def test_edge_shapes(attn, shape):
+    B, Hq, Hkv, N, D, causal = shape
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, seed=3000 + N + D + Hq)
+    check_full(attn, q, k, v, causal, 1.0 / math.sqrt(D), str(shape))
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.0883883, 0.02, 0.5])
+@pytest.mark.parametrize("causal", [False, True])
+def test_scales(attn, scale, causal):
+    q, k, v = make_qkv(1, 2, 2, 300, 128, seed=4001)
+    check_full(attn, q, k, v, causal, scale, f"scale={scale}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_growing_scores_exercise_rescale(attn, causal):
+    """Keys whose norm grows along the sequence push each row's running max up by far
+    more than the lazy-rescale threshold several times, so the O correction runs."""
+    q, k, v = make_qkv(1, 2, 1, 1024, 128, seed=4002)
+    grow = torch.linspace(0.2, 6.0, 1024).reshape(1, 1, 1024, 1)
+    k = (k.float() * grow).to(torch.bfloat16)
+    q = (q.float() * 2.0).to(torch.bfloat16)
+    check_full(attn, q, k, v, causal, 1.0 / math.sqrt(128), "growing scores")
+
+
+def test_large_magnitude_inputs(attn):
+    q, k, v = make_qkv(1, 2, 2, 512, 64, seed=4003)
+    q = (q.float() * 8).to(torch.bfloat16)
+    k = (k.float() * 8).to(torch.bfloat16)
+    check_full(attn, q, k, v, True, 0.125, "large magnitude")
+
+
+# ------------------------------------------------------------------ invariants on the GPU path
+
+def test_identical_v_rows_give_that_row(attn):
+    q, k, v = make_qkv(2, 4, 2, 700, 128, seed=4004)
+    r = v[:, :, :1, :].expand(-1, -1, 700, -1).contiguous()
+    for causal in (False, True):
+        o, _ = gpu_forward(attn, q, k, r, causal, 1 / math.sqrt(128))
+        ref = np.repeat(r.float().numpy()[:, :, :1, :].repeat(2, axis=1), 700, axis=2)
+        assert np.max(np.abs(o - ref)) <= TOL_O_MAX
+
+
+def test_causal_first_query_returns_v0(attn):
+    q, k, v = make_qkv(2, 4, 1, 384, 64, seed=4005)
+    o, lse = gpu_forward(attn, q, k, v, True, 0.125)
+    v0 = v.float().numpy()[:, 0, 0, :]
+    for h in range(4):
+        assert np.max(np.abs(o[:, h, 0, :] - v0)) <= TOL_O_MAX
+        lse0 = 0.125 * (q.double()[:, h, 0, :] * k.double()[:, 0, 0, :]).sum(-1).numpy()
+        assert np.max(np.abs(lse[:, h, 0] - lse0)) <= TOL_LSE
+
+
+def test_noncausal_kv_permutation_invariance(attn):
+    q, k, v = make_qkv(1, 2, 2, 512, 128, seed=4006)
+    perm = torch.randperm(512, generator=torch.Generator().manual_seed(1))
+    o1, l1 = gpu_forward(attn, q, k, v, False, 0.09)
+    o2, l2 = gpu_forward(attn, q, k[:, :, perm].contiguous(), v[:, :, perm].contiguous(), False, 0.09)
+    assert np.max(np.abs(o1 - o2)) <= TOL_O_MAX and np.max(np.abs(l1 - l2)) <= TOL_LSE
+
+
+# ------------------------------------------------------------------ robustness
+
+def test_every_output_written_and_guard_bands_untouched(attn):
+    B, Hq, Hkv, N, D = 2, 4, 2, 333, 128
+    q, k, v = (x.cuda() for x in make_qkv(B, Hq, Hkv, N, D, seed=4007))
+    guard = 4096
+    o_buf = torch.full((B * Hq * N * D + guard,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    l_buf = torch.full((B * Hq * N + guard,), float("nan"), dtype=torch.float32, device="cuda")
+    o = o_buf[: B * Hq * N * D].view(B, Hq, N, D)
+    lse = l_buf[: B * Hq * N].view(B, Hq, N)
+    attn.forward(q, k, v, causal=True, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    assert torch.isnan(o_buf[B * Hq * N * D:]).all() and torch.isnan(l_buf[B * Hq * N:]).all()
+
+
+def test_bitwise_deterministic(attn):
+    q, k, v = (x.cuda() for x in make_qkv(2, 8, 2, 1536, 128, seed=4008))
+    o1, l1 = attn.forward(q, k, v, causal=True)
+    o2, l2 = attn.forward(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_side_stream_and_host_path(attn):
+    q, k, v = make_qkv(1, 4, 4, 640, 64, seed=4009)
+    s = torch.cuda.Stream()
+    o_h, l_h = attn.forward_from_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), causal=True, stream=s)
+    o_ref, l_ref = attention_forward(q, k, v, True, 0.125)
+    assert_close(o_h.float().numpy().astype(np.float64), l_h.numpy().astype(np.float64), o_ref, l_ref, "host path")
+
+
+def test_misaligned_device_pointer_rejected(attn):
+    q, k, v = (x.cuda() for x in make_qkv(1, 1, 1, 128, 64, seed=4010))
+    o = torch.empty(1 * 128 * 64 + 8, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(128, dtype=torch.float32, device="cuda")
+    st = attn.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr() + 2, lse.data_ptr(),
+                       1, 1, 1, 128, 64, 0, 0.125, torch.cuda.current_stream().cuda_stream)
+    assert st == attn.ATTN_ERR_MISALIGNED

@@ -1,0 +1,179 @@
+"""bf16 attention forward on B200 (sm_100a): Python binding of the C ABI in include/attn.h.
+
+The binding only marshals arguments: every step of the computation runs in the
+CUDA kernel inside ``libattn_fwd.so``.  There is no CPU fallback; if the library
+cannot be loaded, importing this package raises.
+
+    import tiled_attention_forward_03_b200 as attn
+    o, lse = attn.forward(q, k, v, causal=True)        # q,k,v: CUDA bf16 [B, H, N, D]
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+from . import build as _build
+
+__all__ = [
+    "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED",
+    "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "AttnError", "lib", "lib_path", "attn_fwd",
+    "attn_status_string", "attn_last_cuda_error", "attn_device_status", "attn_num_units",
+    "attn_version", "forward", "forward_from_host", "device_status",
+]
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_MISALIGNED = 3
+ATTN_ERR_CUDA = 4
+ATTN_ERR_TIMEOUT = 5
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str = "attn_fwd"):
+        self.status = status
+        detail = attn_last_cuda_error() if status in (ATTN_ERR_CUDA,) else ""
+        super().__init__(f"{where} failed: {attn_status_string(status)}" + (f" ({detail})" if detail else ""))
+
+
+def _load() -> ctypes.CDLL:
+    path = _build.LIB_PATH
+    if not _build.up_to_date():
+        try:
+            _build.build()
+        except Exception as exc:  # no toolchain: only an existing library will do
+            if not os.path.exists(path):
+                raise ImportError(f"attention CUDA library missing and could not be built: {exc}") from exc
+    if not os.path.exists(path):
+        raise ImportError(f"attention CUDA library not found at {path}")
+    L = ctypes.CDLL(path)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+    L.attn_fwd.restype = i
+    L.attn_status_string.argtypes = [i]
+    L.attn_status_string.restype = ctypes.c_char_p
+    L.attn_last_cuda_error.argtypes = []
+    L.attn_last_cuda_error.restype = ctypes.c_char_p
+    L.attn_device_status.argtypes = [vp, ctypes.POINTER(i)]
+    L.attn_device_status.restype = i
+    L.attn_num_units.argtypes = [i, i, i]
+    L.attn_num_units.restype = ctypes.c_longlong
+    L.attn_version.argtypes = []
+    L.attn_version.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+lib_path = _build.LIB_PATH
+
+
+# ---------------------------------------------------------------- raw C calls
+
+def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, stream) -> int:
+    """Direct call of the C entry point; pointers and stream are integers (or None)."""
+    return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, D, int(bool(causal)), float(scale), stream)
+
+
+def attn_status_string(status: int) -> str:
+    return lib.attn_status_string(status).decode()
+
+
+def attn_last_cuda_error() -> str:
+    return lib.attn_last_cuda_error().decode()
+
+
+def attn_device_status(stream=None):
+    site = ctypes.c_int(0)
+    st = lib.attn_device_status(stream, ctypes.byref(site))
+    return st, site.value
+
+
+def attn_num_units(B: int, Hq: int, N: int) -> int:
+    return lib.attn_num_units(B, Hq, N)
+
+
+def attn_version() -> str:
+    return lib.attn_version().decode()
+
+
+# ---------------------------------------------------------------- torch conveniences
+
+def _check(t, name, dtype, shape):
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):
+    """Attention forward on CUDA bf16 tensors [B, H, N, D]; returns (o bf16, lse fp32 [B, Hq, N]).
+
+    Runs on ``stream`` (a torch.cuda.Stream) or torch's current stream.
+    """
+    import torch
+
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, N, D]")
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    _check(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _check(k, "k", torch.bfloat16, (B, Hkv, N, D))
+    _check(v, "v", torch.bfloat16, (B, Hkv, N, D))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, (B, Hq, N, D))
+    _check(lse, "lse", torch.float32, (B, Hq, N))
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                      B, Hq, Hkv, N, D, causal, scale, s.cuda_stream)
+    if st != ATTN_OK:
+        raise AttnError(st)
+    return out, lse
+
+
+def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None, device=None,
+                      out_host=None, lse_host=None, stream=None):
+    """End-to-end call on host (ideally pinned) bf16 tensors: copy in, attention, copy out.
+
+    Returns host tensors (o, lse).  The copies and the kernel are enqueued on one
+    stream; the call returns after the device-to-host copies have completed.
+    """
+    import torch
+
+    dev = torch.device(device if device is not None else "cuda")
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    with torch.cuda.stream(s):
+        qd = q.to(dev, non_blocking=True)
+        kd = k.to(dev, non_blocking=True)
+        vd = v.to(dev, non_blocking=True)
+        o, lse = forward(qd, kd, vd, causal=causal, scale=scale, stream=s)
+        if out_host is None:
+            out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        if lse_host is None:
+            lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        out_host.copy_(o, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+    s.synchronize()
+    return out_host, lse_host
+
+
+def device_status(stream=None):
+    """Synchronise and report whether a kernel wait gave up: (status, site)."""
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return attn_device_status(s.cuda_stream)

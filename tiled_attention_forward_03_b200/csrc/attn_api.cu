@@ -1,0 +1,223 @@
+// attn_api.cu -- host side of the C ABI declared in include/attn.h.
+//
+// Validates arguments before any CUDA call, encodes the TMA tensor maps for Q, K
+// and V, sizes the persistent grid to the SM count and launches the sm_100a kernel
+// on the caller's stream.  Nothing is allocated per call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_fwd_kernel.cuh"
+
+#define ATTN_VERSION_STRING "b200-attn 0.1 (sm_100a, tcgen05/TMA/TMEM)"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+thread_local char g_last_cuda_error[256] = "";
+
+void record_cuda_error(const char* what, cudaError_t e) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s (%d)", what, cudaGetErrorString(e),
+                (int)e);
+}
+
+void record_driver_error(const char* what, int code) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: CUresult %d", what, code);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* sym = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &sym, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(sym);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  std::once_flag once;
+  int num_sms = 0;
+  bool attrs_ok = false;
+  bool bad_regs = false;
+  cudaError_t err = cudaSuccess;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+// Per device: SM count and the kernels' dynamic shared memory opt-in.
+bool device_setup(int dev, int* num_sms) {
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  DeviceInfo& d = g_dev[dev];
+  std::call_once(d.once, [&d, dev] {
+    cudaError_t e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn::attn_fwd_sm100<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn::SmemPlan<64>::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn::attn_fwd_sm100<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn::SmemPlan<128>::kAlloc);
+    // The kernels' register split (setmaxnreg) assumes exactly kRegsAtLaunch registers
+    // per thread at launch; a build that differs would make the increase wait forever,
+    // so such a build refuses to launch.
+    cudaFuncAttributes fa64, fa128;
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa64, attn::attn_fwd_sm100<64>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa128, attn::attn_fwd_sm100<128>);
+    d.err = e;
+    d.attrs_ok = (e == cudaSuccess);
+    if (d.attrs_ok && (fa64.numRegs != attn::kRegsAtLaunch || fa128.numRegs != attn::kRegsAtLaunch)) {
+      d.attrs_ok = false;
+      d.err = cudaErrorInvalidDeviceFunction;
+      d.bad_regs = true;
+    }
+  });
+  if (!d.attrs_ok && d.bad_regs) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "kernel register count differs from the register split it was written for");
+    return false;
+  }
+  if (!d.attrs_ok) {
+    record_cuda_error("device setup", d.err);
+    return false;
+  }
+  *num_sms = d.num_sms;
+  return true;
+}
+
+// [heads, N, D] bf16 tensor viewed by TMA as 3-D (D fastest), boxes of 64 x 128 x 1
+// with 128-byte swizzle; rows past N read as zero.
+int encode_map(CUtensorMap* map, const void* base, long long heads, int N, int D) {
+  auto enc = tensor_map_encoder();
+  if (!enc) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled entry point unavailable");
+    return ATTN_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * (cuuint64_t)D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)attn::kBlockM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    record_driver_error("cuTensorMapEncodeTiled", (int)r);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_MISALIGNED: return "ATTN_ERR_MISALIGNED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    default: return "ATTN_ERR_UNKNOWN";
+  }
+}
+
+const char* attn_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* attn_version(void) { return ATTN_VERSION_STRING; }
+
+long long attn_num_units(int B, int Hq, int N) {
+  if (B < 0 || Hq < 1 || N < 0) return -1;
+  const long long pairs = ((long long)N + 2 * attn::kBlockM - 1) / (2 * attn::kBlockM);
+  return (long long)B * Hq * pairs;
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+             int D, int causal, float scale, void* stream) {
+  // ---- host-side validation (no CUDA call before this block passes)
+  if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
+    return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return ATTN_OK;  // empty problem: nothing to compute or write
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return ATTN_ERR_MISALIGNED;
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    record_cuda_error("cudaGetDevice", e);
+    return ATTN_ERR_CUDA;
+  }
+  int num_sms = 0;
+  if (!device_setup(dev, &num_sms)) return ATTN_ERR_CUDA;
+
+  CUtensorMap mq, mk, mv;
+  int st;
+  if ((st = encode_map(&mq, q, (long long)B * Hq, N, D)) != ATTN_OK) return st;
+  if ((st = encode_map(&mk, k, (long long)B * Hkv, N, D)) != ATTN_OK) return st;
+  if ((st = encode_map(&mv, v, (long long)B * Hkv, N, D)) != ATTN_OK) return st;
+
+  attn::FwdParams p;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.num_pairs = (int)(((long long)N + 2 * attn::kBlockM - 1) / (2 * attn::kBlockM));
+  p.num_blocks = (int)(((long long)N + attn::kBlockN - 1) / attn::kBlockN);
+  p.num_units = attn_num_units(B, Hq, N);
+  p.causal = causal ? 1 : 0;
+  p.c = std::fabs(scale) * 1.44269504088896340736f;
+  p.idesc_s = attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, scale < 0.f);
+  p.idesc_pv = attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
+
+  const long long grid = p.num_units < num_sms ? p.num_units : num_sms;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (D == 128) {
+    attn::attn_fwd_sm100<128><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128>::kAlloc, s>>>(mq, mk, mv, p);
+  } else {
+    attn::attn_fwd_sm100<64><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(mq, mk, mv, p);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    record_cuda_error("kernel launch", e);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+int attn_device_status(void* stream, int* site) {
+  if (site) *site = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    record_cuda_error("cudaStreamSynchronize", e);
+    return ATTN_ERR_CUDA;
+  }
+  unsigned int value = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&value, attn::g_attn_fault_site, sizeof(value));
+  if (e == cudaSuccess && value != 0) e = cudaMemcpyToSymbol(attn::g_attn_fault_site, &zero, sizeof(zero));
+  if (e != cudaSuccess) {
+    record_cuda_error("fault-site readback", e);
+    return ATTN_ERR_CUDA;
+  }
+  if (site) *site = (int)value;
+  return value ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,556 @@
+// attn_fwd_kernel.cuh -- tiled attention forward for B200 (sm_100a).
+//
+// Method: the tiled attention forward with an online (running max / running sum)
+// softmax whose hot loop is a score matmul, a base-2 exponential and row sums,
+// followed by the probability-times-V matmul ("Making AMD GPUs go brrr", section
+// "Real kernel example"; "HipKittens: fast and furious AMD kernels", section
+// "Performance results": causal and non-causal, several D and N).  The pages'
+// AMD schedule (two wave groups alternating memory and compute clusters) becomes,
+// on sm_100a, warp specialisation with two Q tiles ping-ponging on the tensor core:
+//
+//   warps 0-3  softmax warpgroup for Q tile 0 (one TMEM lane = one query row per thread)
+//   warps 4-7  softmax warpgroup for Q tile 1
+//   warp  8    TMA producer: Q tiles once per unit, K_j / V_j through a smem ring
+//   warp  9    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j on tcgen05
+//   warps 10-11 idle (they complete the third warpgroup, which gives up registers)
+//
+// A work unit is 256 query rows (two 128-row tiles) of one query head; a persistent
+// grid walks the units with a static stride.  Units of one head are adjacent (and
+// the heads of one GQA group are adjacent) so K/V blocks are re-read from L2; in the
+// causal case a head's units run heaviest first.
+//
+// Tensor memory (512 columns of 128 lanes x 32 bit):
+//   [  0,128) S_0 fp32 scores of tile 0; its first 64 columns are overwritten by P_0 (bf16x2)
+//   [128,256) S_1 / P_1
+//   [256,256+D) O_0 fp32 accumulator;  [384,384+D) O_1
+//
+// Online softmax in base 2 with c = |scale| * log2(e):  m = running max of s*c,
+// p = 2^(s*c - m), l = sum p.  The max is applied lazily: O and l are rescaled only
+// when a row's max grows by more than RESCALE_LOG2 (so p <= 2^RESCALE_LOG2); the final
+// O / l and LSE = (m + log2 l) * ln 2 use the same m, so the result is unchanged.
+//
+// Every mbarrier wait is bounded: on timeout the CTA records a site code in
+// g_attn_fault_site, all roles leave their loops, in-flight copies and MMAs are
+// drained (bounded again), TMEM is freed and the kernel returns.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+constexpr int kThreads = 384;  // three warpgroups
+// Register split (launch: 384 x 168): softmax warpgroups 2 x 128 x 200, the
+// producer/MMA warpgroup 128 x 104; 2*128*200 + 128*104 == 384*168.
+constexpr int kRegsAtLaunch = 168;
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsControl = 104;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsAtLaunch,
+              "register split exceeds the launch allocation");
+constexpr int kBlockM = 128;  // query rows per tile
+constexpr int kBlockN = 128;  // keys per KV block
+constexpr float kRescaleLog2 = 8.0f;
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s for any single wait
+
+// Fault-site codes written to g_attn_fault_site when a bounded wait gives up.
+enum : unsigned {
+  kSiteProducerQ = 1,
+  kSiteProducerKV = 2,
+  kSiteMmaQ = 3,
+  kSiteMmaKV = 4,
+  kSiteMmaP = 5,
+  kSiteMmaOFree = 6,
+  kSiteSoftmaxS = 7,
+  kSiteSoftmaxO = 8,
+  kSiteDrain = 9,
+};
+
+__device__ unsigned int g_attn_fault_site = 0;
+
+template <int D>
+struct SmemPlan {
+  static constexpr int kTileBytes = kBlockM * D * 2;       // one 128-row bf16 tile
+  static constexpr int kChunks = D / 64;                    // 64-column (128 B) swizzle chunks per row
+  static constexpr int kChunkBytes = kBlockM * 128;         // one chunk of a tile: 16 KB
+  static constexpr int kStages = (D == 128) ? 4 : 8;        // K/V ring depth
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] o_free[2] drain
+  static constexpr int kNumBars = 4 + 2 * kStages + 8 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base (u32), abort flag (u32)
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;              // slack for 1024-byte alignment
+};
+
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int Hq, Hkv, N;
+  int group;         // Hq / Hkv
+  int num_pairs;     // ceil(N / 256): units per head
+  int num_blocks;    // ceil(N / 128): KV blocks per head
+  long long num_units;
+  int causal;
+  float c;           // |scale| * log2(e)
+  uint32_t idesc_s;  // S = Q K^T instruction descriptor (negates A when scale < 0)
+  uint32_t idesc_pv; // O += P V instruction descriptor
+};
+
+struct Unit {
+  int q0;          // first query row of tile 0
+  int head_q;      // b * Hq + hq
+  int head_kv;     // b * Hkv + hq / group
+  int n0, n1;      // KV blocks visited by tile 0 / tile 1
+  bool valid1;     // tile 1 holds at least one row < N
+  int nmax;
+};
+
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, long long u) {
+  Unit w;
+  const long long head = u / p.num_pairs;
+  int pair = (int)(u - head * p.num_pairs);
+  if (p.causal) pair = p.num_pairs - 1 - pair;  // heaviest units of a head first
+  const int hq = (int)(head % p.Hq);
+  const int b = (int)(head / p.Hq);
+  w.q0 = pair * 2 * kBlockM;
+  w.head_q = (int)head;
+  w.head_kv = b * p.Hkv + hq / p.group;
+  w.valid1 = (w.q0 + kBlockM) < p.N;
+  if (p.causal) {
+    w.n0 = min(p.num_blocks, 2 * pair + 1);
+    w.n1 = min(p.num_blocks, 2 * pair + 2);
+  } else {
+    w.n0 = p.num_blocks;
+    w.n1 = p.num_blocks;
+  }
+  w.nmax = w.valid1 ? w.n1 : w.n0;
+  return w;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false (and raises the CTA abort flag,
+// recording `site` once per launch) if the phase did not complete in time, or if
+// another role of the CTA has already aborted.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                           unsigned site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      *abort_flag = 1u;
+      atomicCAS(&g_attn_fault_site, 0u, site);
+      return false;
+    }
+  }
+}
+
+// Bounded wait used when draining in-flight copies/MMAs before exit: it does not stop
+// early on the abort flag, only on its own time limit.
+__device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      *abort_flag = 1u;
+      atomicCAS(&g_attn_fault_site, 0u, (unsigned)kSiteDrain);
+      return;
+    }
+  }
+}
+
+// Ring position: stage index and the parity of its current fill.
+struct Ring {
+  uint32_t stage = 0, phase = 0;
+  template <int S>
+  __device__ __forceinline__ void advance() {
+    if (++stage == S) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_sm100(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                   const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
+  using Plan = SmemPlan<D>;
+  constexpr int S = Plan::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte swizzled TMA tiles and UMMA descriptors need 1024-byte aligned tiles.
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+
+  uint8_t* sQ = smem + Plan::kQOff;
+  uint8_t* sKV = smem + Plan::kKVOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 2;
+  uint64_t* kv_full = bars + 4;
+  uint64_t* kv_empty = bars + 4 + S;
+  uint64_t* s_full = bars + 4 + 2 * S;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = s_full + 4;
+  uint64_t* o_free = s_full + 6;
+  uint64_t* drain = s_full + 8;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Plan::kMiscOff);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Plan::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kBlockM);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_free[i], kBlockM);
+    }
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    regs_decrease<kRegsControl>();
+    if (lane == 0) {
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const uint64_t pol_q = l2_policy_evict_first();
+      Ring ring;
+      uint32_t q_par[2] = {1u, 1u};     // empty-barrier waits start on the completed "previous" phase
+      uint32_t filled = 0u, fill_par = 0u;  // per stage: ever filled / parity of its last fill
+      bool q_filled[2] = {false, false};
+      uint32_t q_fill_par[2] = {0u, 0u};
+
+      auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int row, int head,
+                           uint64_t pol) {
+#pragma unroll
+        for (int ch = 0; ch < Plan::kChunks; ++ch)
+          tma_load_3d(dst + ch * Plan::kChunkBytes, map, bar, ch * 64, row, head, pol);
+      };
+      auto load_kv = [&](const CUtensorMap* map, int row, int head) -> bool {
+        if (!wait_phase(&kv_empty[ring.stage], ring.phase ^ 1u, abort_flag, kSiteProducerKV)) return false;
+        mbar_arrive_expect_tx(&kv_full[ring.stage], Plan::kTileBytes);
+        load_tile(map, sKV + ring.stage * Plan::kTileBytes, &kv_full[ring.stage], row, head, pol_kv);
+        filled |= 1u << ring.stage;
+        fill_par = (fill_par & ~(1u << ring.stage)) | (ring.phase << ring.stage);
+        ring.advance<S>();
+        return true;
+      };
+      auto load_q = [&](int t, int row, int head) -> bool {
+        if (!wait_phase(&q_empty[t], q_par[t], abort_flag, kSiteProducerQ)) return false;
+        q_par[t] ^= 1u;
+        mbar_arrive_expect_tx(&q_full[t], Plan::kTileBytes);
+        load_tile(&tmap_q, sQ + t * Plan::kTileBytes, &q_full[t], row, head, pol_q);
+        q_fill_par[t] = q_filled[t] ? (q_fill_par[t] ^ 1u) : 0u;
+        q_filled[t] = true;
+        return true;
+      };
+
+      for (long long u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+        const Unit w = decode_unit(p, u);
+        if (!load_q(0, w.q0, w.head_q)) break;
+        if (!load_kv(&tmap_k, 0, w.head_kv)) break;
+        if (w.valid1 && !load_q(1, w.q0 + kBlockM, w.head_q)) break;
+        if (!load_kv(&tmap_v, 0, w.head_kv)) break;
+        bool ok = true;
+        for (int j = 1; j < w.nmax && ok; ++j) {
+          ok = load_kv(&tmap_k, j * kBlockN, w.head_kv) && load_kv(&tmap_v, j * kBlockN, w.head_kv);
+        }
+        if (!ok) break;
+      }
+      // Drain: every issued copy must have landed before the CTA may exit.
+      for (int s = 0; s < S; ++s)
+        if (filled & (1u << s)) drain_phase(&kv_full[s], (fill_par >> s) & 1u, abort_flag);
+      for (int t = 0; t < 2; ++t)
+        if (q_filled[t]) drain_phase(&q_full[t], q_fill_par[t], abort_flag);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    regs_decrease<kRegsControl>();
+    if (lane == 0) {
+      Ring ring;
+      uint32_t q_par[2] = {0u, 0u}, pf_par[2] = {0u, 0u}, of_par[2] = {1u, 1u};
+      const uint32_t sQ_addr = smem_u32(sQ);
+      const uint32_t sKV_addr = smem_u32(sKV);
+
+      // S_t = Q_t K^T over D in steps of 16 (K-major A and B, 128-byte swizzle).
+      auto issue_s = [&](int t, uint32_t stage) {
+        const uint32_t qa = sQ_addr + t * Plan::kTileBytes;
+        const uint32_t ka = sKV_addr + stage * Plan::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
+          mma_ss(tmem_base + t * 128, smem_desc_kmajor_sw128(qa + off), smem_desc_kmajor_sw128(ka + off),
+                 p.idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t += P_t V over the 128 keys in steps of 16 (P from TMEM, V MN-major in smem).
+      auto issue_pv = [&](int t, uint32_t stage, bool accumulate) {
+        const uint32_t va = sKV_addr + stage * Plan::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          mma_ts(tmem_base + 256 + t * 128, tmem_base + t * 128 + kk * 8,
+                 smem_desc_mnmajor_sw128(va + kk * 2048, Plan::kChunkBytes), p.idesc_pv,
+                 (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = true;
+      for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(p, u);
+        const int n[2] = {w.n0, w.n1};
+        const bool valid[2] = {true, w.valid1};
+
+        // Block 0 scores for both tiles.
+        if (!(ok = wait_phase(&q_full[0], q_par[0], abort_flag, kSiteMmaQ))) break;
+        q_par[0] ^= 1u;
+        const uint32_t k0_stage = ring.stage;
+        if (!(ok = wait_phase(&kv_full[k0_stage], ring.phase, abort_flag, kSiteMmaKV))) break;
+        ring.advance<S>();
+        tc_fence_after();
+        issue_s(0, k0_stage);
+        tc_commit(&s_full[0]);
+        if (n[0] == 1) tc_commit(&q_empty[0]);
+        if (valid[1]) {
+          if (!(ok = wait_phase(&q_full[1], q_par[1], abort_flag, kSiteMmaQ))) break;
+          q_par[1] ^= 1u;
+          tc_fence_after();
+          issue_s(1, k0_stage);
+          tc_commit(&s_full[1]);
+          if (n[1] == 1) tc_commit(&q_empty[1]);
+        }
+        tc_commit(&kv_empty[k0_stage]);
+
+        for (int j = 0; j < w.nmax && ok; ++j) {
+          const uint32_t v_stage = ring.stage;
+          if (!(ok = wait_phase(&kv_full[v_stage], ring.phase, abort_flag, kSiteMmaKV))) break;
+          ring.advance<S>();
+          const bool has_next = (j + 1) < w.nmax;
+          const uint32_t kn_stage = ring.stage, kn_phase = ring.phase;
+          bool kn_ready = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!valid[t] || j >= n[t]) continue;
+            if (!(ok = wait_phase(&p_full[t], pf_par[t], abort_flag, kSiteMmaP))) break;
+            pf_par[t] ^= 1u;
+            if (j == 0) {
+              if (!(ok = wait_phase(&o_free[t], of_par[t], abort_flag, kSiteMmaOFree))) break;
+              of_par[t] ^= 1u;
+            }
+            tc_fence_after();
+            issue_pv(t, v_stage, j > 0);
+            if (j == n[t] - 1) tc_commit(&o_full[t]);
+            if (j + 1 < n[t]) {
+              if (!kn_ready) {
+                if (!(ok = wait_phase(&kv_full[kn_stage], kn_phase, abort_flag, kSiteMmaKV))) break;
+                kn_ready = true;
+                tc_fence_after();
+              }
+              issue_s(t, kn_stage);
+              tc_commit(&s_full[t]);
+              if (j + 2 == n[t]) tc_commit(&q_empty[t]);
+            }
+          }
+          if (!ok) break;
+          tc_commit(&kv_empty[v_stage]);
+          if (has_next) {
+            tc_commit(&kv_empty[kn_stage]);
+            ring.advance<S>();
+          }
+        }
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is released.
+      tc_commit(drain);
+      drain_phase(drain, 0u, abort_flag);
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax warpgroups
+    regs_increase<kRegsSoftmax>();
+    const int t = warp >> 2;                       // Q tile of this warpgroup
+    const int r = threadIdx.x & 127;               // row within the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem_base + lane_off + t * 128;
+    const uint32_t t_o = tmem_base + lane_off + 256 + t * 128;
+    const float c = p.c;
+    uint32_t s_par = 0u, o_par = 0u;
+    bool ok = true;
+
+    for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      const Unit w = decode_unit(p, u);
+      if (t == 1 && !w.valid1) continue;
+      const int n = t ? w.n1 : w.n0;
+      const int row = w.q0 + t * kBlockM + r;
+      const int key_lim = p.causal ? min(row, p.N - 1) : (p.N - 1);
+      float m = -INFINITY, l = 0.f;
+
+      for (int j = 0; j < n; ++j) {
+        if (!(ok = wait_phase(&s_full[t], s_par, abort_flag, kSiteSoftmaxS))) break;
+        s_par ^= 1u;
+        tc_fence_after();
+        float s[kBlockN];
+        {
+          uint32_t a0[32], a1[32], a2[32], a3[32];
+          tmem_ld32(t_s + 0, a0);
+          tmem_ld32(t_s + 32, a1);
+          tmem_ld32(t_s + 64, a2);
+          tmem_ld32(t_s + 96, a3);
+          tmem_ld_wait();
+          reg_fence32(a0);
+          reg_fence32(a1);
+          reg_fence32(a2);
+          reg_fence32(a3);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            s[i] = __uint_as_float(a0[i]);
+            s[32 + i] = __uint_as_float(a1[i]);
+            s[64 + i] = __uint_as_float(a2[i]);
+            s[96 + i] = __uint_as_float(a3[i]);
+          }
+        }
+        const int k0 = j * kBlockN;
+        const bool masked = (k0 + kBlockN - 1) > key_lim;
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < kBlockN; ++i)
+            if (k0 + i > key_lim) s[i] = -INFINITY;
+        }
+        float mx[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+        for (int i = 8; i < kBlockN; i += 8) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[i + e]);
+        }
+        const float rowmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float m_new = fmaxf(m, rowmax * c);
+        // Lazy correction: adopt a new max only when it grew by more than kRescaleLog2.
+        float alpha = 1.f;
+        bool any_rescale = false;
+        if (j == 0) {
+          m = m_new;
+        } else {
+          const bool need = m_new > m + kRescaleLog2;
+          any_rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = ex2_approx(m - m_new);
+            l *= alpha;
+            m = m_new;
+          }
+        }
+        const float neg_m = -m;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        // P = 2^(s*c - m) in two halves of 64 keys; each half is packed to bf16 pairs and
+        // written over the (already loaded) score columns it came from.
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+          if (masked) {
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) {
+              const int col = half * 64 + i;
+              const float p0 = (k0 + col > key_lim) ? 0.f : ex2_approx(fmaf(s[col], c, neg_m));
+              const float p1 = (k0 + col + 1 > key_lim) ? 0.f : ex2_approx(fmaf(s[col + 1], c, neg_m));
+              acc[(i >> 1) & 3] += p0 + p1;
+              pk[i >> 1] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) {
+              const int col = half * 64 + i;
+              const float p0 = ex2_approx(fmaf(s[col], c, neg_m));
+              const float p1 = ex2_approx(fmaf(s[col + 1], c, neg_m));
+              acc[(i >> 1) & 3] += p0 + p1;
+              pk[i >> 1] = pack_bf16x2(p0, p1);
+            }
+          }
+          tmem_st32(t_s + half * 32, pk);
+        }
+        l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        if (any_rescale) {
+          // O_t holds blocks < j (their MMAs completed before S_t(j) was signalled) and
+          // P_t(j) V has not been issued yet, so the accumulator can be rescaled here.
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32(t_o + ch * 32, ov);
+            tmem_ld_wait();
+            reg_fence32(ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(t_o + ch * 32, ov);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+      if (!ok) break;
+
+      // Epilogue: O = O_acc / l -> bf16, LSE = (m + log2 l) ln 2.
+      if (!(ok = wait_phase(&o_full[t], o_par, abort_flag, kSiteSoftmaxO))) break;
+      o_par ^= 1u;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool row_ok = row < p.N;
+      __nv_bfloat16* orow = p.o + ((size_t)w.head_q * p.N + (row_ok ? row : 0)) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t ov[32];
+        tmem_ld32(t_o + ch * 32, ov);
+        tmem_ld_wait();
+        reg_fence32(ov);
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          packed[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&o_free[t]);
+      if (row_ok) p.lse[(size_t)w.head_q * p.N + row] = (m + log2f(l)) * 0.69314718055994530942f;
+    }
+  } else {
+    regs_decrease<kRegsControl>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace attn
