@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 bf16 attention forward (TFLOP/s, % of the dense BF16 peak).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all] [--impl ours|reference]
+
+One step = one attention forward pass over the workload's batch (one kernel
+launch).  Default workload: B=4, Hq=Hkv=16, N=2048, D=128, non-causal, bf16
+inputs drawn i.i.d. N(0,1) from a seeded CPU generator.  Its inputs (100 MB)
+fit in the 126 MB L2, so a 512 MB buffer is written between timed steps to
+flush L2; each step's kernel is timed with CUDA events on its launching stream.
+
+FLOPs counted: 4*B*Hq*N^2*D, halved for causal.  `value` is the whole-job
+throughput (all ranks' FLOPs / the slowest rank's time).  With N>1 GPUs
+(torchrun), every rank runs its own batch of the workload (weak scaling): the
+query heads are independent, so no collective touches the data path; NCCL only
+carries the barrier and the max-over-ranks timing.
+
+`--impl reference` times the fp64 CPU oracle instead (the only other
+implementation of this path): each step is a bounded sample of the workload's
+heads on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DATASHEET_BF16_TFLOPS = 2250.0   # B200 dense BF16 (no sparsity)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+DEFAULT_WORKLOAD = "cfg2"
+METRIC = "attention fwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
+L2_FLUSH_BYTES = 512 << 20
+CPU_SAMPLE_SECONDS = 12.0
+
+
+# ------------------------------------------------------------------ distributed helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Largest value of x over all ranks (x itself on one rank)."""
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        import torch
+
+        t = torch.zeros(1, device=device)
+        dist.all_reduce(t)
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch of the workload."""
+    return seed + 7919 * rank
+
+
+# ------------------------------------------------------------------ peaks and clocks
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), \
+            float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, 1400.0, FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples of one GPU while a region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.proc = None
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        busy = [r for r in rows if (num(r[4]) or 0) > 50] or rows
+        sm = [num(r[1]) for r in busy if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i in range(4) if r[6 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(num(r[2]) or 0 for r in rows),
+                "reasons": reasons, "samples": len(busy),
+                "power_w_max": max(num(r[3]) or 0 for r in rows)}
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+def profile_traffic(workload_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload_name}_dram.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    from tiled_attention_forward_03_b200.build import kernel_source_digest
+
+    if d.get("kernel_source_sha256") != kernel_source_digest():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        import numpy  # noqa: F401
+
+        info = threadpool_info()
+        if info:
+            return max(int(x.get("num_threads", 1)) for x in info)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def time_oracle(w, seconds: float, heads: int | None = None):
+    """Run the fp64 oracle on whole heads of workload w for about `seconds` (or `heads` heads).
+
+    Returns (TFLOP/s, FLOPs done, seconds, heads done, sample description)."""
+    from oracle import head_forward
+    from tiled_attention_forward_03_b200.synth import make_qkv
+
+    q, k, v = make_qkv(1, w.Hq, w.Hkv, w.N, w.D, w.seed)  # one batch row holds all heads
+    g = w.Hq // w.Hkv
+    per_head = w.flops / (w.B * w.Hq)
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        h = done % w.Hq
+        head_forward(q[0, h], k[0, h // g], v[0, h // g], w.causal, w.softmax_scale)
+        done += 1
+        el = time.perf_counter() - t0
+        if heads is not None and done >= heads:
+            break
+        if heads is None and el >= seconds:
+            break
+    tflops = per_head * done / el / 1e12
+    sample = (f"{done} of {w.B * w.Hq} heads of {w.name} (each head's full {w.N}x{w.N} fp64 score matrix), "
+              f"{el:.1f} s")
+    return tflops, per_head * done, el, done, sample
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, w):
+    import torch
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+
+    import tiled_attention_forward_03_b200 as attn
+    from tiled_attention_forward_03_b200.synth import make_qkv
+
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.D, rank_seed(w.seed, rank))
+    qd, kd, vd = (x.to(device) for x in (q, k, v))
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    scale = w.softmax_scale
+
+    def step():
+        attn.forward(qd, kd, vd, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    st, site = attn.device_status()
+    if st != attn.ATTN_OK:
+        raise RuntimeError(f"kernel wait gave up during warm-up (site {site})")
+
+    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # keep the GPU busy long enough for the clock sampler to see the timed region
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    for i in range(args.steps):
+        flush.zero_()                       # L2 flush between timed steps (not timed)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    clk = clocks.stop() if clocks else None
+    kernel_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    local_ms = sum(kernel_ms)
+    total_ms = max_over_ranks(local_ms, dist, device)
+    st, site = attn.device_status()
+    if st != attn.ATTN_OK:
+        raise RuntimeError(f"kernel wait gave up during timing (site {site})")
+
+    # ---- end to end through the public host-buffer call
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        attn.forward_from_host(qh, kh, vh, causal=w.causal, scale=scale, device=device, out_host=oh,
+                               lse_host=lh, stream=stream)
+    barrier(dist, device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        attn.forward_from_host(qh, kh, vh, causal=w.causal, scale=scale, device=device, out_host=oh,
+                               lse_host=lh, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+    barrier(dist, device)
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return None
+
+    peak_burst, peak_sustained, hbm, peak_kind = measured_peaks()
+    flops_step = w.flops
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    achieved = flops_step / (statistics.mean(kernel_ms) * 1e-3) / 1e12
+    e2e_value = world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+    traffic = profile_traffic(w.name)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {**w.describe(), "l2": "flushed between timed steps (512 MB write)",
+                   "parallelism": f"replicas{world}: each rank its own batch, no collective on the data path"},
+        "pct_of_dense_bf16_peak": round(100.0 * value / world / DATASHEET_BF16_TFLOPS, 2),
+        "pct_of_measured_bf16_peak": round(100.0 * value / world / peak_burst, 2),
+        "hbm_gbs_algorithmic": round(w.algorithmic_bytes / (statistics.mean(kernel_ms) * 1e-3) / 1e9, 1),
+        "clocks": clk,
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "path": "forward_from_host: pinned host q,k,v -> device, attn_fwd, o,lse -> pinned host"},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_burst,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak_burst, 4), "traffic": traffic,
+                     "peak_kind": f"{peak_kind} bf16 matmul, burst (kernel timed alone)",
+                     "kernel": f"attn_fwd_sm100<{w.D}>"},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        tf, _, el, done, sample = time_oracle(w, CPU_SAMPLE_SECONDS)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                                "sample": sample}
+    if dist is not None:
+        dist.destroy_process_group()
+    return line
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        tf, flops, el, done, sample = time_oracle(w, 0.0, heads=1)
+        if i >= args.warmup:
+            per_step.append((flops, el))
+    flops = sum(f for f, _ in per_step)
+    secs = sum(e for _, e in per_step)
+    value = flops / secs / 1e12
+    cores = cpu_threads()
+    sample = f"one head of {w.name} per step (full {w.N}x{w.N} fp64 score matrix), {args.steps} steps"
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": w.describe(),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="cfg1..cfg4, a sweep point name (e.g. sweep_D128_N8192_causal), or 'all'")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from tiled_attention_forward_03_b200.synth import WORKLOADS, get_workload
+
+    names = list(WORKLOADS) if args.workload == "all" else [args.workload]
+    for i, name in enumerate(names):
+        w = get_workload(name)
+        if args.impl == "reference":
+            line = run_reference(args, w)
+        else:
+            if i > 0:
+                args.no_cpu_baseline = True
+            line = run_ours(args, w)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

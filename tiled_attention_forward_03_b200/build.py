@@ -78,6 +78,18 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB_PATH
 
 
+
+def kernel_source_digest() -> str:
+    """SHA-256 over the CUDA sources and headers (identifies the kernel an ncu capture measured)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in SOURCES + HEADERS:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
 if __name__ == "__main__":
     path = build(force="--force" in sys.argv, verbose=True)
     print(path)
