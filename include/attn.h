@@ -107,6 +107,26 @@ long long attn_num_units(int B, int Hq, int N);
 /* Version string of the library build (static). */
 const char* attn_version(void);
 
+/* ---- self-test entry points (used by the library's tests; no part of the forward pass) ---- */
+
+/*
+ * attn_selftest_exp2_poly -- evaluate, on the device, the polynomial 2^x that the
+ * softmax uses for part of its exponentials (round-to-nearest range reduction,
+ * degree-3 minimax polynomial on [-1/2, 1/2], exponent-field scaling; inputs below
+ * -125 are clamped).  x, y: device fp32 arrays of n elements (y written).  Enqueued
+ * on `stream`.  Returns ATTN_ERR_INVALID_ARG for n < 0 or null pointers with n > 0.
+ */
+int attn_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
+
+/*
+ * attn_selftest_wait_timeout -- launch a one-CTA kernel whose bounded mbarrier wait
+ * can never complete, with a limit of `timeout_us` microseconds (1..1000000).  The
+ * wait gives up, records its site and the kernel returns normally; a following
+ * attn_device_status() reports ATTN_ERR_TIMEOUT.  Used to test the failure path of
+ * the forward kernel's bounded waits without faulting or hanging the GPU.
+ */
+int attn_selftest_wait_timeout(unsigned int timeout_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

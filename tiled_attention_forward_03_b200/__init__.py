@@ -19,7 +19,8 @@ __all__ = [
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED",
     "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "AttnError", "lib", "lib_path", "attn_fwd",
     "attn_status_string", "attn_last_cuda_error", "attn_device_status", "attn_num_units",
-    "attn_version", "forward", "forward_from_host", "device_status",
+    "attn_version", "attn_selftest_exp2_poly", "attn_selftest_wait_timeout", "forward",
+    "forward_from_host", "device_status",
 ]
 
 ATTN_OK = 0
@@ -40,11 +41,15 @@ class AttnError(RuntimeError):
 def _load() -> ctypes.CDLL:
     path = _build.LIB_PATH
     if not _build.up_to_date():
-        try:
-            _build.build()
-        except Exception as exc:  # no toolchain: only an existing library will do
-            if not os.path.exists(path):
-                raise ImportError(f"attention CUDA library missing and could not be built: {exc}") from exc
+        # Sources newer than the library (or no library): rebuild.  A failed build is an
+        # error; only a machine without nvcc may use an existing library as shipped.
+        if _build.have_nvcc():
+            try:
+                _build.build()
+            except Exception as exc:
+                raise ImportError(f"building the attention CUDA library failed: {exc}") from exc
+        elif not os.path.exists(path):
+            raise ImportError(f"attention CUDA library not found at {path} and nvcc is unavailable")
     if not os.path.exists(path):
         raise ImportError(f"attention CUDA library not found at {path}")
     L = ctypes.CDLL(path)
@@ -61,6 +66,10 @@ def _load() -> ctypes.CDLL:
     L.attn_num_units.restype = ctypes.c_longlong
     L.attn_version.argtypes = []
     L.attn_version.restype = ctypes.c_char_p
+    L.attn_selftest_exp2_poly.argtypes = [vp, vp, i, vp]
+    L.attn_selftest_exp2_poly.restype = i
+    L.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    L.attn_selftest_wait_timeout.restype = i
     return L
 
 
@@ -95,6 +104,14 @@ def attn_num_units(B: int, Hq: int, N: int) -> int:
 
 def attn_version() -> str:
     return lib.attn_version().decode()
+
+
+def attn_selftest_exp2_poly(x_ptr, y_ptr, n: int, stream) -> int:
+    return lib.attn_selftest_exp2_poly(x_ptr, y_ptr, n, stream)
+
+
+def attn_selftest_wait_timeout(timeout_us: int, stream) -> int:
+    return lib.attn_selftest_wait_timeout(timeout_us, stream)
 
 
 # ---------------------------------------------------------------- torch conveniences

@@ -41,6 +41,14 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found: the CUDA toolkit is required to build the attention library")
 
 
+def have_nvcc() -> bool:
+    try:
+        _nvcc()
+        return True
+    except RuntimeError:
+        return False
+
+
 def _inputs() -> list[str]:
     files = [os.path.join(CSRC, s) for s in SOURCES + HEADERS]
     files.append(os.path.join(INCLUDE, "attn.h"))
@@ -66,9 +74,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
     log = proc.stdout + proc.stderr
     if proc.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + log)
-    regs = [int(x) for x in re.findall(r"Used (\d+) registers", log)]
-    spills = [int(x) for x in re.findall(r"(\d+) bytes spill stores", log)]
-    if not regs or any(r != EXPECTED_REGS for r in regs):
+    # register count of each forward-kernel instance (the self-test kernels are exempt)
+    regs, spills, current = [], [], None
+    for line in log.splitlines():
+        m = re.search(r"Compiling entry function '(\w+)'", line)
+        if m:
+            current = m.group(1)
+        m = re.search(r"Used (\d+) registers", line)
+        if m and current and "attn_fwd_sm100" in current:
+            regs.append(int(m.group(1)))
+        m = re.search(r"(\d+) bytes spill stores", line)
+        if m and current and "attn_fwd_sm100" in current:
+            spills.append(int(m.group(1)))
+    if len(regs) != 2 or any(r != EXPECTED_REGS for r in regs):
         os.remove(tmp)
         raise RuntimeError(f"unexpected kernel register counts {regs} (want {EXPECTED_REGS}):\n{log}")
     if verbose:

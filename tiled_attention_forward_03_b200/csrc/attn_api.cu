@@ -182,11 +182,13 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.num_blocks = (int)(((long long)N + attn::kBlockN - 1) / attn::kBlockN);
   p.num_units = attn_num_units(B, Hq, N);
   p.causal = causal ? 1 : 0;
+  p.units_per_step = p.causal ? 2 : 1;
+  p.num_steps = p.causal ? (long long)B * Hq * ((p.num_pairs + 1) / 2) : p.num_units;
   p.c = std::fabs(scale) * 1.44269504088896340736f;
   p.idesc_s = attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, scale < 0.f);
   p.idesc_pv = attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
 
-  const long long grid = p.num_units < num_sms ? p.num_units : num_sms;
+  const long long grid = p.num_steps < num_sms ? p.num_steps : num_sms;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (D == 128) {
     attn::attn_fwd_sm100<128><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128>::kAlloc, s>>>(mq, mk, mv, p);
@@ -218,6 +220,34 @@ int attn_device_status(void* stream, int* site) {
   }
   if (site) *site = (int)value;
   return value ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+int attn_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  if (!x || !y) return ATTN_ERR_INVALID_ARG;
+  const int pairs = (n + 1) / 2;
+  const int threads = 256;
+  attn::selftest_exp2_poly<<<(pairs + threads - 1) / threads, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      x, y, n);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    record_cuda_error("selftest_exp2_poly launch", e);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+int attn_selftest_wait_timeout(unsigned int timeout_us, void* stream) {
+  if (timeout_us == 0 || timeout_us > 1000000u) return ATTN_ERR_INVALID_ARG;
+  attn::selftest_wait_timeout<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)timeout_us * 1000ull);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    record_cuda_error("selftest_wait_timeout launch", e);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 
 }  // extern "C"

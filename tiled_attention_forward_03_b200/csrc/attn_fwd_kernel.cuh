@@ -11,7 +11,7 @@
 //   warps 0-3  softmax warpgroup for Q tile 0 (one TMEM lane = one query row per thread)
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp  8    TMA producer: Q tiles once per unit, K_j / V_j through a smem ring
-//   warp  9    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j on tcgen05
+//   warp  9    MMA issuer (one elected lane): S_t = Q_t K_j^T and O_t += P_t V_j on tcgen05
 //   warps 10-11 idle (they complete the third warpgroup, which gives up registers)
 //
 // A work unit is 256 query rows (two 128-row tiles) of one query head; a persistent
@@ -51,6 +51,11 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsAtL
 constexpr int kBlockM = 128;  // query rows per tile
 constexpr int kBlockN = 128;  // keys per KV block
 constexpr float kRescaleLog2 = 8.0f;
+// Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial instead of the
+// special-function unit; measured best on B200: 2 at D=128, 1 at D=64 (more polynomial work
+// costs issue slots that the MMA-issuing warp shares with the softmax warps).
+template <int D>
+__host__ __device__ constexpr int poly_pairs_per8() { return D == 128 ? 2 : 1; }
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s for any single wait
 
 // Fault-site codes written to g_attn_fault_site when a bounded wait gives up.
@@ -64,6 +69,7 @@ enum : unsigned {
   kSiteSoftmaxS = 7,
   kSiteSoftmaxO = 8,
   kSiteDrain = 9,
+  kSiteSelfTest = 10,
 };
 
 __device__ unsigned int g_attn_fault_site = 0;
@@ -92,6 +98,8 @@ struct FwdParams {
   int num_pairs;     // ceil(N / 256): units per head
   int num_blocks;    // ceil(N / 128): KV blocks per head
   long long num_units;
+  long long num_steps;  // scheduling steps walked by the persistent grid
+  int units_per_step;   // 1 (non-causal) or 2 (causal: heaviest + lightest pair of a head)
   int causal;
   float c;           // |scale| * log2(e)
   uint32_t idesc_s;  // S = Q K^T instruction descriptor (negates A when scale < 0)
@@ -107,11 +115,8 @@ struct Unit {
   int nmax;
 };
 
-__device__ __forceinline__ Unit decode_unit(const FwdParams& p, long long u) {
+__device__ __forceinline__ Unit make_unit(const FwdParams& p, long long head, int pair) {
   Unit w;
-  const long long head = u / p.num_pairs;
-  int pair = (int)(u - head * p.num_pairs);
-  if (p.causal) pair = p.num_pairs - 1 - pair;  // heaviest units of a head first
   const int hq = (int)(head % p.Hq);
   const int b = (int)(head / p.Hq);
   w.q0 = pair * 2 * kBlockM;
@@ -129,17 +134,39 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, long long u) {
   return w;
 }
 
+// Unit `part` of scheduling step `step`.  Non-causal: one unit per step, the pairs of
+// a head in order.  Causal: the work of pair j grows linearly with j, so step s of a
+// head holds its pair P-1-s (heaviest first) and pair s; every step then costs the
+// same and a static stride over steps balances the grid.  Consecutive steps stay in
+// one head (and the heads of one GQA group are consecutive), so K/V tiles are shared
+// through L2 by the CTAs running at the same time.  Returns false if the step has no
+// such unit (the middle pair of a head with an odd pair count).
+__device__ __forceinline__ bool unit_at(const FwdParams& p, long long step, int part, Unit& w) {
+  if (!p.causal) {
+    const long long head = step / p.num_pairs;
+    w = make_unit(p, head, (int)(step - head * p.num_pairs));
+    return true;
+  }
+  const int steps_per_head = (p.num_pairs + 1) / 2;
+  const long long head = step / steps_per_head;
+  const int s = (int)(step - head * steps_per_head);
+  const int pair = part == 0 ? p.num_pairs - 1 - s : s;
+  if (part == 1 && pair == p.num_pairs - 1 - s) return false;
+  w = make_unit(p, head, pair);
+  return true;
+}
+
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA abort flag,
-// recording `site` once per launch) if the phase did not complete in time, or if
-// another role of the CTA has already aborted.
+// recording `site` once per launch) if the phase did not complete within `timeout_ns`,
+// or if another role of the CTA has already aborted.
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                           unsigned site) {
+                                           unsigned site, uint64_t timeout_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > timeout_ns) {
       *abort_flag = 1u;
       atomicCAS(&g_attn_fault_site, 0u, site);
       return false;
@@ -270,17 +297,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
-      for (long long u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-        const Unit w = decode_unit(p, u);
-        if (!load_q(0, w.q0, w.head_q)) break;
-        if (!load_kv(&tmap_k, 0, w.head_kv)) break;
-        if (w.valid1 && !load_q(1, w.q0 + kBlockM, w.head_q)) break;
-        if (!load_kv(&tmap_v, 0, w.head_kv)) break;
-        bool ok = true;
-        for (int j = 1; j < w.nmax && ok; ++j) {
-          ok = load_kv(&tmap_k, j * kBlockN, w.head_kv) && load_kv(&tmap_v, j * kBlockN, w.head_kv);
+      bool ok = true;
+      for (long long step = blockIdx.x; step < p.num_steps && ok; step += gridDim.x) {
+        for (int part = 0; part < p.units_per_step && ok; ++part) {
+          Unit w;
+          if (!unit_at(p, step, part, w)) continue;
+          ok = load_q(0, w.q0, w.head_q) && load_kv(&tmap_k, 0, w.head_kv) &&
+               (!w.valid1 || load_q(1, w.q0 + kBlockM, w.head_q)) && load_kv(&tmap_v, 0, w.head_kv);
+          for (int j = 1; j < w.nmax && ok; ++j)
+            ok = load_kv(&tmap_k, j * kBlockN, w.head_kv) && load_kv(&tmap_v, j * kBlockN, w.head_kv);
         }
-        if (!ok) break;
       }
       // Drain: every issued copy must have landed before the CTA may exit.
       for (int s = 0; s < S; ++s)
@@ -291,100 +317,124 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    // The whole warp walks the schedule, so control flow and descriptor arithmetic stay
+    // warp-uniform (kept in uniform registers); one elected lane issues each tcgen05
+    // instruction.
     regs_decrease<kRegsControl>();
-    if (lane == 0) {
+    {
       Ring ring;
       uint32_t q_par[2] = {0u, 0u}, pf_par[2] = {0u, 0u}, of_par[2] = {1u, 1u};
-      const uint32_t sQ_addr = smem_u32(sQ);
-      const uint32_t sKV_addr = smem_u32(sKV);
+      const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_base, 0);
+      const uint64_t desc_q = smem_desc_kmajor_sw128(smem_u32(sQ));
+      const uint64_t desc_k = smem_desc_kmajor_sw128(smem_u32(sKV));
+      const uint64_t desc_v = smem_desc_mnmajor_sw128(smem_u32(sKV), Plan::kChunkBytes);
+      const uint32_t idesc_s = p.idesc_s, idesc_pv = p.idesc_pv;
 
+      // Adds a byte offset to a descriptor's start-address field (bits 0-13, in 16-byte units).
+      auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
       // S_t = Q_t K^T over D in steps of 16 (K-major A and B, 128-byte swizzle).
       auto issue_s = [&](int t, uint32_t stage) {
-        const uint32_t qa = sQ_addr + t * Plan::kTileBytes;
-        const uint32_t ka = sKV_addr + stage * Plan::kTileBytes;
+        const uint64_t da = adv(desc_q, t * Plan::kTileBytes);
+        const uint64_t db = adv(desc_k, stage * Plan::kTileBytes);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
-          mma_ss(tmem_base + t * 128, smem_desc_kmajor_sw128(qa + off), smem_desc_kmajor_sw128(ka + off),
-                 p.idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
+            mma_ss(tmem + t * 128, adv(da, off), adv(db, off), idesc_s, kk > 0 ? 1u : 0u);
+          }
         }
+        __syncwarp();
       };
       // O_t += P_t V over the 128 keys in steps of 16 (P from TMEM, V MN-major in smem).
       auto issue_pv = [&](int t, uint32_t stage, bool accumulate) {
-        const uint32_t va = sKV_addr + stage * Plan::kTileBytes;
+        const uint64_t dv = adv(desc_v, stage * Plan::kTileBytes);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          mma_ts(tmem_base + 256 + t * 128, tmem_base + t * 128 + kk * 8,
-                 smem_desc_mnmajor_sw128(va + kk * 2048, Plan::kChunkBytes), p.idesc_pv,
-                 (accumulate || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBlockN / 16; ++kk)
+            mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, adv(dv, kk * 2048), idesc_pv,
+                   (accumulate || kk > 0) ? 1u : 0u);
         }
+        __syncwarp();
+      };
+      auto commit = [&](uint64_t* bar) {
+        if (elect_one()) tc_commit(bar);
+        __syncwarp();
+      };
+      // Every lane waits; the warp proceeds only if all lanes saw the phase complete.
+      auto wait_all = [&](uint64_t* bar, uint32_t parity, unsigned site) -> bool {
+        const bool mine = wait_phase(bar, parity, abort_flag, site);
+        return __all_sync(0xffffffffu, mine);
       };
 
       bool ok = true;
-      for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(p, u);
-        const int n[2] = {w.n0, w.n1};
-        const bool valid[2] = {true, w.valid1};
+      for (long long step = blockIdx.x; step < p.num_steps && ok; step += gridDim.x) {
+      for (int part = 0; part < p.units_per_step && ok; ++part) {
+        Unit w;
+        if (!unit_at(p, step, part, w)) continue;
+        const int n0 = w.n0, n1 = w.valid1 ? w.n1 : 0;
 
         // Block 0 scores for both tiles.
-        if (!(ok = wait_phase(&q_full[0], q_par[0], abort_flag, kSiteMmaQ))) break;
+        if (!(ok = wait_all(&q_full[0], q_par[0], kSiteMmaQ))) break;
         q_par[0] ^= 1u;
         const uint32_t k0_stage = ring.stage;
-        if (!(ok = wait_phase(&kv_full[k0_stage], ring.phase, abort_flag, kSiteMmaKV))) break;
+        if (!(ok = wait_all(&kv_full[k0_stage], ring.phase, kSiteMmaKV))) break;
         ring.advance<S>();
         tc_fence_after();
         issue_s(0, k0_stage);
-        tc_commit(&s_full[0]);
-        if (n[0] == 1) tc_commit(&q_empty[0]);
-        if (valid[1]) {
-          if (!(ok = wait_phase(&q_full[1], q_par[1], abort_flag, kSiteMmaQ))) break;
+        commit(&s_full[0]);
+        if (n0 == 1) commit(&q_empty[0]);
+        if (n1 > 0) {
+          if (!(ok = wait_all(&q_full[1], q_par[1], kSiteMmaQ))) break;
           q_par[1] ^= 1u;
           tc_fence_after();
           issue_s(1, k0_stage);
-          tc_commit(&s_full[1]);
-          if (n[1] == 1) tc_commit(&q_empty[1]);
+          commit(&s_full[1]);
+          if (n1 == 1) commit(&q_empty[1]);
         }
-        tc_commit(&kv_empty[k0_stage]);
+        commit(&kv_empty[k0_stage]);
 
         for (int j = 0; j < w.nmax && ok; ++j) {
           const uint32_t v_stage = ring.stage;
-          if (!(ok = wait_phase(&kv_full[v_stage], ring.phase, abort_flag, kSiteMmaKV))) break;
+          if (!(ok = wait_all(&kv_full[v_stage], ring.phase, kSiteMmaKV))) break;
           ring.advance<S>();
           const bool has_next = (j + 1) < w.nmax;
           const uint32_t kn_stage = ring.stage, kn_phase = ring.phase;
           bool kn_ready = false;
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (!valid[t] || j >= n[t]) continue;
-            if (!(ok = wait_phase(&p_full[t], pf_par[t], abort_flag, kSiteMmaP))) break;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int n = t ? n1 : n0;
+            if (!ok || j >= n) continue;
+            if (!(ok = wait_all(&p_full[t], pf_par[t], kSiteMmaP))) continue;
             pf_par[t] ^= 1u;
             if (j == 0) {
-              if (!(ok = wait_phase(&o_free[t], of_par[t], abort_flag, kSiteMmaOFree))) break;
+              if (!(ok = wait_all(&o_free[t], of_par[t], kSiteMmaOFree))) continue;
               of_par[t] ^= 1u;
             }
             tc_fence_after();
             issue_pv(t, v_stage, j > 0);
-            if (j == n[t] - 1) tc_commit(&o_full[t]);
-            if (j + 1 < n[t]) {
+            if (j == n - 1) commit(&o_full[t]);
+            if (j + 1 < n) {
               if (!kn_ready) {
-                if (!(ok = wait_phase(&kv_full[kn_stage], kn_phase, abort_flag, kSiteMmaKV))) break;
+                if (!(ok = wait_all(&kv_full[kn_stage], kn_phase, kSiteMmaKV))) continue;
                 kn_ready = true;
                 tc_fence_after();
               }
               issue_s(t, kn_stage);
-              tc_commit(&s_full[t]);
-              if (j + 2 == n[t]) tc_commit(&q_empty[t]);
+              commit(&s_full[t]);
+              if (j + 2 == n) commit(&q_empty[t]);
             }
           }
           if (!ok) break;
-          tc_commit(&kv_empty[v_stage]);
+          commit(&kv_empty[v_stage]);
           if (has_next) {
-            tc_commit(&kv_empty[kn_stage]);
+            commit(&kv_empty[kn_stage]);
             ring.advance<S>();
           }
         }
       }
-      // Drain: all MMAs issued by this thread complete before TMEM is released.
-      tc_commit(drain);
+      }
+      // Drain: all MMAs issued by this warp complete before TMEM is released.
+      commit(drain);
       drain_phase(drain, 0u, abort_flag);
     }
     __syncwarp();
@@ -400,8 +450,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_par = 0u, o_par = 0u;
     bool ok = true;
 
-    for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-      const Unit w = decode_unit(p, u);
+    for (long long step = blockIdx.x; step < p.num_steps && ok; step += gridDim.x) {
+    for (int part = 0; part < p.units_per_step && ok; ++part) {
+      Unit w;
+      if (!unit_at(p, step, part, w)) continue;
       if (t == 1 && !w.valid1) continue;
       const int n = t ? w.n1 : w.n0;
       const int row = w.q0 + t * kBlockM + r;
@@ -439,16 +491,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < kBlockN; ++i)
             if (k0 + i > key_lim) s[i] = -INFINITY;
         }
-        float mx[8];
+        // Row maximum: four independent chains of three-input max, then combined.
+        float mx[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = s[i];
+        for (int e = 0; e < 4; ++e) mx[e] = max3f(s[e], s[4 + e], s[8 + e]);
 #pragma unroll
-        for (int i = 8; i < kBlockN; i += 8) {
+        for (int i = 12; i < kBlockN; i += 8) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[i + e]);
+          for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[i + e], s[i + 4 + e]);
         }
-        const float rowmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float rowmax = fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]);
         const float m_new = fmaxf(m, rowmax * c);
         // Lazy correction: adopt a new max only when it grew by more than kRescaleLog2.
         float alpha = 1.f;
@@ -465,9 +517,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float neg_m = -m;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 c2 = make_float2(c, c);
+        const float2 nm2 = make_float2(neg_m, neg_m);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
         // P = 2^(s*c - m) in two halves of 64 keys; each half is packed to bf16 pairs and
-        // written over the (already loaded) score columns it came from.
+        // written over the (already loaded) score columns it came from.  In unmasked
+        // blocks, poly_pairs_per8<D>() of every 8 column pairs take the FMA-pipe
+        // polynomial instead of the special-function unit.
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
@@ -475,24 +532,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
               const int col = half * 64 + i;
-              const float p0 = (k0 + col > key_lim) ? 0.f : ex2_approx(fmaf(s[col], c, neg_m));
-              const float p1 = (k0 + col + 1 > key_lim) ? 0.f : ex2_approx(fmaf(s[col + 1], c, neg_m));
-              acc[(i >> 1) & 3] += p0 + p1;
-              pk[i >> 1] = pack_bf16x2(p0, p1);
+              const float2 x = fma2(make_float2(s[col], s[col + 1]), c2, nm2);
+              float2 pr;
+              pr.x = (k0 + col > key_lim) ? 0.f : ex2_approx(x.x);
+              pr.y = (k0 + col + 1 > key_lim) ? 0.f : ex2_approx(x.y);
+              acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], pr);
+              pk[i >> 1] = pack_bf16x2(pr.x, pr.y);
             }
           } else {
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
               const int col = half * 64 + i;
-              const float p0 = ex2_approx(fmaf(s[col], c, neg_m));
-              const float p1 = ex2_approx(fmaf(s[col + 1], c, neg_m));
-              acc[(i >> 1) & 3] += p0 + p1;
-              pk[i >> 1] = pack_bf16x2(p0, p1);
+              const float2 x = fma2(make_float2(s[col], s[col + 1]), c2, nm2);
+              float2 pr;
+              if (((col >> 1) & 7) < poly_pairs_per8<D>()) {
+                pr = exp2_poly2(x);
+              } else {
+                pr.x = ex2_approx(x.x);
+                pr.y = ex2_approx(x.y);
+              }
+              acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], pr);
+              pk[i >> 1] = pack_bf16x2(pr.x, pr.y);
             }
           }
           tmem_st32(t_s + half * 32, pk);
         }
-        l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        {
+          const float2 a01 = add2(acc[0], acc[1]);
+          const float2 a23 = add2(acc[2], acc[3]);
+          const float2 a = add2(a01, a23);
+          l += a.x + a.y;
+        }
         if (any_rescale) {
           // O_t holds blocks < j (their MMAs completed before S_t(j) was signalled) and
           // P_t(j) V has not been issued yet, so the accumulator can be rescaled here.
@@ -541,6 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&o_free[t]);
       if (row_ok) p.lse[(size_t)w.head_q * p.N + row] = (m + log2f(l)) * 0.69314718055994530942f;
     }
+    }
   } else {
     regs_decrease<kRegsControl>();
   }
@@ -551,6 +622,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+}
+
+// ---------------------------------------------------------------- self-test kernels
+
+// Evaluates the polynomial exp2 used by the softmax on n inputs (n even is not required).
+__global__ void selftest_exp2_poly(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 in = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  const float2 out = exp2_poly2(in);
+  y[i] = out.x;
+  if (i + 1 < n) y[i + 1] = out.y;
+}
+
+// Waits on an mbarrier that nothing ever arrives on, with a short limit: exercises the
+// bounded-wait path (abort flag, fault-site record, orderly return) without a fault.
+__global__ void selftest_wait_timeout(unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_phase(&bar, 0u, &abort_flag, kSiteSelfTest, timeout_ns);
+  __syncthreads();
 }
 
 }  // namespace attn

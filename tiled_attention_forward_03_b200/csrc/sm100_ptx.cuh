@@ -200,6 +200,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          (b_mn_major ? (1u << 16) : 0u) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- warp helpers
+
+// True on exactly one (the lowest) active lane of a fully active warp.
+ATTN_DEV bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------- register reallocation
 
 // Warpgroup-wide register budget changes.  The increases must be covered by decreases
@@ -219,6 +232,58 @@ ATTN_DEV float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Three-input maximum (sm_100).
+ATTN_DEV float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Paired fp32 arithmetic (one instruction for two lanes of data, sm_100).
+ATTN_DEV float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+ATTN_DEV float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for a pair, on the FMA pipe: x = n + f with n = round(x), |f| <= 1/2;
+// 2^f by a degree-3 polynomial (minimax relative error 7.5e-5 on [-1/2, 1/2],
+// coefficients fitted by csrc/fit_exp2_poly.py with the Remez exchange algorithm);
+// 2^n applied by adding n to the exponent field.  Inputs below -125 are clamped
+// (2^-125 is negligible next to the row maximum's 1); inputs must be < 2^22.
+ATTN_DEV float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound holds round(x) in its low bits
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 j = add2(x, make_float2(kRound, kRound));
+  const float2 n = add2(j, make_float2(-kRound, -kRound));
+  const float2 f = fma2(n, make_float2(-1.0f, -1.0f), x);
+  float2 q = fma2(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                  make_float2(0.2426111251115799f, 0.2426111251115799f));
+  q = fma2(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  q = fma2(q, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  float2 r;
+  r.x = __int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23));
+  r.y = __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23));
+  return r;
 }
 
 // Two floats -> packed bf16x2 (round to nearest even); `lo` in bits 0-15.
