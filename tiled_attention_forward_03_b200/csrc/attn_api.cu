@@ -184,7 +184,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.causal = causal ? 1 : 0;
   p.units_per_step = p.causal ? 2 : 1;
   p.num_steps = p.causal ? (long long)B * Hq * ((p.num_pairs + 1) / 2) : p.num_units;
-  p.c = std::fabs(scale) * 1.44269504088896340736f;
+  // c > 0 always: masked scores are -inf and -inf * c must stay -inf.  For scale == 0 every
+  // allowed score gives 2^(tiny) == 1 in fp32, the same softmax as c == 0.
+  p.c = std::fmax(std::fabs(scale) * 1.44269504088896340736f, 1e-30f);
   p.idesc_s = attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, scale < 0.f);
   p.idesc_pv = attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
 

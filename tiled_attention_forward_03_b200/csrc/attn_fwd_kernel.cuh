@@ -41,11 +41,11 @@
 namespace attn {
 
 constexpr int kThreads = 384;  // three warpgroups
-// Register split (launch: 384 x 168): softmax warpgroups 2 x 128 x 200, the
-// producer/MMA warpgroup 128 x 104; 2*128*200 + 128*104 == 384*168.
+// Register split (launch: 384 x 168): softmax warpgroups 2 x 128 x 224, the
+// producer/MMA warpgroup 128 x 56; 2*128*224 + 128*56 == 384*168.
 constexpr int kRegsAtLaunch = 168;
-constexpr int kRegsSoftmax = 200;
-constexpr int kRegsControl = 104;
+constexpr int kRegsSoftmax = 224;
+constexpr int kRegsControl = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsAtLaunch,
               "register split exceeds the launch allocation");
 constexpr int kBlockM = 128;  // query rows per tile
@@ -492,54 +492,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (k0 + i > key_lim) s[i] = -INFINITY;
         }
         // Row maximum: four independent chains of three-input max, then combined.
-        float mx[4];
+        auto row_max = [&]() -> float {
+          float mx[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) mx[e] = max3f(s[e], s[4 + e], s[8 + e]);
+          for (int e = 0; e < 4; ++e) mx[e] = max3f(s[e], s[4 + e], s[8 + e]);
 #pragma unroll
-        for (int i = 12; i < kBlockN; i += 8) {
+          for (int i = 12; i < kBlockN; i += 8) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[i + e], s[i + 4 + e]);
-        }
-        const float rowmax = fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]);
-        const float m_new = fmaxf(m, rowmax * c);
-        // Lazy correction: adopt a new max only when it grew by more than kRescaleLog2.
-        float alpha = 1.f;
-        bool any_rescale = false;
-        if (j == 0) {
-          m = m_new;
-        } else {
-          const bool need = m_new > m + kRescaleLog2;
-          any_rescale = __any_sync(0xffffffffu, need);
-          if (need) {
-            alpha = ex2_approx(m - m_new);
-            l *= alpha;
-            m = m_new;
+            for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[i + e], s[i + 4 + e]);
           }
-        }
-        const float neg_m = -m;
-        const float2 c2 = make_float2(c, c);
-        const float2 nm2 = make_float2(neg_m, neg_m);
-        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                         make_float2(0.f, 0.f)};
-        // P = 2^(s*c - m) in two halves of 64 keys; each half is packed to bf16 pairs and
-        // written over the (already loaded) score columns it came from.  In unmasked
-        // blocks, poly_pairs_per8<D>() of every 8 column pairs take the FMA-pipe
-        // polynomial instead of the special-function unit.
+          return fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]);
+        };
+        // P = 2^(s*c - m_use) in two halves of 64 keys; each half is packed to bf16 pairs and
+        // written over the (already loaded) score columns it came from.  Returns the row
+        // sum of the fp32 values.  Masked keys hold s = -inf, so their p is 0 from the
+        // special-function unit and 2^-125 (negligible) from the polynomial (c > 0 always).
+        // poly_pairs_per8<D>() of every 8 column pairs use the FMA-pipe polynomial instead
+        // of the special-function unit.  Warp-collective (TMEM stores).
+        auto exp_row = [&](float m_use) -> float {
+          const float2 c2 = make_float2(c, c);
+          const float2 nm2 = make_float2(-m_use, -m_use);
+          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-          if (masked) {
-#pragma unroll
-            for (int i = 0; i < 64; i += 2) {
-              const int col = half * 64 + i;
-              const float2 x = fma2(make_float2(s[col], s[col + 1]), c2, nm2);
-              float2 pr;
-              pr.x = (k0 + col > key_lim) ? 0.f : ex2_approx(x.x);
-              pr.y = (k0 + col + 1 > key_lim) ? 0.f : ex2_approx(x.y);
-              acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], pr);
-              pk[i >> 1] = pack_bf16x2(pr.x, pr.y);
-            }
-          } else {
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
               const int col = half * 64 + i;
@@ -554,15 +531,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], pr);
               pk[i >> 1] = pack_bf16x2(pr.x, pr.y);
             }
+            tmem_st32(t_s + half * 32, pk);
           }
-          tmem_st32(t_s + half * 32, pk);
+          const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+          return a.x + a.y;
+        };
+
+        // Lazy correction: the running max m is replaced only when the row's maximum
+        // exceeds it by more than kRescaleLog2, and then O and l are rescaled by 2^(m-m_new).
+        const float m_new = fmaxf(m, row_max() * c);
+        float alpha = 1.f;
+        bool any_rescale = false;
+        if (j == 0) {
+          m = m_new;
+        } else {
+          const bool need = m_new > m + kRescaleLog2;
+          any_rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = ex2_approx(m - m_new);
+            l *= alpha;
+            m = m_new;
+          }
         }
-        {
-          const float2 a01 = add2(acc[0], acc[1]);
-          const float2 a23 = add2(acc[2], acc[3]);
-          const float2 a = add2(a01, a23);
-          l += a.x + a.y;
-        }
+        l += exp_row(m);
         if (any_rescale) {
           // O_t holds blocks < j (their MMAs completed before S_t(j) was signalled) and
           // P_t(j) V has not been issued yet, so the accumulator can be rescaled here.
