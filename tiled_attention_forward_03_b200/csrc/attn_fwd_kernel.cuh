@@ -399,7 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ring.advance<S>();
           const bool has_next = (j + 1) < w.nmax;
           const uint32_t kn_stage = ring.stage, kn_phase = ring.phase;
-          bool kn_ready = false;
+          // K_{j+1} is waited for before P: it was loaded an iteration ago, and this way the
+          // P V and next-S MMAs of a tile are issued back to back once P is ready.
+          if (has_next && !(ok = wait_all(&kv_full[kn_stage], kn_phase, kSiteMmaKV))) break;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             const int n = t ? n1 : n0;
@@ -414,11 +416,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_pv(t, v_stage, j > 0);
             if (j == n - 1) commit(&o_full[t]);
             if (j + 1 < n) {
-              if (!kn_ready) {
-                if (!(ok = wait_all(&kv_full[kn_stage], kn_phase, kSiteMmaKV))) continue;
-                kn_ready = true;
-                tc_fence_after();
-              }
               issue_s(t, kn_stage);
               commit(&s_full[t]);
               if (j + 2 == n) commit(&q_empty[t]);
