@@ -20,6 +20,8 @@
 #ifndef ATTN_H_
 #define ATTN_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -75,6 +77,34 @@ typedef enum {
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int D, int causal, float scale,
              void* stream);
+
+/*
+ * attn_fwd_ws -- attn_fwd with a caller-provided device workspace.
+ *
+ * Same operation, arguments, errors and numerics as attn_fwd.  When the problem is
+ * non-causal and its last wave of work units would leave at least half of the GPU
+ * idle, each unit of that wave is split into two ranges of KV blocks that run on
+ * separate SMs; the range that finishes first writes its unnormalised fp32 O rows and
+ * (max, sum) to the workspace and the other merges them with its own (always in range
+ * order: results are deterministic, and equal attn_fwd's up to fp32 rounding order).
+ *   workspace        device pointer, 256-byte aligned, or NULL (then no split is made)
+ *   workspace_bytes  its size; must be >= attn_fwd_workspace_bytes() for the problem
+ *                    whenever a split is planned, else ATTN_ERR_INVALID_ARG
+ * The workspace needs no initialisation and is left in a state any later call accepts.
+ * Calls that share a workspace must not run concurrently (same stream, or ordered).
+ */
+int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse,
+                int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_fwd_workspace_bytes -- workspace attn_fwd_ws needs for these sizes on the current
+ * device (0 if it makes no split, e.g. causal problems or full last waves).  At most
+ * SMs/2 x 2 x 128 x (D + 2) x 4 bytes plus 16 bytes per split unit rounded up to 256
+ * (about 9.9 MB on a 148-SM B200 at D=128).
+ * Queries the current device's SM count; returns -1 on invalid sizes or a CUDA error.
+ */
+long long attn_fwd_workspace_bytes(int B, int Hq, int N, int D, int causal);
 
 /* Human-readable name of an attn_status_t value (static string, never null). */
 const char* attn_status_string(int status);

@@ -89,3 +89,25 @@ def test_num_units():
     assert attn.attn_num_units(1, 1, 257) == 2
     assert attn.attn_num_units(0, 1, 100) == 0
     assert attn.attn_num_units(1, 0, 100) == -1
+
+
+def call_ws(ws, nbytes, **kw):
+    args = dict(q=P, k=P, v=P, o=P, lse=P, B=1, Hq=2, Hkv=1, N=128, D=128, causal=0, scale=0.125, stream=None)
+    args.update(kw)
+    return attn.attn_fwd_ws(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["Hq"],
+                            args["Hkv"], args["N"], args["D"], args["causal"], args["scale"], ws, nbytes, None)
+
+
+def test_workspace_entry_point_host_checks():
+    assert call_ws(P + 128, 1 << 20) == MISALIGNED          # workspace must be 256-byte aligned
+    assert call_ws(None, 4096) == INVALID                  # size without a buffer
+    assert call_ws(P, 1 << 20, D=96) == UNSUPPORTED        # the usual checks still apply first
+    assert call_ws(P, 1 << 20, q=None) == INVALID
+    assert call_ws(None, 0, B=0) == OK                     # empty problem
+
+
+def test_workspace_bytes_host_cases():
+    assert attn.attn_fwd_workspace_bytes(-1, 2, 128, 128, 0) == -1
+    assert attn.attn_fwd_workspace_bytes(1, 2, 128, 96, 0) == -1
+    assert attn.attn_fwd_workspace_bytes(4, 16, 2048, 128, 1) == 0   # causal never splits
+    assert attn.attn_fwd_workspace_bytes(0, 16, 2048, 128, 0) == 0

@@ -214,3 +214,59 @@ def test_misaligned_device_pointer_rejected(attn):
     st = attn.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr() + 2, lse.data_ptr(),
                        1, 1, 1, 128, 64, 0, 0.125, torch.cuda.current_stream().cuda_stream)
     assert st == attn.ATTN_ERR_MISALIGNED
+
+
+# ------------------------------------------------------------------ split last wave (workspace path)
+
+SPLIT = [
+    # (B, Hq, Hkv, N, D): non-causal shapes whose last wave is split into KV ranges
+    (1, 1, 1, 2048, 128),   # 1 head x 8 pairs = 8 units, all in the split last wave
+    (2, 3, 1, 1000, 128),   # ragged N, GQA 3:1
+    (1, 4, 2, 1100, 64),    # tile 1 of the last pair empty, D=64
+    (1, 2, 2, 1111, 128),   # ragged last block
+    (4, 16, 16, 2048, 128), # the cfg2 shape: 3 whole waves + 68 units split in 2
+]
+
+
+@pytest.mark.parametrize("shape", SPLIT, ids=lambda s: "B{}_Hq{}_Hkv{}_N{}_D{}".format(*s))
+def test_split_tail_matches_oracle_and_unsplit_path(attn, shape):
+    B, Hq, Hkv, N, D = shape
+    assert attn.attn_fwd_workspace_bytes(B, Hq, N, D, False) > 0, "shape does not exercise the split"
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, seed=5000 + N + D)
+    scale = 1 / math.sqrt(D)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    o1, l1 = attn.forward(qd, kd, vd, causal=False, scale=scale, split=True)
+    o2, l2 = attn.forward(qd, kd, vd, causal=False, scale=scale, split=False)
+    torch.cuda.synchronize()
+    assert attn.device_status() == (attn.ATTN_OK, 0)
+    o_ref, l_ref = attention_forward(q, k, v, False, scale)
+    for o, l in ((o1, l1), (o2, l2)):
+        assert_close(o.float().cpu().numpy().astype(np.float64), l.cpu().numpy().astype(np.float64),
+                     o_ref, l_ref, str(shape))
+    # the two schedules differ only in fp32 summation order
+    assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
+    assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+def test_split_tail_deterministic_across_calls_sharing_a_workspace(attn):
+    q, k, v = (x.cuda() for x in make_qkv(1, 4, 4, 2048, 128, seed=5100))
+    outs = [attn.forward(q, k, v, causal=False) for _ in range(3)]
+    torch.cuda.synchronize()
+    for o, l in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1])
+
+
+def test_split_workspace_too_small_is_rejected(attn):
+    B, Hq, N, D = 1, 2, 2048, 128
+    need = attn.attn_fwd_workspace_bytes(B, Hq, N, D, False)
+    assert need > 0
+    q, k, v = (x.cuda() for x in make_qkv(B, Hq, Hq, N, D, seed=5200))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hq, N, D, 0, 0.0883)
+    assert attn.attn_fwd_ws(*args, ws.data_ptr(), need - 256, s) == attn.ATTN_ERR_INVALID_ARG
+    assert attn.attn_fwd_ws(*args, ws.data_ptr(), need, s) == attn.ATTN_OK
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all()

@@ -17,7 +17,8 @@ from . import build as _build
 
 __all__ = [
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED",
-    "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "AttnError", "lib", "lib_path", "attn_fwd",
+    "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "AttnError", "lib", "lib_path", "attn_fwd", "attn_fwd_ws",
+    "attn_fwd_workspace_bytes",
     "attn_status_string", "attn_last_cuda_error", "attn_device_status", "attn_num_units",
     "attn_version", "attn_selftest_exp2_poly", "attn_selftest_wait_timeout", "forward",
     "forward_from_host", "device_status",
@@ -56,6 +57,10 @@ def _load() -> ctypes.CDLL:
     vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.attn_fwd.restype = i
+    L.attn_fwd_ws.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, ctypes.c_size_t, vp]
+    L.attn_fwd_ws.restype = i
+    L.attn_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.attn_fwd_workspace_bytes.restype = ctypes.c_longlong
     L.attn_status_string.argtypes = [i]
     L.attn_status_string.restype = ctypes.c_char_p
     L.attn_last_cuda_error.argtypes = []
@@ -82,6 +87,16 @@ lib_path = _build.LIB_PATH
 def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, stream) -> int:
     """Direct call of the C entry point; pointers and stream are integers (or None)."""
     return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, D, int(bool(causal)), float(scale), stream)
+
+
+def attn_fwd_ws(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, workspace, workspace_bytes, stream) -> int:
+    """Direct call of the workspace entry point (pointers, sizes and stream as integers)."""
+    return lib.attn_fwd_ws(q, k, v, o, lse, B, Hq, Hkv, N, D, int(bool(causal)), float(scale),
+                           workspace, workspace_bytes, stream)
+
+
+def attn_fwd_workspace_bytes(B: int, Hq: int, N: int, D: int, causal: bool) -> int:
+    return lib.attn_fwd_workspace_bytes(B, Hq, N, D, int(bool(causal)))
 
 
 def attn_status_string(status: int) -> str:
@@ -131,10 +146,30 @@ def _check(t, name, dtype, shape):
         raise ValueError(f"{name} must be contiguous")
 
 
-def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):
+_workspaces: dict = {}
+
+
+def _workspace(device, nbytes: int):
+    """A cached device buffer of at least nbytes for the split-tail schedule (per device)."""
+    import torch
+
+    key = (device.type, device.index)
+    buf = _workspaces.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _workspaces[key] = buf
+    return buf
+
+
+def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None,
+            split: bool = True):
     """Attention forward on CUDA bf16 tensors [B, H, N, D]; returns (o bf16, lse fp32 [B, Hq, N]).
 
-    Runs on ``stream`` (a torch.cuda.Stream) or torch's current stream.
+    Runs on ``stream`` (a torch.cuda.Stream) or torch's current stream.  With ``split``
+    (default) a non-causal problem whose last wave would leave the GPU half idle splits
+    that wave's KV ranges across SMs (attn_fwd_ws, workspace cached per device);
+    ``split=False`` calls attn_fwd.  Calls that share the cached workspace are ordered
+    on one stream; pass distinct streams only with split=False.
     """
     import torch
 
@@ -155,8 +190,16 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     _check(lse, "lse", torch.float32, (B, Hq, N))
     s = stream if stream is not None else torch.cuda.current_stream(q.device)
     with torch.cuda.device(q.device):
-        st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                      B, Hq, Hkv, N, D, causal, scale, s.cuda_stream)
+        ws_bytes = attn_fwd_workspace_bytes(B, Hq, N, D, causal) if split else 0
+        if ws_bytes < 0:
+            raise AttnError(ATTN_ERR_CUDA, "attn_fwd_workspace_bytes")
+        if ws_bytes > 0:
+            ws = _workspace(q.device, ws_bytes)
+            st = attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             B, Hq, Hkv, N, D, causal, scale, ws.data_ptr(), ws.numel(), s.cuda_stream)
+        else:
+            st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                          B, Hq, Hkv, N, D, causal, scale, s.cuda_stream)
     if st != ATTN_OK:
         raise AttnError(st)
     return out, lse

@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "attn.h"
@@ -118,6 +119,52 @@ int encode_map(CUtensorMap* map, const void* base, long long heads, int N, int D
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// How a non-causal problem is spread over the persistent grid.  Whole units run round
+// robin; if the last wave would be at most half full, each of its units is split into two
+// KV ranges (of at least two KV blocks) that run on separate CTAs and are merged through
+// a workspace holding the first-finished range's rows.  Since 2 x tail_units <= SMs, the
+// workspace is bounded by SMs/2 x 2 tiles x 128 rows x (D + 2) floats.
+struct Schedule {
+  long long grid = 0;
+  int whole_per_cta = 0, tail_units = 0, parts = 1;
+  size_t cnt_bytes = 0, ml_bytes = 0, o_bytes = 0;
+  size_t ws_bytes() const { return cnt_bytes + ml_bytes + o_bytes; }
+};
+
+Schedule plan_schedule(long long units, long long steps, int num_blocks, int num_sms, int causal, int D,
+                       bool allow_split) {
+  Schedule sc;
+  sc.grid = steps < num_sms ? steps : num_sms;
+  if (causal || !allow_split || units <= 0) return sc;
+  const long long tail = units % num_sms, whole = units / num_sms;
+  if (tail == 0) return sc;
+  // two KV ranges per unit of the last wave, each of at least two KV blocks
+  if (2 * tail > num_sms || num_blocks < 4) return sc;
+  const long long k = 2;
+  sc.whole_per_cta = (int)whole;
+  sc.tail_units = (int)tail;
+  sc.parts = (int)k;
+  sc.grid = whole > 0 ? num_sms : tail * k;
+  const size_t slots = (size_t)tail * 2;  // the first range's rows, per unit and tile
+  sc.cnt_bytes = ((size_t)tail * 2 * 2 * sizeof(unsigned) + 255) / 256 * 256;
+  sc.ml_bytes = slots * attn::kBlockM * 2 * sizeof(float);
+  sc.o_bytes = slots * attn::kBlockM * (size_t)D * sizeof(float);
+  return sc;
+}
+
+unsigned next_epoch() {
+  static std::atomic<unsigned> counter{0};
+  unsigned e;
+  do {
+    e = (counter.fetch_add(1u) + 1u) & 0xFFFFFFu;
+  } while (e == 0u);
+  return e;
+}
+
+int launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                   int N, int D, int causal, float scale, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
 }  // namespace
 
 extern "C" {
@@ -146,6 +193,35 @@ long long attn_num_units(int B, int Hq, int N) {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
              int D, int causal, float scale, void* stream) {
+  return launch_forward(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, nullptr, 0, stream);
+}
+
+int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                int D, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (workspace == nullptr && workspace_bytes != 0) return ATTN_ERR_INVALID_ARG;
+  if (workspace != nullptr && !aligned(workspace, 256)) return ATTN_ERR_MISALIGNED;
+  return launch_forward(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, workspace, workspace_bytes, stream);
+}
+
+long long attn_fwd_workspace_bytes(int B, int Hq, int N, int D, int causal) {
+  if (B < 0 || Hq < 1 || N < 0 || (D != 64 && D != 128)) return -1;
+  if (B == 0 || N == 0 || causal) return 0;
+  int dev = 0, num_sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  const long long units = attn_num_units(B, Hq, N);
+  const int nb = (int)(((long long)N + attn::kBlockN - 1) / attn::kBlockN);
+  return (long long)plan_schedule(units, units, nb, num_sms, 0, D, true).ws_bytes();
+}
+
+}  // extern "C"
+
+namespace {
+
+int launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                   int N, int D, int causal, float scale, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+
   // ---- host-side validation (no CUDA call before this block passes)
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
     return ATTN_ERR_INVALID_ARG;
@@ -190,7 +266,19 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.idesc_s = attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, scale < 0.f);
   p.idesc_pv = attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
 
-  const long long grid = p.num_steps < num_sms ? p.num_steps : num_sms;
+  // Split the last wave only when a workspace big enough for it was given.
+  const Schedule plan0 = plan_schedule(p.num_units, p.num_steps, p.num_blocks, num_sms, p.causal, D, true);
+  const bool split = workspace != nullptr && plan0.parts > 1;
+  if (split && workspace_bytes < plan0.ws_bytes()) return ATTN_ERR_INVALID_ARG;
+  const Schedule sc = split ? plan0 : plan_schedule(p.num_units, p.num_steps, p.num_blocks, num_sms, p.causal, D, false);
+  p.whole_per_cta = sc.whole_per_cta;
+  p.tail_units = sc.tail_units;
+  p.parts = sc.parts;
+  p.ws_cnt = split ? reinterpret_cast<unsigned*>(workspace) : nullptr;
+  p.ws_ml = split ? reinterpret_cast<float*>(static_cast<char*>(workspace) + sc.cnt_bytes) : nullptr;
+  p.ws_o = split ? reinterpret_cast<float*>(static_cast<char*>(workspace) + sc.cnt_bytes + sc.ml_bytes) : nullptr;
+  p.epoch = split ? next_epoch() : 0u;
+  const long long grid = sc.grid;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (D == 128) {
     attn::attn_fwd_sm100<128><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128>::kAlloc, s>>>(mq, mk, mv, p);
@@ -204,6 +292,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   }
   return ATTN_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 int attn_device_status(void* stream, int* site) {
   if (site) *site = 0;

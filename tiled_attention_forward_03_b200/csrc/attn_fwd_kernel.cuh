@@ -70,6 +70,7 @@ enum : unsigned {
   kSiteSoftmaxO = 8,
   kSiteDrain = 9,
   kSiteSelfTest = 10,
+  kSiteSplitMerge = 11,
 };
 
 __device__ unsigned int g_attn_fault_site = 0;
@@ -85,7 +86,8 @@ struct SmemPlan {
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] o_free[2] drain
   static constexpr int kNumBars = 4 + 2 * kStages + 8 + 1;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base (u32), abort flag (u32)
+  // tmem base (u32), abort flag (u32), per-tile "last range" flags (2 x u32)
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;              // slack for 1024-byte alignment
 };
@@ -101,6 +103,16 @@ struct FwdParams {
   long long num_steps;  // scheduling steps walked by the persistent grid
   int units_per_step;   // 1 (non-causal) or 2 (causal: heaviest + lightest pair of a head)
   int causal;
+  // Split tail (non-causal): every CTA first runs `whole_per_cta` whole units; the
+  // `tail_units` units of the last, partial wave are each split into `parts` (= 2) KV
+  // ranges, one per CTA.  parts == 1: no split, whole units round robin until num_units.
+  int whole_per_cta;
+  int tail_units;
+  int parts;
+  float* ws_o;        // first range's O rows [tail_units][2 tiles][D/4][128 rows] float4
+  float* ws_ml;       // first range's (m, l) [tail_units][2 tiles][128 rows] float2
+  unsigned* ws_cnt;   // [tail_units][2 tiles][2]: finished ranges ((epoch << 8) | count), ready flag (epoch)
+  unsigned epoch;     // launch tag (24 bits, non-zero): counts of other launches read as 0
   float c;           // |scale| * log2(e)
   uint32_t idesc_s;  // S = Q K^T instruction descriptor (negates A when scale < 0)
   uint32_t idesc_pv; // O += P V instruction descriptor
@@ -110,9 +122,13 @@ struct Unit {
   int q0;          // first query row of tile 0
   int head_q;      // b * Hq + hq
   int head_kv;     // b * Hkv + hq / group
-  int n0, n1;      // KV blocks visited by tile 0 / tile 1
+  int jb;          // first KV block of this work item (0 unless the unit is split)
+  int n0, n1;      // end (exclusive) of the KV blocks visited by tile 0 / tile 1
   bool valid1;     // tile 1 holds at least one row < N
   int nmax;
+  int parts;       // KV ranges the unit is split into (1: whole unit)
+  int part;        // which range this item is
+  int tail;        // index of the split unit among the tail units
 };
 
 __device__ __forceinline__ Unit make_unit(const FwdParams& p, long long head, int pair) {
@@ -131,6 +147,10 @@ __device__ __forceinline__ Unit make_unit(const FwdParams& p, long long head, in
     w.n1 = p.num_blocks;
   }
   w.nmax = w.valid1 ? w.n1 : w.n0;
+  w.jb = 0;
+  w.parts = 1;
+  w.part = 0;
+  w.tail = 0;
   return w;
 }
 
@@ -154,6 +174,53 @@ __device__ __forceinline__ bool unit_at(const FwdParams& p, long long step, int 
   if (part == 1 && pair == p.num_pairs - 1 - s) return false;
   w = make_unit(p, head, pair);
   return true;
+}
+
+// Counts one finished KV range of a split unit and returns how many had finished before
+// it in this launch.  The word holds (epoch << 8) | count; a word left by another launch
+// (different epoch) counts as zero, so the workspace never needs clearing.  Each failed
+// compare-and-swap means another range's update succeeded, so the loop ends after at
+// most `parts` attempts.
+__device__ __forceinline__ unsigned count_finished(unsigned* cnt, unsigned epoch) {
+  unsigned old = atomicAdd(cnt, 0u);
+  while (true) {
+    const unsigned before = ((old >> 8) == epoch) ? (old & 255u) : 0u;
+    const unsigned prev = atomicCAS(cnt, old, (epoch << 8) | (before + 1u));
+    if (prev == old) return before;
+    old = prev;
+  }
+}
+
+// Work item `it` of this CTA.  Returns 0 when the CTA has no more items, 1 for an item
+// in `w`, 2 for an empty slot (causal: the middle pair of a head with an odd pair count).
+// Causal: two units per step (see unit_at), steps round robin.  Non-causal: whole units
+// round robin; with a split tail, each CTA then runs at most one KV range of one of the
+// last wave's units (ranges of a unit go to adjacent CTAs).
+__device__ __forceinline__ int item_at(const FwdParams& p, int it, Unit& w) {
+  if (p.causal) {
+    const long long step = blockIdx.x + (long long)(it >> 1) * gridDim.x;
+    if (step >= p.num_steps) return 0;
+    return unit_at(p, step, it & 1, w) ? 1 : 2;
+  }
+  if (p.parts <= 1 || it < p.whole_per_cta) {
+    const long long u = blockIdx.x + (long long)it * gridDim.x;
+    if (u >= p.num_units) return 0;
+    const long long head = u / p.num_pairs;
+    w = make_unit(p, head, (int)(u - head * p.num_pairs));
+    return 1;
+  }
+  if (it > p.whole_per_cta) return 0;
+  const int q = blockIdx.x;
+  if (q >= p.tail_units * p.parts) return 0;
+  const long long u = (long long)p.whole_per_cta * gridDim.x + q / p.parts;
+  const long long head = u / p.num_pairs;
+  w = make_unit(p, head, (int)(u - head * p.num_pairs));
+  w.parts = p.parts;
+  w.part = q % p.parts;
+  w.tail = q / p.parts;
+  w.jb = (int)((long long)w.part * p.num_blocks / p.parts);
+  w.n0 = w.n1 = w.nmax = (int)((long long)(w.part + 1) * p.num_blocks / p.parts);
+  return 1;
 }
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA abort flag,
@@ -298,15 +365,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       bool ok = true;
-      for (long long step = blockIdx.x; step < p.num_steps && ok; step += gridDim.x) {
-        for (int part = 0; part < p.units_per_step && ok; ++part) {
-          Unit w;
-          if (!unit_at(p, step, part, w)) continue;
-          ok = load_q(0, w.q0, w.head_q) && load_kv(&tmap_k, 0, w.head_kv) &&
-               (!w.valid1 || load_q(1, w.q0 + kBlockM, w.head_q)) && load_kv(&tmap_v, 0, w.head_kv);
-          for (int j = 1; j < w.nmax && ok; ++j)
-            ok = load_kv(&tmap_k, j * kBlockN, w.head_kv) && load_kv(&tmap_v, j * kBlockN, w.head_kv);
-        }
+      for (int it = 0; ok; ++it) {
+        Unit w;
+        const int got = item_at(p, it, w);
+        if (got == 0) break;
+        if (got == 2) continue;
+        ok = load_q(0, w.q0, w.head_q) && load_kv(&tmap_k, w.jb * kBlockN, w.head_kv) &&
+             (!w.valid1 || load_q(1, w.q0 + kBlockM, w.head_q)) && load_kv(&tmap_v, w.jb * kBlockN, w.head_kv);
+        for (int j = w.jb + 1; j < w.nmax && ok; ++j)
+          ok = load_kv(&tmap_k, j * kBlockN, w.head_kv) && load_kv(&tmap_v, j * kBlockN, w.head_kv);
       }
       // Drain: every issued copy must have landed before the CTA may exit.
       for (int s = 0; s < S; ++s)
@@ -367,13 +434,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       bool ok = true;
-      for (long long step = blockIdx.x; step < p.num_steps && ok; step += gridDim.x) {
-      for (int part = 0; part < p.units_per_step && ok; ++part) {
+      for (int it = 0; ok; ++it) {
         Unit w;
-        if (!unit_at(p, step, part, w)) continue;
+        const int got = item_at(p, it, w);
+        if (got == 0) break;
+        if (got == 2) continue;
+        const int jb = w.jb;
         const int n0 = w.n0, n1 = w.valid1 ? w.n1 : 0;
 
-        // Block 0 scores for both tiles.
+        // First block's scores for both tiles.
         if (!(ok = wait_all(&q_full[0], q_par[0], kSiteMmaQ))) break;
         q_par[0] ^= 1u;
         const uint32_t k0_stage = ring.stage;
@@ -382,18 +451,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_s(0, k0_stage);
         commit(&s_full[0]);
-        if (n0 == 1) commit(&q_empty[0]);
+        if (n0 == jb + 1) commit(&q_empty[0]);
         if (n1 > 0) {
           if (!(ok = wait_all(&q_full[1], q_par[1], kSiteMmaQ))) break;
           q_par[1] ^= 1u;
           tc_fence_after();
           issue_s(1, k0_stage);
           commit(&s_full[1]);
-          if (n1 == 1) commit(&q_empty[1]);
+          if (n1 == jb + 1) commit(&q_empty[1]);
         }
         commit(&kv_empty[k0_stage]);
 
-        for (int j = 0; j < w.nmax && ok; ++j) {
+        for (int j = jb; j < w.nmax && ok; ++j) {
           const uint32_t v_stage = ring.stage;
           if (!(ok = wait_all(&kv_full[v_stage], ring.phase, kSiteMmaKV))) break;
           ring.advance<S>();
@@ -408,12 +477,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok || j >= n) continue;
             if (!(ok = wait_all(&p_full[t], pf_par[t], kSiteMmaP))) continue;
             pf_par[t] ^= 1u;
-            if (j == 0) {
+            if (j == jb) {
               if (!(ok = wait_all(&o_free[t], of_par[t], kSiteMmaOFree))) continue;
               of_par[t] ^= 1u;
             }
             tc_fence_after();
-            issue_pv(t, v_stage, j > 0);
+            issue_pv(t, v_stage, j > jb);
             if (j == n - 1) commit(&o_full[t]);
             if (j + 1 < n) {
               issue_s(t, kn_stage);
@@ -428,7 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ring.advance<S>();
           }
         }
-      }
       }
       // Drain: all MMAs issued by this warp complete before TMEM is released.
       commit(drain);
@@ -447,17 +515,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_par = 0u, o_par = 0u;
     bool ok = true;
 
-    for (long long step = blockIdx.x; step < p.num_steps && ok; step += gridDim.x) {
-    for (int part = 0; part < p.units_per_step && ok; ++part) {
+    for (int it = 0; ok; ++it) {
       Unit w;
-      if (!unit_at(p, step, part, w)) continue;
+      const int got_item = item_at(p, it, w);
+      if (got_item == 0) break;
+      if (got_item == 2) continue;
       if (t == 1 && !w.valid1) continue;
       const int n = t ? w.n1 : w.n0;
       const int row = w.q0 + t * kBlockM + r;
       const int key_lim = p.causal ? min(row, p.N - 1) : (p.N - 1);
       float m = -INFINITY, l = 0.f;
 
-      for (int j = 0; j < n; ++j) {
+      for (int j = w.jb; j < n; ++j) {
         if (!(ok = wait_phase(&s_full[t], s_par, abort_flag, kSiteSoftmaxS))) break;
         s_par ^= 1u;
         tc_fence_after();
@@ -539,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_new = fmaxf(m, row_max() * c);
         float alpha = 1.f;
         bool any_rescale = false;
-        if (j == 0) {
+        if (j == w.jb) {
           m = m_new;
         } else {
           const bool need = m_new > m + kRescaleLog2;
@@ -572,33 +641,137 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
 
       // Epilogue: O = O_acc / l -> bf16, LSE = (m + log2 l) ln 2.
-      if (!(ok = wait_phase(&o_full[t], o_par, abort_flag, kSiteSoftmaxO))) break;
+      {
+        const bool got_o = wait_phase(&o_full[t], o_par, abort_flag, kSiteSoftmaxO);
+        // a split unit's epilogue has tile-wide barriers: agree on the outcome first
+        ok = (w.parts > 1) ? bar_and(1 + t, kBlockM, got_o) : got_o;
+        if (!ok) break;
+      }
       o_par ^= 1u;
       tc_fence_after();
-      const float inv_l = 1.f / l;
       const bool row_ok = row < p.N;
       __nv_bfloat16* orow = p.o + ((size_t)w.head_q * p.N + (row_ok ? row : 0)) * D;
+      if (w.parts == 1) {
+        const float inv_l = 1.f / l;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t ov[32];
-        tmem_ld32(t_o + ch * 32, ov);
-        tmem_ld_wait();
-        reg_fence32(ov);
-        uint32_t packed[16];
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t ov[32];
+          tmem_ld32(t_o + ch * 32, ov);
+          tmem_ld_wait();
+          reg_fence32(ov);
+          uint32_t packed[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          packed[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+          for (int i = 0; i < 16; ++i)
+            packed[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&o_free[t]);
+        if (row_ok) p.lse[(size_t)w.head_q * p.N + row] = (m + log2f(l)) * 0.69314718055994530942f;
+      } else {
+        // One of the two KV ranges of a split unit.  The ranges first agree on their
+        // finishing order; the first publishes its unnormalised O rows and (m, l) and
+        // raises a ready flag, the second waits for the flag (bounded) and merges:
+        //   M = max(m0, m1),  O = (O0 2^(m0-M) + O1 2^(m1-M)) / (l0 2^(m0-M) + l1 2^(m1-M))
+        // with the ranges always taken in range order, so the result does not depend on
+        // which range finished first.
+        volatile unsigned* order = reinterpret_cast<volatile unsigned*>(smem + Plan::kMiscOff + 8 + 4 * t);
+        unsigned* cnt = &p.ws_cnt[(w.tail * 2 + t) * 2];    // finished ranges (epoch-tagged)
+        unsigned* ready = cnt + 1;                          // epoch once range "first" published
+        if (r == 0) *order = count_finished(cnt, p.epoch);
+        named_bar_sync(1 + t, kBlockM);
+        const bool first = (*order == 0u);
+        const size_t slot = (size_t)w.tail * 2 + t;
+        float4* o_ws = reinterpret_cast<float4*>(p.ws_o) + slot * (kBlockM * D / 4);  // [D/4][128] float4
+        float2* ml_ws = reinterpret_cast<float2*>(p.ws_ml) + slot * kBlockM;         // [128]
+        if (first) {
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32(t_o + ch * 32, ov);
+            tmem_ld_wait();
+            reg_fence32(ov);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              o_ws[(ch * 8 + i) * kBlockM + r] = make_float4(__uint_as_float(ov[4 * i]), __uint_as_float(ov[4 * i + 1]),
+                                                             __uint_as_float(ov[4 * i + 2]), __uint_as_float(ov[4 * i + 3]));
+          }
+          tc_fence_before();
+          mbar_arrive(&o_free[t]);
+          ml_ws[r] = make_float2(m, l);
+          __threadfence();
+          named_bar_sync(1 + t, kBlockM);
+          if (r == 0) st_release_gpu(ready, p.epoch);
+        } else {
+          // wait for the other range's rows (it has counted itself finished, so it is
+          // only storing them); one thread polls, the tile's threads then all read.
+          bool have = true;
+          if (r == 0) {
+            const uint64_t t0 = global_timer_ns();
+            while (ld_acquire_gpu(ready) != p.epoch) {
+              if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+                *abort_flag = 1u;
+                atomicCAS(&g_attn_fault_site, 0u, (unsigned)kSiteSplitMerge);
+                have = false;
+                break;
+              }
+            }
+            *order = have ? 1u : 2u;
+          }
+          named_bar_sync(1 + t, kBlockM);
+          if (*order == 2u) {
+            ok = false;
+          } else {
+            __threadfence();
+            const float2 mo = __ldcg(ml_ws + r);                       // the other range
+            const bool own_is_0 = (w.part == 0);
+            const float m0 = own_is_0 ? m : mo.x, l0 = own_is_0 ? l : mo.y;
+            const float m1 = own_is_0 ? mo.x : m, l1 = own_is_0 ? mo.y : l;
+            const float mt = fmaxf(m0, m1);
+            const float w0 = ex2_approx(m0 - mt), w1 = ex2_approx(m1 - mt);
+            const float lt = fmaf(l1, w1, l0 * w0);
+            const float inv_l = 1.f / lt;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+              float4 other[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) other[i] = __ldcg(o_ws + (ch * 8 + i) * kBlockM + r);
+              uint32_t ov[32];
+              tmem_ld32(t_o + ch * 32, ov);
+              tmem_ld_wait();
+              reg_fence32(ov);
+              uint32_t packed[16];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float oth[4] = {other[i].x, other[i].y, other[i].z, other[i].w};
+                float res[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float mine = __uint_as_float(ov[4 * i + e]);
+                  const float x0 = own_is_0 ? mine : oth[e], x1 = own_is_0 ? oth[e] : mine;
+                  res[e] = fmaf(x1, w1, x0 * w0) * inv_l;
+                }
+                packed[2 * i] = pack_bf16x2(res[0], res[1]);
+                packed[2 * i + 1] = pack_bf16x2(res[2], res[3]);
+              }
+              if (row_ok) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+              }
+            }
+            if (row_ok) p.lse[(size_t)w.head_q * p.N + row] = (mt + log2f(lt)) * 0.69314718055994530942f;
+          }
+          tc_fence_before();
+          mbar_arrive(&o_free[t]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(&o_free[t]);
-      if (row_ok) p.lse[(size_t)w.head_q * p.N + row] = (m + log2f(l)) * 0.69314718055994530942f;
-    }
     }
   } else {
     regs_decrease<kRegsControl>();

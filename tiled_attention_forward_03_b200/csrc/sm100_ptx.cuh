@@ -260,6 +260,21 @@ ATTN_DEV bool bar_and(uint32_t id, uint32_t count, bool pred) {
   return r != 0;
 }
 
+// Named barrier `id` over `count` threads (a subset of the CTA).
+ATTN_DEV void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("barrier.cta.sync.aligned %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Release store / acquire load of a 32-bit word at GPU scope (cross-CTA flags).
+ATTN_DEV void st_release_gpu(unsigned* addr, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+ATTN_DEV unsigned ld_acquire_gpu(const unsigned* addr) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
 // ---------------------------------------------------------------- register reallocation
 
 // Warpgroup-wide register budget changes.  The increases must be covered by decreases
