@@ -106,6 +106,34 @@ int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse
  */
 long long attn_fwd_workspace_bytes(int B, int Hq, int N, int D, int causal);
 
+/*
+ * attn_fwd_noalloc -- attn_fwd_ws for callers that cannot allocate device memory.
+ *
+ * (The pages have no counterpart: this is an interface convenience.)  Some callers may
+ * not call cudaMalloc to provide attn_fwd_ws's workspace: code whose device memory is all
+ * owned by another allocator (a framework's caching allocator, an embedded runtime that
+ * forbids allocation after start-up), or latency-critical code that must not risk the
+ * device-wide synchronisation an allocation can cause.  This entry point takes no
+ * workspace argument and allocates nothing: the workspace is a 10 MiB
+ * array inside the library, present once on every device that loads the library and kept
+ * until the process exits.  Arguments, errors and numerics are those of attn_fwd; the
+ * caller still owns q, k, v, o and lse.
+ *   - Problems whose split needs more than the array (attn_fwd_workspace_bytes() larger
+ *     than attn_fwd_noalloc_scratch_bytes(); not reachable at D <= 128 on a 148-SM B200)
+ *     are rejected with ATTN_ERR_UNSUPPORTED and a message in attn_last_cuda_error().
+ *   - The first call on a device looks up the array's device address and clears the
+ *     array (a synchronous cudaMemset); make that first call before any stream capture.
+ *   - Every call shares the one array and leaves its contents behind; no later call
+ *     needs them cleared.  Calls whose kernels overlap on the GPU (different streams
+ *     without ordering) race on the array and must be avoided.
+ */
+int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+                     void* stream);
+
+/* Size in bytes of the array attn_fwd_noalloc uses as its workspace. */
+size_t attn_fwd_noalloc_scratch_bytes(void);
+
 /* Human-readable name of an attn_status_t value (static string, never null). */
 const char* attn_status_string(int status);
 

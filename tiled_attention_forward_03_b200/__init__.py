@@ -18,7 +18,7 @@ from . import build as _build
 __all__ = [
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED",
     "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "AttnError", "lib", "lib_path", "attn_fwd", "attn_fwd_ws",
-    "attn_fwd_workspace_bytes",
+    "attn_fwd_workspace_bytes", "attn_fwd_noalloc", "attn_fwd_noalloc_scratch_bytes",
     "attn_status_string", "attn_last_cuda_error", "attn_device_status", "attn_num_units",
     "attn_version", "attn_selftest_exp2_poly", "attn_selftest_wait_timeout", "forward",
     "forward_from_host", "device_status",
@@ -61,6 +61,10 @@ def _load() -> ctypes.CDLL:
     L.attn_fwd_ws.restype = i
     L.attn_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
     L.attn_fwd_workspace_bytes.restype = ctypes.c_longlong
+    L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+    L.attn_fwd_noalloc.restype = i
+    L.attn_fwd_noalloc_scratch_bytes.argtypes = []
+    L.attn_fwd_noalloc_scratch_bytes.restype = ctypes.c_size_t
     L.attn_status_string.argtypes = [i]
     L.attn_status_string.restype = ctypes.c_char_p
     L.attn_last_cuda_error.argtypes = []
@@ -93,6 +97,16 @@ def attn_fwd_ws(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, workspace, wor
     """Direct call of the workspace entry point (pointers, sizes and stream as integers)."""
     return lib.attn_fwd_ws(q, k, v, o, lse, B, Hq, Hkv, N, D, int(bool(causal)), float(scale),
                            workspace, workspace_bytes, stream)
+
+
+def attn_fwd_noalloc(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, stream) -> int:
+    """Direct call of the entry point that allocates nothing (its workspace is a static
+    device array in the library); for callers that may not allocate device memory."""
+    return lib.attn_fwd_noalloc(q, k, v, o, lse, B, Hq, Hkv, N, D, int(bool(causal)), float(scale), stream)
+
+
+def attn_fwd_noalloc_scratch_bytes() -> int:
+    return lib.attn_fwd_noalloc_scratch_bytes()
 
 
 def attn_fwd_workspace_bytes(B: int, Hq: int, N: int, D: int, causal: bool) -> int:

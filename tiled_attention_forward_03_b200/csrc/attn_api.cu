@@ -297,6 +297,84 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
 
 extern "C" {
 
+// ---------------------------------------------------------------------------------------
+// Entry point for callers that cannot allocate device memory.
+//
+// Some callers may not call cudaMalloc: code whose device memory is all owned by another
+// allocator (a framework's caching allocator, an embedded runtime that forbids allocation
+// after start-up), or latency-critical code that must not risk the device-wide
+// synchronisation an allocation can cause.  They cannot provide the workspace attn_fwd_ws
+// wants for its split last wave.  attn_fwd_noalloc gives them the same kernel with the
+// workspace taken from this file-scope device array instead: it exists once per device
+// that loads the library and stays allocated until the process exits.
+static __device__ __align__(256) unsigned char g_attn_noalloc_scratch[10u << 20];
+
+namespace {
+
+constexpr size_t kNoallocScratchBytes = sizeof(g_attn_noalloc_scratch);
+
+struct NoallocScratch {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+NoallocScratch g_noalloc[kMaxDevices];
+
+// Device address of the scratch array on `dev` (the current device).  In host code the
+// array's name is only a stand-in for it, so the address is looked up once per device,
+// and the array is cleared then (nothing in it must start at zero afterwards: the
+// kernel tags its counters with a per-launch epoch).
+void* noalloc_scratch(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  NoallocScratch& ns = g_noalloc[dev];
+  std::call_once(ns.once, [&ns] {
+    void* ptr = nullptr;
+    ns.err = cudaGetSymbolAddress(&ptr, g_attn_noalloc_scratch);
+    if (ns.err == cudaSuccess) ns.err = cudaMemset(ptr, 0, kNoallocScratchBytes);
+    if (ns.err == cudaSuccess) ns.ptr = ptr;
+  });
+  if (ns.ptr == nullptr) record_cuda_error("no-alloc scratch set-up", ns.err);
+  return ns.ptr;
+}
+
+}  // namespace
+
+int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                     int N, int D, int causal, float scale, void* stream) {
+  // the same host checks as attn_fwd, before any CUDA call
+  if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
+    return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return ATTN_OK;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return ATTN_ERR_MISALIGNED;
+  const long long need = attn_fwd_workspace_bytes(B, Hq, N, D, causal);
+  if (need < 0) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "workspace size query failed");
+    return ATTN_ERR_CUDA;
+  }
+  if ((size_t)need > kNoallocScratchBytes) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "attn_fwd_noalloc: this problem needs %lld bytes of scratch, more than the %zu-byte "
+                  "static array; use attn_fwd_ws with a caller workspace",
+                  need, kNoallocScratchBytes);
+    return ATTN_ERR_UNSUPPORTED;
+  }
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    record_cuda_error("cudaGetDevice", e);
+    return ATTN_ERR_CUDA;
+  }
+  void* scratch = noalloc_scratch(dev);
+  if (scratch == nullptr) return ATTN_ERR_CUDA;
+  return launch_forward(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, scratch, kNoallocScratchBytes, stream);
+}
+
+size_t attn_fwd_noalloc_scratch_bytes(void) { return kNoallocScratchBytes; }
+
 int attn_device_status(void* stream, int* site) {
   if (site) *site = 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
