@@ -29,7 +29,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = 1, /* null pointer, negative size, Hq % Hkv != 0, non-finite scale */
-  ATTN_ERR_UNSUPPORTED = 2, /* head dim D other than 64 or 128, or a size beyond the limits below */
+  ATTN_ERR_UNSUPPORTED = 2, /* head dim D other than 32, 64, 96 or 128, or a size beyond the limits below */
   ATTN_ERR_MISALIGNED = 3,  /* a q/k/v/o pointer not 16-byte aligned, or lse not 4-byte aligned */
   ATTN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
   ATTN_ERR_TIMEOUT = 5      /* a kernel wait gave up (reported by attn_device_status) */
@@ -50,7 +50,7 @@ typedef enum {
  *         B >= 0, N >= 0, Hq >= 1, Hkv >= 1, Hq % Hkv == 0.  B == 0 or N == 0
  *         is an empty problem: ATTN_OK is returned and nothing is launched
  *         (pointers may then be null).  Limits: B*Hq <= 2^31-1 and N <= 2^31-1.
- *   D     head dim of q, k, v and o: 64 or 128.
+ *   D     head dim of q, k, v and o: 32, 64, 96 or 128.
  *   causal  0: every key is visible; non-zero: key j is visible to query i
  *         iff j <= i (queries and keys share positions 0..N-1).
  *   scale   finite float multiplying q.k before the softmax (1/sqrt(D) is

@@ -61,7 +61,7 @@ def call(**kw):
     (dict(o=None), INVALID), (dict(lse=None), INVALID),
     (dict(B=-1), INVALID), (dict(N=-5), INVALID), (dict(Hq=0), INVALID), (dict(Hkv=0), INVALID),
     (dict(Hq=3, Hkv=2), INVALID), (dict(scale=math.nan), INVALID), (dict(scale=math.inf), INVALID),
-    (dict(D=96), UNSUPPORTED), (dict(D=256), UNSUPPORTED), (dict(D=0), UNSUPPORTED),
+    (dict(D=80), UNSUPPORTED), (dict(D=256), UNSUPPORTED), (dict(D=0), UNSUPPORTED), (dict(D=48), UNSUPPORTED),
     (dict(q=P + 8), MISALIGNED), (dict(k=P + 2), MISALIGNED), (dict(v=P + 4), MISALIGNED),
     (dict(o=P + 1), MISALIGNED), (dict(lse=P + 2), MISALIGNED),
 ])
@@ -101,13 +101,13 @@ def call_ws(ws, nbytes, **kw):
 def test_workspace_entry_point_host_checks():
     assert call_ws(P + 128, 1 << 20) == MISALIGNED          # workspace must be 256-byte aligned
     assert call_ws(None, 4096) == INVALID                  # size without a buffer
-    assert call_ws(P, 1 << 20, D=96) == UNSUPPORTED        # the usual checks still apply first
+    assert call_ws(P, 1 << 20, D=80) == UNSUPPORTED        # the usual checks still apply first
     assert call_ws(P, 1 << 20, q=None) == INVALID
     assert call_ws(None, 0, B=0) == OK                     # empty problem
 
 
 def test_workspace_bytes_host_cases():
     assert attn.attn_fwd_workspace_bytes(-1, 2, 128, 128, 0) == -1
-    assert attn.attn_fwd_workspace_bytes(1, 2, 128, 96, 0) == -1
+    assert attn.attn_fwd_workspace_bytes(1, 2, 128, 80, 0) == -1
     assert attn.attn_fwd_workspace_bytes(4, 16, 2048, 128, 1) == 0   # causal never splits
     assert attn.attn_fwd_workspace_bytes(0, 16, 2048, 128, 0) == 0

@@ -121,6 +121,21 @@ def test_edge_shapes(attn, shape):
     check_full(attn, q, k, v, causal, 1.0 / math.sqrt(D), str(shape))
 
 
+HEAD_DIMS = [
+    # (B, Hq, Hkv, N, D, causal): head dims 32 and 96 (the last 64-column chunk partly used)
+    (1, 2, 2, 1, 32, False), (1, 2, 1, 129, 32, True), (2, 4, 4, 700, 32, False), (1, 4, 2, 1025, 32, True),
+    (1, 2, 2, 1, 96, True), (1, 2, 1, 255, 96, False), (2, 4, 4, 700, 96, True), (1, 4, 2, 1025, 96, False),
+    (1, 8, 8, 2048, 96, False), (1, 8, 2, 2048, 96, True),
+]
+
+
+@pytest.mark.parametrize("shape", HEAD_DIMS, ids=lambda s: "B{}_Hq{}_Hkv{}_N{}_D{}_{}".format(*s[:5], "c" if s[5] else "nc"))
+def test_head_dims_32_and_96(attn, shape):
+    B, Hq, Hkv, N, D, causal = shape
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, seed=3500 + N + D + Hq)
+    check_full(attn, q, k, v, causal, 1.0 / math.sqrt(D), str(shape))
+
+
 @pytest.mark.parametrize("scale", [0.0, -0.0883883, 0.02, 0.5])
 @pytest.mark.parametrize("causal", [False, True])
 def test_scales(attn, scale, causal):
@@ -225,6 +240,8 @@ SPLIT = [
     (1, 4, 2, 1100, 64),    # tile 1 of the last pair empty, D=64
     (1, 2, 2, 1111, 128),   # ragged last block
     (4, 16, 16, 2048, 128), # the cfg2 shape: 3 whole waves + 68 units split in 2
+    (1, 4, 4, 1500, 96),    # D=96
+    (1, 3, 3, 2048, 32),    # D=32
 ]
 
 

@@ -69,7 +69,7 @@ def test_noalloc_matches_existing_entry_points_twice(attn, shape):
 def test_noalloc_rejects_bad_arguments_before_touching_the_gpu(attn):
     P = 0x10000
     s = torch.cuda.current_stream().cuda_stream
-    assert attn.attn_fwd_noalloc(P, P, P, P, P, 1, 2, 1, 128, 96, 0, 0.1, s) == attn.ATTN_ERR_UNSUPPORTED
+    assert attn.attn_fwd_noalloc(P, P, P, P, P, 1, 2, 1, 128, 80, 0, 0.1, s) == attn.ATTN_ERR_UNSUPPORTED
     assert attn.attn_fwd_noalloc(None, P, P, P, P, 1, 2, 1, 128, 128, 0, 0.1, s) == attn.ATTN_ERR_INVALID_ARG
     assert attn.attn_fwd_noalloc(P + 2, P, P, P, P, 1, 2, 1, 128, 128, 0, 0.1, s) == attn.ATTN_ERR_MISALIGNED
     assert attn.attn_fwd_noalloc(None, None, None, None, None, 0, 2, 1, 128, 128, 0, 0.1, s) == attn.ATTN_OK

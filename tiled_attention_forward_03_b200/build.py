@@ -86,7 +86,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         m = re.search(r"(\d+) bytes spill stores", line)
         if m and current and "attn_fwd_sm100" in current:
             spills.append(int(m.group(1)))
-    if len(regs) != 2 or any(r != EXPECTED_REGS for r in regs):
+    if len(regs) != 4 or any(r != EXPECTED_REGS for r in regs):
         os.remove(tmp)
         raise RuntimeError(f"unexpected kernel register counts {regs} (want {EXPECTED_REGS}):\n{log}")
     if verbose:

@@ -62,21 +62,24 @@ bool device_setup(int dev, int* num_sms) {
   DeviceInfo& d = g_dev[dev];
   std::call_once(d.once, [&d, dev] {
     cudaError_t e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn::attn_fwd_sm100<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               attn::SmemPlan<64>::kAlloc);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn::attn_fwd_sm100<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               attn::SmemPlan<128>::kAlloc);
-    // The kernels' register split (setmaxnreg) assumes exactly kRegsAtLaunch registers
-    // per thread at launch; a build that differs would make the increase wait forever,
-    // so such a build refuses to launch.
-    cudaFuncAttributes fa64, fa128;
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa64, attn::attn_fwd_sm100<64>);
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa128, attn::attn_fwd_sm100<128>);
+    // Every head-dim instance: dynamic shared memory opt-in, and a check that it has the
+    // register count its warpgroup register split (setmaxnreg) assumes at launch -- a build
+    // that differs would make the increase wait forever, so it refuses to launch.
+    bool regs_ok = true;
+    auto setup = [&](const void* fn, int smem) {
+      if (e != cudaSuccess) return;
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      cudaFuncAttributes fa;
+      if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, fn);
+      if (e == cudaSuccess && fa.numRegs != attn::kRegsAtLaunch) regs_ok = false;
+    };
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<32>), attn::SmemPlan<32>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64>), attn::SmemPlan<64>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<96>), attn::SmemPlan<96>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<128>), attn::SmemPlan<128>::kAlloc);
     d.err = e;
     d.attrs_ok = (e == cudaSuccess);
-    if (d.attrs_ok && (fa64.numRegs != attn::kRegsAtLaunch || fa128.numRegs != attn::kRegsAtLaunch)) {
+    if (d.attrs_ok && !regs_ok) {
       d.attrs_ok = false;
       d.err = cudaErrorInvalidDeviceFunction;
       d.bad_regs = true;
@@ -118,6 +121,8 @@ int encode_map(CUtensorMap* map, const void* base, long long heads, int N, int D
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool supported_head_dim(int D) { return D == 32 || D == 64 || D == 96 || D == 128; }
 
 // How a non-causal problem is spread over the persistent grid.  Whole units run round
 // robin; if the last wave would be at most half full, each of its units is split into two
@@ -204,7 +209,7 @@ int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse
 }
 
 long long attn_fwd_workspace_bytes(int B, int Hq, int N, int D, int causal) {
-  if (B < 0 || Hq < 1 || N < 0 || (D != 64 && D != 128)) return -1;
+  if (B < 0 || Hq < 1 || N < 0 || !supported_head_dim(D)) return -1;
   if (B == 0 || N == 0 || causal) return 0;
   int dev = 0, num_sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -225,7 +230,7 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   // ---- host-side validation (no CUDA call before this block passes)
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
     return ATTN_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
   if ((long long)B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return ATTN_OK;  // empty problem: nothing to compute or write
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
@@ -280,10 +285,19 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   p.epoch = split ? next_epoch() : 0u;
   const long long grid = sc.grid;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (D == 128) {
-    attn::attn_fwd_sm100<128><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128>::kAlloc, s>>>(mq, mk, mv, p);
-  } else {
-    attn::attn_fwd_sm100<64><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(mq, mk, mv, p);
+  switch (D) {
+    case 32:
+      attn::attn_fwd_sm100<32><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32>::kAlloc, s>>>(mq, mk, mv, p);
+      break;
+    case 64:
+      attn::attn_fwd_sm100<64><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(mq, mk, mv, p);
+      break;
+    case 96:
+      attn::attn_fwd_sm100<96><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<96>::kAlloc, s>>>(mq, mk, mv, p);
+      break;
+    default:
+      attn::attn_fwd_sm100<128><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128>::kAlloc, s>>>(mq, mk, mv, p);
+      break;
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -344,7 +358,7 @@ int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float
   // the same host checks as attn_fwd, before any CUDA call
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
     return ATTN_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
   if ((long long)B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return ATTN_OK;
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;

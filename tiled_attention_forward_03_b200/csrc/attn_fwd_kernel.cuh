@@ -56,6 +56,8 @@ constexpr float kRescaleLog2 = 8.0f;
 // costs issue slots that the MMA-issuing warp shares with the softmax warps).
 template <int D>
 __host__ __device__ constexpr int poly_pairs_per8() { return D == 128 ? 2 : 1; }
+// (D = 32 and 96 take 1 of 8, like D = 64: their tensor work per block is smaller than at
+// D = 128, so the exponentials weigh more and fewer issue slots can go to the polynomial.)
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s for any single wait
 
 // Fault-site codes written to g_attn_fault_site when a bounded wait gives up.
@@ -77,10 +79,12 @@ __device__ unsigned int g_attn_fault_site = 0;
 
 template <int D>
 struct SmemPlan {
-  static constexpr int kTileBytes = kBlockM * D * 2;       // one 128-row bf16 tile
-  static constexpr int kChunks = D / 64;                    // 64-column (128 B) swizzle chunks per row
+  static_assert(D == 32 || D == 64 || D == 96 || D == 128, "head dim must be 32, 64, 96 or 128");
+  static constexpr int kChunks = (D + 63) / 64;             // 64-column (128 B) swizzle chunks per row
   static constexpr int kChunkBytes = kBlockM * 128;         // one chunk of a tile: 16 KB
-  static constexpr int kStages = (D == 128) ? 4 : 8;        // K/V ring depth
+  // one 128-row tile; a partly used last chunk (D = 32, 96) is zero-filled by TMA
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = (kChunks == 2) ? 4 : 8;    // K/V ring depth
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
