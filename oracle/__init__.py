@@ -1,12 +1,14 @@
-"""fp64 CPU oracle for the attention forward pass -- test infrastructure only.
+"""fp64 CPU oracle for attention (forward and backward) -- test infrastructure only.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 and reference legs may import this package.  The product path (the CUDA
 library and its Python binding) never does.
 """
 from .attn_ref import (  # noqa: F401
+    attention_backward,
     attention_forward,
     attention_rows,
+    head_backward,
     head_forward,
     head_probs,
     head_scores,

@@ -1,4 +1,4 @@
-"""Plain fp64 CPU oracle for the scaled-dot-product attention forward pass.
+"""Plain fp64 CPU oracle for scaled-dot-product attention: forward pass and its gradients.
 
 TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module:
 only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
@@ -25,9 +25,12 @@ the full score matrix of one head is materialised, no blocking, no online
 softmax.  The readings of what the pages leave open (formula, LSE base,
 causal alignment, head mapping, layout) are listed in the design notes.
 
-Parity status: every function below is pinned by tests/test_oracle.py
+Parity status: every forward function below is pinned by tests/test_oracle.py
 (closed forms, invariants, a scalar brute force and a library special case)
-and by tests/test_oracle_mutants.py (planted mistakes must fail a pin).
+and by tests/test_oracle_mutants.py (planted mistakes must fail a pin).  The
+backward functions are pinned by tests/test_oracle_bwd.py (central differences
+of the forward, autograd through torch's fp64 SDPA, a scalar brute force through
+the softmax Jacobian, closed forms and invariants, planted mistakes).
 """
 from __future__ import annotations
 
@@ -131,3 +134,49 @@ def attention_rows(q, k, v, rows, causal: bool, scale: float):
         out_o.append((e / l) @ vh_arr)
         out_l.append(m + np.log(l))
     return np.stack(out_o), np.asarray(out_l)
+
+
+# ----------------------------------------------------------------------------------------
+# Backward pass (gradients of the forward above), for the attention-backward extension.
+#
+# The pages name an attention backward kernel ("HipKittens: fast and furious AMD
+# kernels", section "Performance results"; "State of the AMD ecosystem" for the SDPA
+# backward baselines) without a formula.  The plain definition: with P the forward's
+# probabilities and dO the gradient of a loss with respect to O,
+#     dP = dO V^T,   delta_i = sum_d dO_id O_id  (= sum_j P_ij dP_ij),
+#     dS = P o (dP - delta),   dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO,
+# and for grouped heads dK, dV of a KV head are summed over its query heads.
+
+def head_backward(qh, kh, vh, doh, causal: bool, scale: float):
+    """One head: returns (dQ [N, D], dK [N, D], dV [N, D]) in fp64."""
+    qh, kh, vh, doh = _as_f64(qh), _as_f64(kh), _as_f64(vh), _as_f64(doh)
+    S = head_scores(qh, kh, causal, scale)
+    m = S.max(axis=1, keepdims=True)
+    E = np.exp(S - m)
+    P = E / E.sum(axis=1, keepdims=True)
+    O = P @ vh
+    dP = doh @ vh.T
+    delta = np.sum(doh * O, axis=1, keepdims=True)
+    dS = P * (dP - delta)
+    return scale * (dS @ kh), scale * (dS.T @ qh), P.T @ doh
+
+
+def attention_backward(q, k, v, do, causal: bool, scale: float):
+    """Gradients of sum(O * do) w.r.t. q [B,Hq,N,D], k and v [B,Hkv,N,D]; fp64.
+
+    Each query head's contributions to its KV head's dK and dV are summed.
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    dq = np.empty_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros((B, Hkv, N, v.shape[3]), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            kh = kv_head(h, Hq, Hkv)
+            gq, gk, gv = head_backward(q[b, h], k[b, kh], v[b, kh], do[b, h], causal, scale)
+            dq[b, h] = gq
+            dk[b, kh] += gk
+            dv[b, kh] += gv
+    return dq, dk, dv
