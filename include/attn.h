@@ -1,5 +1,5 @@
 /*
- * attn.h -- C ABI of the B200 (sm_100a) bf16 attention forward library.
+ * attn.h -- C ABI of the B200 (sm_100a) bf16 attention library (forward and backward).
  *
  * The operation is the tiled attention forward pass named by "HipKittens:
  * fast and furious AMD kernels" (section "Performance results": an attention
@@ -133,6 +133,55 @@ int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float
 
 /* Size in bytes of the array attn_fwd_noalloc uses as its workspace. */
 size_t attn_fwd_noalloc_scratch_bytes(void);
+
+/*
+ * attn_bwd -- enqueue the attention backward pass (gradients of the forward) on `stream`.
+ *
+ * The pages name an attention backward kernel beside the forward ("HipKittens: fast and
+ * furious AMD kernels", section "Performance results") without a formula.  With P the
+ * forward's probabilities (rebuilt from the saved LSE) and dO the gradient of a loss with
+ * respect to O, the library computes the plain definition
+ *
+ *     delta_i = sum_d dO_id O_id,   dS = P o (dO V^T - delta)
+ *     dQ[b,h]    = scale dS K[b,g(h)]
+ *     dK[b,g]    = scale sum over the query heads h of group g of dS^T Q[b,h]
+ *     dV[b,g]    = sum over the query heads h of group g of P^T dO[b,h]
+ *
+ * Arguments (DEVICE pointers; the caller allocates, owns and frees every buffer):
+ *   q, k, v, o, lse   the forward's inputs and outputs, layouts as in attn_fwd     read
+ *                     (o and lse as attn_fwd wrote them for the same q, k, v, causal, scale)
+ *   dout  bf16 [B, Hq,  N, D], contiguous: dL/dO.                                  read
+ *   dq    bf16 [B, Hq,  N, D], contiguous.                           written (every element)
+ *   dk    bf16 [B, Hkv, N, D], contiguous.                           written (every element)
+ *   dv    bf16 [B, Hkv, N, D], contiguous.                           written (every element)
+ *   B, Hq, Hkv, N, D, causal, scale   as in attn_fwd (same limits; additionally
+ *         B * Hq * ceil(N / 128) <= 2^31-1).
+ *   workspace        device pointer, 256-byte aligned, of at least
+ *                    attn_bwd_workspace_bytes(B, Hq, N) bytes (per-row delta and
+ *                    LSE * log2(e)); needs no initialisation; calls sharing it must be
+ *                    ordered (same stream).
+ *   stream  cudaStream_t (void*), as in attn_fwd.  Three kernels are enqueued.
+ *
+ * Errors as in attn_fwd: host checks first (ATTN_ERR_INVALID_ARG also for a null or too
+ * small workspace; ATTN_ERR_MISALIGNED for a tensor pointer not 16-byte aligned, lse not
+ * 4-byte aligned or the workspace not 256-byte aligned); outputs untouched on error.
+ *
+ * Numerics: scores and dP = dO V^T accumulate in fp32 on the tensor cores; P and dS are
+ * rounded to bf16 before the dV, dK and dQ matmuls, which accumulate in fp32 in tensor
+ * memory; the gradients are rounded to bf16 (nearest-even).  Every output row is
+ * produced by one CTA in a fixed order: results are bitwise deterministic.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv,
+             int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_bwd_workspace_bytes -- workspace attn_bwd needs: 2 x B x Hq x ceil(N/128) x 128 x 4
+ * bytes, each half rounded up to 256.  Host-only, no CUDA call; 0 for an empty problem,
+ * -1 on invalid sizes.
+ */
+long long attn_bwd_workspace_bytes(int B, int Hq, int N);
 
 /* Human-readable name of an attn_status_t value (static string, never null). */
 const char* attn_status_string(int status);

@@ -111,3 +111,42 @@ def test_workspace_bytes_host_cases():
     assert attn.attn_fwd_workspace_bytes(1, 2, 128, 80, 0) == -1
     assert attn.attn_fwd_workspace_bytes(4, 16, 2048, 128, 1) == 0   # causal never splits
     assert attn.attn_fwd_workspace_bytes(0, 16, 2048, 128, 0) == 0
+
+
+# ---------------------------------------------------------------- backward entry point
+
+def call_bwd(**kw):
+    args = dict(q=P, k=P, v=P, o=P, lse=P, dout=P, dq=P, dk=P, dv=P, B=1, Hq=2, Hkv=1, N=128, D=128, causal=0,
+                scale=0.125, ws=P, ws_bytes=1 << 20)
+    args.update(kw)
+    return attn.attn_bwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["dout"], args["dq"],
+                         args["dk"], args["dv"], args["B"], args["Hq"], args["Hkv"], args["N"], args["D"],
+                         args["causal"], args["scale"], args["ws"], args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(q=None), INVALID), (dict(dout=None), INVALID), (dict(dq=None), INVALID), (dict(dk=None), INVALID),
+    (dict(dv=None), INVALID), (dict(o=None), INVALID), (dict(lse=None), INVALID), (dict(ws=None), INVALID),
+    (dict(ws_bytes=1024), INVALID), (dict(B=-1), INVALID), (dict(Hq=3, Hkv=2), INVALID),
+    (dict(scale=math.nan), INVALID), (dict(D=80), UNSUPPORTED), (dict(D=256), UNSUPPORTED),
+    (dict(dout=P + 8), MISALIGNED), (dict(dq=P + 2), MISALIGNED), (dict(dk=P + 4), MISALIGNED),
+    (dict(dv=P + 1), MISALIGNED), (dict(lse=P + 2), MISALIGNED), (dict(ws=P + 128), MISALIGNED),
+])
+def test_backward_rejected_before_any_cuda_call(kw, expected):
+    assert call_bwd(**kw) == expected
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(N=0), dict(N=0, q=None, dout=None, ws=None, ws_bytes=0)])
+def test_backward_empty_problem_is_ok_without_launch(kw):
+    assert call_bwd(**kw) == OK
+
+
+def test_backward_workspace_bytes():
+    # two fp32 arrays [B*Hq][N rounded up to 128], each rounded up to 256 bytes
+    assert attn.attn_bwd_workspace_bytes(4, 16, 2048) == 2 * 4 * 16 * 2048 * 4
+    assert attn.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
+    assert attn.attn_bwd_workspace_bytes(1, 3, 129) == 2 * 3 * 256 * 4
+    assert attn.attn_bwd_workspace_bytes(0, 4, 100) == 0
+    assert attn.attn_bwd_workspace_bytes(2, 4, 0) == 0
+    assert attn.attn_bwd_workspace_bytes(-1, 4, 100) == -1
+    assert attn.attn_bwd_workspace_bytes(1, 0, 100) == -1

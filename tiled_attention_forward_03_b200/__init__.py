@@ -1,4 +1,4 @@
-"""bf16 attention forward on B200 (sm_100a): Python binding of the C ABI in include/attn.h.
+"""bf16 attention on B200 (sm_100a), forward and backward: Python binding of the C ABI in include/attn.h.
 
 The binding only marshals arguments: every step of the computation runs in the
 CUDA kernel inside ``libattn_fwd.so``.  There is no CPU fallback; if the library
@@ -6,6 +6,7 @@ cannot be loaded, importing this package raises.
 
     import tiled_attention_forward_03_b200 as attn
     o, lse = attn.forward(q, k, v, causal=True)        # q,k,v: CUDA bf16 [B, H, N, D]
+    dq, dk, dv = attn.backward(q, k, v, o, lse, do, causal=True)
 """
 from __future__ import annotations
 
@@ -21,7 +22,7 @@ __all__ = [
     "attn_fwd_workspace_bytes", "attn_fwd_noalloc", "attn_fwd_noalloc_scratch_bytes",
     "attn_status_string", "attn_last_cuda_error", "attn_device_status", "attn_num_units",
     "attn_version", "attn_selftest_exp2_poly", "attn_selftest_wait_timeout", "forward",
-    "forward_from_host", "device_status",
+    "forward_from_host", "device_status", "attn_bwd", "attn_bwd_workspace_bytes", "backward",
 ]
 
 ATTN_OK = 0
@@ -58,6 +59,10 @@ def _load() -> ctypes.CDLL:
     L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.attn_fwd.restype = i
     L.attn_fwd_ws.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, ctypes.c_size_t, vp]
+    L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, ctypes.c_size_t, vp]
+    L.attn_bwd.restype = i
+    L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
+    L.attn_bwd_workspace_bytes.restype = ctypes.c_longlong
     L.attn_fwd_ws.restype = i
     L.attn_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
     L.attn_fwd_workspace_bytes.restype = ctypes.c_longlong
@@ -103,6 +108,17 @@ def attn_fwd_noalloc(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, stream) -
     """Direct call of the entry point that allocates nothing (its workspace is a static
     device array in the library); for callers that may not allocate device memory."""
     return lib.attn_fwd_noalloc(q, k, v, o, lse, B, Hq, Hkv, N, D, int(bool(causal)), float(scale), stream)
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, causal, scale, workspace, workspace_bytes,
+             stream) -> int:
+    """Direct call of the backward entry point (pointers, sizes and stream as integers)."""
+    return lib.attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, int(bool(causal)), float(scale),
+                        workspace, workspace_bytes, stream)
+
+
+def attn_bwd_workspace_bytes(B: int, Hq: int, N: int) -> int:
+    return lib.attn_bwd_workspace_bytes(B, Hq, N)
 
 
 def attn_fwd_noalloc_scratch_bytes() -> int:
@@ -163,11 +179,12 @@ def _check(t, name, dtype, shape):
 _workspaces: dict = {}
 
 
-def _workspace(device, nbytes: int):
-    """A cached device buffer of at least nbytes for the split-tail schedule (per device)."""
+def _workspace(device, nbytes: int, purpose: str = "fwd"):
+    """A cached device buffer of at least nbytes, per device and purpose ("fwd": the
+    split-tail schedule, "bwd": the backward pass's per-row delta and LSE)."""
     import torch
 
-    key = (device.type, device.index)
+    key = (device.type, device.index, purpose)
     buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
         buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
@@ -243,6 +260,48 @@ def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None,
         lse_host.copy_(lse, non_blocking=True)
     s.synchronize()
     return out_host, lse_host
+
+
+def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None, dq=None, dk=None,
+             dv=None, stream=None):
+    """Attention backward on CUDA tensors: returns (dq, dk, dv), bf16, shaped like q, k, v.
+
+    ``o`` and ``lse`` are the forward's outputs for the same q, k, v, causal and scale;
+    ``dout`` is the bf16 gradient of the loss with respect to o.  The workspace (per-row
+    delta and LSE) is cached per device; calls sharing it are ordered on one stream.
+    """
+    import torch
+
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, N, D]")
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    _check(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _check(k, "k", torch.bfloat16, (B, Hkv, N, D))
+    _check(v, "v", torch.bfloat16, (B, Hkv, N, D))
+    _check(o, "o", torch.bfloat16, (B, Hq, N, D))
+    _check(lse, "lse", torch.float32, (B, Hq, N))
+    _check(dout, "dout", torch.bfloat16, (B, Hq, N, D))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(dq, "dq", torch.bfloat16, (B, Hq, N, D))
+    _check(dk, "dk", torch.bfloat16, (B, Hkv, N, D))
+    _check(dv, "dv", torch.bfloat16, (B, Hkv, N, D))
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        ws_bytes = attn_bwd_workspace_bytes(B, Hq, N)
+        if ws_bytes < 0:
+            raise AttnError(ATTN_ERR_INVALID_ARG, "attn_bwd_workspace_bytes")
+        ws = _workspace(q.device, max(ws_bytes, 256), "bwd")
+        st = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, N, D, causal, scale,
+                      ws.data_ptr(), ws.numel(), s.cuda_stream)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
 
 
 def device_status(stream=None):

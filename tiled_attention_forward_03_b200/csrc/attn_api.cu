@@ -1,8 +1,8 @@
 // attn_api.cu -- host side of the C ABI declared in include/attn.h.
 //
-// Validates arguments before any CUDA call, encodes the TMA tensor maps for Q, K
-// and V, sizes the persistent grid to the SM count and launches the sm_100a kernel
-// on the caller's stream.  Nothing is allocated per call.
+// Validates arguments before any CUDA call, encodes the TMA tensor maps, sizes the
+// grids to the problem and the SM count and launches the sm_100a kernels on the
+// caller's stream.  Nothing is allocated per call.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -16,6 +16,7 @@
 
 #include "attn.h"
 #include "attn_fwd_kernel.cuh"
+#include "attn_bwd_kernel.cuh"
 
 #define ATTN_VERSION_STRING "b200-attn 0.1 (sm_100a, tcgen05/TMA/TMEM)"
 
@@ -431,6 +432,147 @@ int attn_selftest_wait_timeout(unsigned int timeout_us, void* stream) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     record_cuda_error("selftest_wait_timeout launch", e);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Backward pass.
+
+namespace {
+
+struct BwdDeviceInfo {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+};
+BwdDeviceInfo g_bwd_dev[kMaxDevices];
+
+template <int D>
+cudaError_t bwd_setup_dim() {
+  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_bwd_sm100<D, true>),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, attn::BwdPlan<D>::kAlloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_bwd_sm100<D, false>),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, attn::BwdPlan<D>::kAlloc);
+  return e;
+}
+
+bool bwd_device_setup(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  BwdDeviceInfo& d = g_bwd_dev[dev];
+  std::call_once(d.once, [&d] {
+    cudaError_t e = bwd_setup_dim<32>();
+    if (e == cudaSuccess) e = bwd_setup_dim<64>();
+    if (e == cudaSuccess) e = bwd_setup_dim<96>();
+    if (e == cudaSuccess) e = bwd_setup_dim<128>();
+    d.err = e;
+  });
+  if (d.err != cudaSuccess) {
+    record_cuda_error("backward device setup", d.err);
+    return false;
+  }
+  return true;
+}
+
+// Workspace layout: lse2 then delta, each [B*Hq][Npad] fp32 (Npad = N rounded up to 128),
+// each part 256-byte aligned.
+size_t bwd_part_bytes(long long B, int Hq, int N) {
+  const long long npad = ((long long)N + attn::kBlockN - 1) / attn::kBlockN * attn::kBlockN;
+  return ((size_t)B * Hq * npad * sizeof(float) + 255) / 256 * 256;
+}
+
+template <int D>
+void launch_bwd_dim(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                    const attn::BwdParams& p, long long grid_kv, long long grid_q, cudaStream_t s) {
+  attn::attn_bwd_sm100<D, true><<<(unsigned)grid_kv, attn::kBwdThreads, attn::BwdPlan<D>::kAlloc, s>>>(
+      mk, mv, mq, mdo, p);
+  attn::attn_bwd_sm100<D, false><<<(unsigned)grid_q, attn::kBwdThreads, attn::BwdPlan<D>::kAlloc, s>>>(
+      mq, mdo, mk, mv, p);
+}
+
+}  // namespace
+
+extern "C" {
+
+long long attn_bwd_workspace_bytes(int B, int Hq, int N) {
+  if (B < 0 || Hq < 1 || N < 0) return -1;
+  if (B == 0 || N == 0) return 0;
+  return (long long)(2 * bwd_part_bytes(B, Hq, N));
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  // ---- host-side validation (no CUDA call before this block passes)
+  if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
+    return ATTN_ERR_INVALID_ARG;
+  if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq * (((long long)N + attn::kBlockN - 1) / attn::kBlockN) > 0x7fffffffLL)
+    return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return ATTN_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 256))
+    return ATTN_ERR_MISALIGNED;
+  const size_t part = bwd_part_bytes(B, Hq, N);
+  if (workspace_bytes < 2 * part) return ATTN_ERR_INVALID_ARG;
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    record_cuda_error("cudaGetDevice", e);
+    return ATTN_ERR_CUDA;
+  }
+  if (!bwd_device_setup(dev)) return ATTN_ERR_CUDA;
+
+  CUtensorMap mq, mk, mv, mdo;
+  int st;
+  if ((st = encode_map(&mq, q, (long long)B * Hq, N, D)) != ATTN_OK) return st;
+  if ((st = encode_map(&mk, k, (long long)B * Hkv, N, D)) != ATTN_OK) return st;
+  if ((st = encode_map(&mv, v, (long long)B * Hkv, N, D)) != ATTN_OK) return st;
+  if ((st = encode_map(&mdo, dout, (long long)B * Hq, N, D)) != ATTN_OK) return st;
+
+  const int nb = (int)(((long long)N + attn::kBlockN - 1) / attn::kBlockN);
+  attn::BwdParams p;
+  p.dq = reinterpret_cast<__nv_bfloat16*>(dq);
+  p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  float* lse2 = reinterpret_cast<float*>(workspace);
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + part);
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.Npad = nb * attn::kBlockN;
+  p.group = Hq / Hkv;
+  p.num_blocks = nb;
+  p.causal = causal ? 1 : 0;
+  p.c = scale * attn::kLog2e;
+  p.scale = scale;
+  p.idesc_s = attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, false);
+  p.idesc_acc = attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long rows = (long long)B * Hq * p.Npad;
+  const int prep_threads = 256;
+  const long long prep_blocks = (rows + prep_threads / 16 - 1) / (prep_threads / 16);
+  attn::attn_bwd_prep<<<(unsigned)prep_blocks, prep_threads, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
+      rows, N, p.Npad, D);
+  const long long grid_kv = (long long)B * Hkv * nb, grid_q = (long long)B * Hq * nb;
+  switch (D) {
+    case 32: launch_bwd_dim<32>(mq, mk, mv, mdo, p, grid_kv, grid_q, s); break;
+    case 64: launch_bwd_dim<64>(mq, mk, mv, mdo, p, grid_kv, grid_q, s); break;
+    case 96: launch_bwd_dim<96>(mq, mk, mv, mdo, p, grid_kv, grid_q, s); break;
+    default: launch_bwd_dim<128>(mq, mk, mv, mdo, p, grid_kv, grid_q, s); break;
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    record_cuda_error("backward kernel launch", e);
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;

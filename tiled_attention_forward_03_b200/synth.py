@@ -98,6 +98,14 @@ def make_qkv(B: int, Hq: int, Hkv: int, N: int, D: int, seed: int):
     return q, k, v
 
 
+def make_dout(B: int, Hq: int, N: int, D: int, seed: int):
+    """Draw the upstream gradient dL/dO as a contiguous CPU bfloat16 tensor [B, Hq, N, D]
+    (i.i.d. N(0, 1) in fp32, rounded to bf16), from its own seed."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return torch.randn((B, Hq, N, D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
 def make_workload_inputs(w: Workload):
     return make_qkv(w.B, w.Hq, w.Hkv, w.N, w.D, w.seed)
 
