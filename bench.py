@@ -2,6 +2,7 @@
 """Benchmark of the B200 bf16 attention forward (TFLOP/s, % of the dense BF16 peak).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all] [--impl ours|reference]
+                    [--pass fwd|bwd]
 
 One step = one attention forward pass over the workload's batch (one kernel
 launch).  Default workload: B=4, Hq=Hkv=16, N=2048, D=128, non-causal, bf16
@@ -14,6 +15,11 @@ throughput (all ranks' FLOPs / the slowest rank's time).  With N>1 GPUs
 (torchrun), every rank runs its own batch of the workload (weak scaling): the
 query heads are independent, so no collective touches the data path; NCCL only
 carries the barrier and the max-over-ranks timing.
+
+`--pass bwd` times the backward pass instead (one step = one attn_bwd call: the prep,
+dK/dV and dQ launches), on the forward's o and lse computed once before timing; its
+FLOP count is 2.5x the forward's (the five N x N x D matmuls of the gradient), the
+usual convention.
 
 `--impl reference` times the fp64 CPU oracle instead (the only other
 implementation of this path): each step is a bounded sample of the workload's
@@ -39,6 +45,9 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 DEFAULT_WORKLOAD = "cfg2"
 METRIC = "attention fwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
+METRIC_BWD = "attention bwd TFLOP/s (bf16, 1 B200; 2.5x the forward FLOP count) and % of dense BF16 tensor peak"
+BWD_FLOP_RATIO = 2.5      # counted backward FLOPs / forward FLOPs (five matmuls against two)
+BWD_EXECUTED_RATIO = 7 / 5  # matmuls the kernels execute / matmuls counted (S and dP run twice)
 L2_FLUSH_BYTES = 512 << 20
 CPU_SAMPLE_SECONDS = 12.0
 
@@ -163,9 +172,10 @@ def physical_gpu_index(local_rank: int) -> int:
     return local_rank
 
 
-def profile_traffic(workload_name: str):
-    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload_name}_dram.json")
+def profile_traffic(workload_name: str, which: str = "fwd"):
+    """DRAM bytes per launch (per call for the backward) from the committed ncu summary, if
+    it matches the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"attn_{which}_{workload_name}_dram.json")
     try:
         with open(path) as f:
             d = json.load(f)
@@ -194,21 +204,26 @@ def cpu_threads():
     return len(os.sched_getaffinity(0))
 
 
-def time_oracle(w, seconds: float, heads: int | None = None):
-    """Run the fp64 oracle on whole heads of workload w for about `seconds` (or `heads` heads).
+def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = False):
+    """Run the fp64 oracle on whole heads of workload w for about `seconds` (or `heads` heads);
+    the forward, or with `backward` the gradients of one query head.
 
     Returns (TFLOP/s, FLOPs done, seconds, heads done, sample description)."""
-    from oracle import head_forward
-    from tiled_attention_forward_03_b200.synth import make_qkv
+    from oracle import head_backward, head_forward
+    from tiled_attention_forward_03_b200.synth import make_dout, make_qkv
 
     q, k, v = make_qkv(1, w.Hq, w.Hkv, w.N, w.D, w.seed)  # one batch row holds all heads
+    do = make_dout(1, w.Hq, w.N, w.D, w.seed + 500) if backward else None
     g = w.Hq // w.Hkv
-    per_head = w.flops / (w.B * w.Hq)
+    per_head = w.flops / (w.B * w.Hq) * (BWD_FLOP_RATIO if backward else 1.0)
     done = 0
     t0 = time.perf_counter()
     while True:
         h = done % w.Hq
-        head_forward(q[0, h], k[0, h // g], v[0, h // g], w.causal, w.softmax_scale)
+        if backward:
+            head_backward(q[0, h], k[0, h // g], v[0, h // g], do[0, h], w.causal, w.softmax_scale)
+        else:
+            head_forward(q[0, h], k[0, h // g], v[0, h // g], w.causal, w.softmax_scale)
         done += 1
         el = time.perf_counter() - t0
         if heads is not None and done >= heads:
@@ -216,8 +231,9 @@ def time_oracle(w, seconds: float, heads: int | None = None):
         if heads is None and el >= seconds:
             break
     tflops = per_head * done / el / 1e12
-    sample = (f"{done} of {w.B * w.Hq} heads of {w.name} (each head's full {w.N}x{w.N} fp64 score matrix), "
-              f"{el:.1f} s")
+    what = "gradients" if backward else "forward"
+    sample = (f"{what} of {done} heads, cycling over the {w.Hq} query heads of one batch row of {w.name} "
+              f"(each head's full {w.N}x{w.N} fp64 score matrix), {el:.1f} s")
     return tflops, per_head * done, el, done, sample
 
 
@@ -226,13 +242,14 @@ def time_oracle(w, seconds: float, heads: int | None = None):
 def run_ours(args, w):
     import torch
 
+    backward = args.pass_ == "bwd"
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     dist = init_dist(world, "nccl")
 
     import tiled_attention_forward_03_b200 as attn
-    from tiled_attention_forward_03_b200.synth import make_qkv
+    from tiled_attention_forward_03_b200.synth import make_dout, make_qkv
 
     q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.D, rank_seed(w.seed, rank))
     qd, kd, vd = (x.to(device) for x in (q, k, v))
@@ -242,8 +259,19 @@ def run_ours(args, w):
     stream = torch.cuda.current_stream(device)
     scale = w.softmax_scale
 
-    def step():
+    if backward:
+        # the backward consumes the forward's saved o and lse: computed once, untimed
+        do = make_dout(w.B, w.Hq, w.N, w.D, rank_seed(w.seed + 500, rank))
+        dod = do.to(device)
         attn.forward(qd, kd, vd, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
+        dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+
+        def step():
+            attn.backward(qd, kd, vd, o, lse, dod, causal=w.causal, scale=scale, dq=dq, dk=dk, dv=dv,
+                          stream=stream)
+    else:
+        def step():
+            attn.forward(qd, kd, vd, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -275,21 +303,38 @@ def run_ours(args, w):
         raise RuntimeError(f"kernel wait gave up during timing (site {site})")
 
     # ---- end to end through the public host-buffer call
-    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
-    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     e2e_steps = max(3, min(args.steps, 20))
+    if backward:
+        host_in = tuple(x.pin_memory() for x in (q, k, v, o.cpu(), lse.cpu(), do))
+        host_out = tuple(torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (dq, dk, dv))
+
+        def e2e_call():
+            attn.backward_from_host(*host_in, causal=w.causal, scale=scale, device=device, out_host=host_out,
+                                    stream=stream)
+        h2d = sum(x.numel() * x.element_size() for x in host_in)
+        d2h = sum(x.numel() * x.element_size() for x in host_out)
+        e2e_path = ("backward_from_host: pinned host q,k,v,o,lse,dO -> device, attn_bwd, "
+                    "dq,dk,dv -> pinned host")
+    else:
+        qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+        oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e_call():
+            attn.forward_from_host(qh, kh, vh, causal=w.causal, scale=scale, device=device, out_host=oh,
+                                   lse_host=lh, stream=stream)
+        h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
+        d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+        e2e_path = "forward_from_host: pinned host q,k,v -> device, attn_fwd, o,lse -> pinned host"
     for _ in range(2):
-        attn.forward_from_host(qh, kh, vh, causal=w.causal, scale=scale, device=device, out_host=oh,
-                               lse_host=lh, stream=stream)
+        e2e_call()
     barrier(dist, device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(device)
     e0.record(stream)
     for _ in range(e2e_steps):
-        attn.forward_from_host(qh, kh, vh, causal=w.causal, scale=scale, device=device, out_host=oh,
-                               lse_host=lh, stream=stream)
+        e2e_call()
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
@@ -301,16 +346,24 @@ def run_ours(args, w):
         return None
 
     peak_burst, peak_sustained, hbm, peak_kind = measured_peaks()
-    flops_step = w.flops
+    flops_step = w.flops * (BWD_FLOP_RATIO if backward else 1.0)
     value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
     achieved = flops_step / (statistics.mean(kernel_ms) * 1e-3) / 1e12
     e2e_value = world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
-    h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
-    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-    traffic = profile_traffic(w.name)
+    traffic = profile_traffic(w.name, "bwd" if backward else "fwd")
+    if backward:
+        kernel = (f"attn_bwd call: attn_bwd_prep + attn_bwd_sm100<{w.D}, dK/dV> + attn_bwd_sm100<{w.D}, dQ>, "
+                  f"timed together")
+        # read q, o, dO (query heads), k, v (KV heads), lse; write dq, dk, dv; all bf16 but lse
+        q_side = w.B * w.Hq * w.N * w.D * 2
+        kv_side = w.B * w.Hkv * w.N * w.D * 2
+        algo_bytes = 4 * q_side + 4 * kv_side + 4 * w.B * w.Hq * w.N
+    else:
+        kernel = f"attn_fwd_sm100<{w.D}>"
+        algo_bytes = w.algorithmic_bytes
 
     line = {
-        "metric": METRIC,
+        "metric": METRIC_BWD if backward else METRIC,
         "value": round(value, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -322,23 +375,27 @@ def run_ours(args, w):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {**w.describe(), "l2": "flushed between timed steps (512 MB write)",
+        "config": {**w.describe(), "pass": "backward" if backward else "forward",
+                   "l2": "flushed between timed steps (512 MB write)",
                    "parallelism": f"replicas{world}: each rank its own batch, no collective on the data path"},
         "pct_of_dense_bf16_peak": round(100.0 * value / world / DATASHEET_BF16_TFLOPS, 2),
         "pct_of_measured_bf16_peak": round(100.0 * value / world / peak_burst, 2),
-        "hbm_gbs_algorithmic": round(w.algorithmic_bytes / (statistics.mean(kernel_ms) * 1e-3) / 1e9, 1),
+        "hbm_gbs_algorithmic": round(algo_bytes / (statistics.mean(kernel_ms) * 1e-3) / 1e9, 1),
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "path": "forward_from_host: pinned host q,k,v -> device, attn_fwd, o,lse -> pinned host"},
-        "gpu_launches": args.steps,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps, "path": e2e_path},
+        "gpu_launches": args.steps * (3 if backward else 1),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_burst,
                      "unit": "TFLOP/s", "frac": round(achieved / peak_burst, 4), "traffic": traffic,
                      "peak_kind": f"{peak_kind} bf16 matmul, burst (kernel timed alone)",
-                     "kernel": f"attn_fwd_sm100<{w.D}>"},
+                     "kernel": kernel},
     }
+    if backward:
+        line["roofline"]["executed_tflops"] = round(achieved * BWD_EXECUTED_RATIO, 2)
+        line["roofline"]["executed_note"] = ("the kernels run 7 N x N x D matmuls where 5 are counted "
+                                             "(scores and dP are formed in both the dK/dV and dQ kernels)")
     if world == 1 and not args.no_cpu_baseline:
-        tf, _, el, done, sample = time_oracle(w, CPU_SAMPLE_SECONDS)
+        tf, _, el, done, sample = time_oracle(w, CPU_SAMPLE_SECONDS, backward=backward)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                                 "sample": sample}
     if dist is not None:
@@ -352,19 +409,21 @@ def run_reference(args, w):
     world, rank, _ = dist_env()
     if rank != 0:
         return None
+    backward = args.pass_ == "bwd"
     per_step = []
     for i in range(args.warmup + args.steps):
-        tf, flops, el, done, sample = time_oracle(w, 0.0, heads=1)
+        tf, flops, el, done, sample = time_oracle(w, 0.0, heads=1, backward=backward)
         if i >= args.warmup:
             per_step.append((flops, el))
     flops = sum(f for f, _ in per_step)
     secs = sum(e for _, e in per_step)
     value = flops / secs / 1e12
     cores = cpu_threads()
-    sample = f"one head of {w.name} per step (full {w.N}x{w.N} fp64 score matrix), {args.steps} steps"
+    what = "gradients of one head" if backward else "one head"
+    sample = f"{what} of {w.name} per step (full {w.N}x{w.N} fp64 score matrix), {args.steps} steps"
     return {
         "impl": "reference",
-        "metric": METRIC,
+        "metric": METRIC_BWD if backward else METRIC,
         "value": value,
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -376,7 +435,7 @@ def run_reference(args, w):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": w.describe(),
+        "config": {**w.describe(), "pass": "backward" if backward else "forward"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -391,6 +450,8 @@ def main(argv=None):
                     help="cfg1..cfg4, a sweep point name (e.g. sweep_D128_N8192_causal), or 'all'")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
+                    help="fwd: the attention forward (default); bwd: the backward pass (attn_bwd)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

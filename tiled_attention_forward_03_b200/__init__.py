@@ -23,6 +23,7 @@ __all__ = [
     "attn_status_string", "attn_last_cuda_error", "attn_device_status", "attn_num_units",
     "attn_version", "attn_selftest_exp2_poly", "attn_selftest_wait_timeout", "forward",
     "forward_from_host", "device_status", "attn_bwd", "attn_bwd_workspace_bytes", "backward",
+    "backward_from_host",
 ]
 
 ATTN_OK = 0
@@ -302,6 +303,26 @@ def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
     if st != ATTN_OK:
         raise AttnError(st, "attn_bwd")
     return dq, dk, dv
+
+
+def backward_from_host(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None, device=None,
+                       out_host=None, stream=None):
+    """End-to-end backward on host (ideally pinned) tensors: copy q, k, v, o, lse and dout in,
+    run attn_bwd, copy dq, dk, dv out.  Returns host tensors (dq, dk, dv); ``out_host`` may
+    hold three preallocated host tensors for them.  Returns after the copies completed."""
+    import torch
+
+    dev = torch.device(device if device is not None else "cuda")
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    with torch.cuda.stream(s):
+        qd, kd, vd, od, ld, dd = (x.to(dev, non_blocking=True) for x in (q, k, v, o, lse, dout))
+        grads = backward(qd, kd, vd, od, ld, dd, causal=causal, scale=scale, stream=s)
+        if out_host is None:
+            out_host = tuple(torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads)
+        for h, g in zip(out_host, grads):
+            h.copy_(g, non_blocking=True)
+    s.synchronize()
+    return tuple(out_host)
 
 
 def device_status(stream=None):
