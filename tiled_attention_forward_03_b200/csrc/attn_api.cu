@@ -477,7 +477,7 @@ bool bwd_device_setup(int dev) {
   return true;
 }
 
-// Workspace layout: lse2 then delta, each [B*Hq][Npad] fp32 (Npad = N rounded up to 128),
+// Workspace layout: -lse2 then -delta, each [B*Hq][Npad] fp32 (Npad = N rounded up to 128),
 // each part 256-byte aligned.
 size_t bwd_part_bytes(long long B, int Hq, int N) {
   const long long npad = ((long long)N + attn::kBlockN - 1) / attn::kBlockN * attn::kBlockN;
@@ -540,10 +540,10 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   p.dq = reinterpret_cast<__nv_bfloat16*>(dq);
   p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
   p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
-  float* lse2 = reinterpret_cast<float*>(workspace);
-  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + part);
-  p.lse2 = lse2;
-  p.delta = delta;
+  float* nlse2 = reinterpret_cast<float*>(workspace);
+  float* ndelta = reinterpret_cast<float*>(static_cast<char*>(workspace) + part);
+  p.nlse2 = nlse2;
+  p.ndelta = ndelta;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.N = N;
@@ -561,7 +561,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   const int prep_threads = 256;
   const long long prep_blocks = (rows + prep_threads / 16 - 1) / (prep_threads / 16);
   attn::attn_bwd_prep<<<(unsigned)prep_blocks, prep_threads, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
+      reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), lse, nlse2, ndelta,
       rows, N, p.Npad, D);
   const long long grid_kv = (long long)B * Hkv * nb, grid_q = (long long)B * Hq * nb;
   switch (D) {

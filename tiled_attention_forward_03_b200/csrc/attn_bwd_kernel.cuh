@@ -39,16 +39,19 @@
 //   warp  9    MMA issuer (one elected lane)
 //
 // Tensor memory (512 columns):
-//   [  0,128) S fp32; P (bf16 pairs, KV pass) overwrites columns [0,32) and [64,96)
-//   [128,256) dP fp32; dS (bf16 pairs) overwrites columns [128,160) and [192,224)
+//   [  0,128) S fp32 (released to the next tile's S as soon as the softmax has loaded it)
+//   [128,256) dP fp32; once loaded, each softmax warpgroup writes into its 64 columns
+//             P (bf16 pairs, KV pass) over the first 32 and dS (bf16 pairs) over the second 32
 //   [256,256+D) acc_p (dV);  [384,384+D) acc_ds (dK or dQ)
-// Each softmax warpgroup writes its packed P / dS over the first half of the columns it
-// has just read, so the two warpgroups never touch each other's columns.
+// The two warpgroups never touch each other's columns.
 //
 // MMA order per column tile t (tcgen05 MMAs of one CTA run in issue order):
-//   acc_p(t)  S(t+1)  acc_ds(t)  dP(t+1)
-// S(t+1) overwrites P(t) only after acc_p(t) has read it, and dP(t+1) overwrites dS(t)
-// only after acc_ds(t); the softmax of t+1 (exponentials) overlaps acc_ds(t) and dP(t+1).
+//   S(t+1)  acc_ds(t)  acc_p(t)  dP(t+1)
+// S(t+1) is issued once the softmax holds S(t) in registers, so the exponentials of tile
+// t+1 overlap all of tile t's gradient matmuls; dP(t+1) overwrites dS(t) and P(t) only
+// after the MMAs reading them.  C0 and C1 tiles have rings of their own, each stage
+// refilled as soon as its last reader has completed (C0 after acc_ds, C1 after acc_p, or
+// after dP in the Q pass), so the next tiles are in flight while the current ones are used.
 //
 // Every wait is bounded, as in the forward kernel.
 #pragma once
@@ -61,6 +64,11 @@ namespace attn {
 
 constexpr int kBwdThreads = 320;
 constexpr float kLog2e = 1.4426950408889634f;
+// Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial (exp2_poly2)
+// instead of the special-function unit.  Measured on B200: none is best here (the
+// backward's exponentials are not the limit; the polynomial's FMA work only delays P).
+template <int D, bool kKV>
+__host__ __device__ constexpr int bwd_poly_pairs_per8() { return 0; }
 
 enum : unsigned {
   kSiteBwdProducer = 12,
@@ -94,8 +102,9 @@ struct BwdPlan {
   static constexpr int kVecOff = kCOff + kStages * 2 * kTileBytes;  // per stage: lse2[128], delta[128]
   static constexpr int kVecBytes = 2 * kBlockN * 4;
   static constexpr int kBarOff = kVecOff + kStages * kVecBytes;
-  // r_full c_full[S] c_empty[S] s_full dp_full p_ready ds_ready acc_full drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 6;
+  // r_full c0_full[S] c0_empty[S] c1_full[S] c1_empty[S] s_full s_free dp_full p_ready ds_ready
+  // acc_full drain
+  static constexpr int kNumBars = 1 + 4 * kStages + 7;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -105,8 +114,8 @@ struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  const float* lse2;    // [B*Hq][Npad] LSE * log2(e)
-  const float* delta;   // [B*Hq][Npad] rowsum(dO o O)
+  const float* nlse2;   // [B*Hq][Npad] -LSE * log2(e)
+  const float* ndelta;  // [B*Hq][Npad] -rowsum(dO o O)
   int Hq, Hkv, N, Npad, group, num_blocks;
   int causal;
   float c;              // scale * log2(e)
@@ -115,11 +124,12 @@ struct BwdParams {
   uint32_t idesc_acc;   // 128 x D x 128, A from TMEM, B MN-major
 };
 
-// delta_i = sum_d dO_id O_id (fp32 sums of the bf16 products) and lse2_i = LSE_i log2(e),
-// one 16-thread group per row of the padded [B*Hq][Npad] layout; pad rows get 0.
+// -delta_i = -sum_d dO_id O_id (fp32 sums of the bf16 products) and -lse2_i = -LSE_i log2(e),
+// one 16-thread group per row of the padded [B*Hq][Npad] layout; pad rows get 0.  (Stored
+// negated so that the kernels add them with paired fp32 instructions.)
 __global__ void attn_bwd_prep(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-                              const float* __restrict__ lse, float* __restrict__ lse2,
-                              float* __restrict__ delta, long long rows, int N, int Npad, int D) {
+                              const float* __restrict__ lse, float* __restrict__ nlse2,
+                              float* __restrict__ ndelta, long long rows, int N, int Npad, int D) {
   const long long row = (long long)blockIdx.x * (blockDim.x >> 4) + (threadIdx.x >> 4);
   const int l16 = threadIdx.x & 15;
   if (row >= rows) return;  // whole 16-lane groups leave together
@@ -148,8 +158,8 @@ __global__ void attn_bwd_prep(const __nv_bfloat16* __restrict__ o, const __nv_bf
   acc += __shfl_xor_sync(mask, acc, 2, 16);
   acc += __shfl_xor_sync(mask, acc, 1, 16);
   if (l16 == 0) {
-    delta[row] = acc;
-    lse2[row] = qi < N ? lse[(size_t)bh * N + qi] * kLog2e : 0.f;
+    ndelta[row] = -acc;
+    nlse2[row] = qi < N ? -lse[(size_t)bh * N + qi] * kLog2e : 0.f;
   }
 }
 
@@ -214,14 +224,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* sVec = reinterpret_cast<float*>(smem + Plan::kVecOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kBarOff);
   uint64_t* r_full = bars;
-  uint64_t* c_full = bars + 1;
-  uint64_t* c_empty = bars + 1 + S;
-  uint64_t* s_full = bars + 1 + 2 * S;
-  uint64_t* dp_full = s_full + 1;
-  uint64_t* p_ready = s_full + 2;
-  uint64_t* ds_ready = s_full + 3;
-  uint64_t* acc_full = s_full + 4;
-  uint64_t* drain = s_full + 5;
+  uint64_t* c0_full = bars + 1;
+  uint64_t* c0_empty = c0_full + S;
+  uint64_t* c1_full = c0_full + 2 * S;
+  uint64_t* c1_empty = c0_full + 3 * S;
+  uint64_t* s_full = c0_full + 4 * S;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* dp_full = s_full + 2;
+  uint64_t* p_ready = s_full + 3;
+  uint64_t* ds_ready = s_full + 4;
+  uint64_t* acc_full = s_full + 5;
+  uint64_t* drain = s_full + 6;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Plan::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Plan::kMiscOff + 4);
 
@@ -232,10 +245,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(r_full, 1);
     for (int i = 0; i < S; ++i) {
-      mbar_init(&c_full[i], 1);
-      mbar_init(&c_empty[i], 1);
+      mbar_init(&c0_full[i], 1);
+      mbar_init(&c0_empty[i], 1);
+      mbar_init(&c1_full[i], 1);
+      mbar_init(&c1_empty[i], 1);
     }
     mbar_init(s_full, 1);
+    mbar_init(s_free, 256);
     mbar_init(dp_full, 1);
     mbar_init(p_ready, 256);
     mbar_init(ds_ready, 256);
@@ -261,6 +277,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
+    // Two rings of S stages: C0 tiles (with the KV pass's per-query vectors) and C1 tiles,
+    // each refilled as soon as the MMAs that read it have completed.
     if (lane == 0) {
       const uint64_t pol_once = l2_policy_evict_first();
       const uint64_t pol_shared = l2_policy_evict_last();
@@ -275,32 +293,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       Ring ring;
       uint32_t filled = 0u, fill_par = 0u;
       for (int it = 0; it < w.n; ++it) {
-        if (!wait_phase(&c_empty[ring.stage], ring.phase ^ 1u, abort_flag, kSiteBwdProducer)) break;
         int cb, chead;
         bwd_col<kKV>(p, w, it, cb, chead);
-        uint64_t* bar = &c_full[ring.stage];
-        mbar_arrive_expect_tx(bar, 2 * Plan::kTileBytes + (kKV ? Plan::kVecBytes : 0));
         uint8_t* dst = sC + ring.stage * 2 * Plan::kTileBytes;
-        load_tile(&tmap_c0, dst, bar, cb * kBlockN, chead, pol_shared);
-        load_tile(&tmap_c1, dst + Plan::kTileBytes, bar, cb * kBlockN, chead, pol_shared);
+        if (!wait_phase(&c0_empty[ring.stage], ring.phase ^ 1u, abort_flag, kSiteBwdProducer)) break;
+        uint64_t* bar0 = &c0_full[ring.stage];
+        mbar_arrive_expect_tx(bar0, Plan::kTileBytes + (kKV ? Plan::kVecBytes : 0));
+        load_tile(&tmap_c0, dst, bar0, cb * kBlockN, chead, pol_shared);
         if (kKV) {
           const size_t off = (size_t)chead * p.Npad + (size_t)cb * kBlockN;
           float* vec = sVec + ring.stage * 2 * kBlockN;
-          bulk_load_1d(vec, p.lse2 + off, kBlockN * 4, bar);
-          bulk_load_1d(vec + kBlockN, p.delta + off, kBlockN * 4, bar);
+          bulk_load_1d(vec, p.nlse2 + off, kBlockN * 4, bar0);
+          bulk_load_1d(vec + kBlockN, p.ndelta + off, kBlockN * 4, bar0);
         }
+        if (!wait_phase(&c1_empty[ring.stage], ring.phase ^ 1u, abort_flag, kSiteBwdProducer)) {
+          filled |= 1u << ring.stage;
+          fill_par = (fill_par & ~(1u << ring.stage)) | (ring.phase << ring.stage);
+          break;
+        }
+        uint64_t* bar1 = &c1_full[ring.stage];
+        mbar_arrive_expect_tx(bar1, Plan::kTileBytes);
+        load_tile(&tmap_c1, dst + Plan::kTileBytes, bar1, cb * kBlockN, chead, pol_shared);
+        filled |= 1u << (S + ring.stage);
         filled |= 1u << ring.stage;
         fill_par = (fill_par & ~(1u << ring.stage)) | (ring.phase << ring.stage);
         ring.advance<S>();
       }
       // Drain: every issued copy lands before the CTA may exit.
       drain_phase(r_full, 0u, abort_flag);
-      for (int s = 0; s < S; ++s)
-        if (filled & (1u << s)) drain_phase(&c_full[s], (fill_par >> s) & 1u, abort_flag);
+      for (int s = 0; s < S; ++s) {
+        if (filled & (1u << s)) drain_phase(&c0_full[s], (fill_par >> s) & 1u, abort_flag);
+        if (filled & (1u << (S + s))) drain_phase(&c1_full[s], (fill_par >> s) & 1u, abort_flag);
+      }
     }
     __syncwarp();
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    // Per column tile t (tcgen05 MMAs of one CTA run in issue order):
+    //   S(t+1) once the softmax has S(t) in registers;
+    //   acc_ds(t) once dS(t) is in TMEM, then C0(t) is released;
+    //   acc_p(t) (KV pass) once P(t) is in TMEM, then C1(t) is released;
+    //   dP(t+1), which overwrites the dP columns holding dS(t) and P(t).
+    // The Q pass releases C1(t) as soon as dP(t) has completed (its only reader).
     const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_base, 0);
     const uint64_t desc_r0 = smem_desc_kmajor_sw128(smem_u32(sR));
     const uint64_t desc_r1 = smem_desc_kmajor_sw128(smem_u32(sR + Plan::kTileBytes));
@@ -318,8 +352,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       __syncwarp();
     };
-    // acc (+)= X C over the 128 tile columns (X bf16 pairs in TMEM at columns a_col + [0,32)
-    // and a_col + 64 + [0,32); C MN-major in shared memory).
+    // acc (+)= X C over the 128 tile columns: X bf16 pairs in TMEM at columns a_col + [0,32)
+    // (tile columns 0-63) and a_col + 64 + [0,32) (tile columns 64-127); C MN-major in smem.
     auto issue_acc = [&](uint32_t d_col, uint32_t a_col, uint64_t db, bool accumulate) {
       if (elect_one()) {
 #pragma unroll
@@ -337,39 +371,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool mine = wait_phase(bar, parity, abort_flag, site);
       return __all_sync(0xffffffffu, mine);
     };
-    auto stage_bytes = [](uint32_t st) -> uint32_t { return st * 2 * Plan::kTileBytes; };
+    auto c0_bytes = [](uint32_t st) -> uint32_t { return st * 2 * Plan::kTileBytes; };
+    auto c1_bytes = [](uint32_t st) -> uint32_t { return st * 2 * Plan::kTileBytes + Plan::kTileBytes; };
 
     bool ok = wait_all(r_full, 0u, kSiteBwdMmaRow);
     Ring ring;
-    if (ok && w.n > 0) ok = wait_all(&c_full[0], 0u, kSiteBwdMmaCol);
+    if (ok && w.n > 0) ok = wait_all(&c0_full[0], 0u, kSiteBwdMmaCol);
     if (ok && w.n > 0) {
       tc_fence_after();
-      issue_rc(0, desc_r0, adv(desc_c_k, stage_bytes(0)));
+      issue_rc(0, desc_r0, adv(desc_c_k, c0_bytes(0)));
       commit(s_full);
-      issue_rc(128, desc_r1, adv(desc_c_k, stage_bytes(0) + Plan::kTileBytes));
+      ok = wait_all(&c1_full[0], 0u, kSiteBwdMmaCol);
+    }
+    if (ok && w.n > 0) {
+      tc_fence_after();
+      issue_rc(128, desc_r1, adv(desc_c_k, c1_bytes(0)));
       commit(dp_full);
+      if (!kKV) commit(&c1_empty[0]);
     }
     for (int it = 0; it < w.n && ok; ++it) {
       const uint32_t st = ring.stage;
       const uint32_t par = (uint32_t)it & 1u;
-      if (!(ok = wait_all(p_ready, par, kSiteBwdMmaP))) break;
-      tc_fence_after();
-      if (kKV) issue_acc(256, 0, adv(desc_c_mn, stage_bytes(st) + Plan::kTileBytes), it > 0);
       ring.advance<S>();
       const bool has_next = it + 1 < w.n;
+      if (!(ok = wait_all(s_free, par, kSiteBwdMmaP))) break;
       if (has_next) {
-        if (!(ok = wait_all(&c_full[ring.stage], ring.phase, kSiteBwdMmaCol))) break;
+        if (!(ok = wait_all(&c0_full[ring.stage], ring.phase, kSiteBwdMmaCol))) break;
         tc_fence_after();
-        issue_rc(0, desc_r0, adv(desc_c_k, stage_bytes(ring.stage)));
+        issue_rc(0, desc_r0, adv(desc_c_k, c0_bytes(ring.stage)));
         commit(s_full);
       }
       if (!(ok = wait_all(ds_ready, par, kSiteBwdMmaDS))) break;
       tc_fence_after();
-      issue_acc(384, 128, adv(desc_c_mn, stage_bytes(st)), it > 0);
-      commit(&c_empty[st]);
+      issue_acc(384, 128 + 32, adv(desc_c_mn, c0_bytes(st)), it > 0);
+      commit(&c0_empty[st]);
+      if (kKV) {
+        if (!(ok = wait_all(p_ready, par, kSiteBwdMmaP))) break;
+        tc_fence_after();
+        issue_acc(256, 128, adv(desc_c_mn, c1_bytes(st)), it > 0);
+        commit(&c1_empty[st]);
+      }
       if (has_next) {
-        issue_rc(128, desc_r1, adv(desc_c_k, stage_bytes(ring.stage) + Plan::kTileBytes));
+        if (!(ok = wait_all(&c1_full[ring.stage], ring.phase, kSiteBwdMmaCol))) break;
+        tc_fence_after();
+        issue_rc(128, desc_r1, adv(desc_c_k, c1_bytes(ring.stage)));
         commit(dp_full);
+        if (!kKV) commit(&c1_empty[ring.stage]);
       }
     }
     if (ok) commit(acc_full);
@@ -386,22 +433,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_dp = tmem_base + lane_off + 128 + 64 * h;
     const float c = p.c;
     const int row = w.rb * kBlockM + r;         // global index of this thread's tile row
-    // Q pass: the row's lse2 and delta are fixed for the whole unit.
-    float row_lse2 = 0.f, row_delta = 0.f;
+    // Q pass: the row's -lse2 and -delta are fixed for the whole unit.
+    float row_nlse2 = 0.f, row_ndelta = 0.f;
     if (!kKV) {
       const size_t off = (size_t)w.row_head * p.Npad + row;
-      row_lse2 = p.lse2[off];
-      row_delta = p.delta[off];
+      row_nlse2 = p.nlse2[off];
+      row_ndelta = p.ndelta[off];
     }
-    uint32_t s_par = 0u;
     bool ok = true;
     Ring ring;
     for (int it = 0; it < w.n && ok; ++it) {
       int cb, chead;
       bwd_col<kKV>(p, w, it, cb, chead);
+      const uint32_t par = (uint32_t)it & 1u;
       const float* vec = sVec + ring.stage * 2 * kBlockN + 64 * h;
-      if (!(ok = wait_phase(s_full, s_par, abort_flag, kSiteBwdSoftS))) break;
-      if (kKV && !(ok = wait_phase(&c_full[ring.stage], ring.phase, abort_flag, kSiteBwdSoftS))) break;
+      if (!(ok = wait_phase(s_full, par, abort_flag, kSiteBwdSoftS))) break;
+      if (kKV && !(ok = wait_phase(&c0_full[ring.stage], ring.phase, abort_flag, kSiteBwdSoftS))) break;
       tc_fence_after();
       float pv[64];
       {
@@ -417,24 +464,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pv[32 + i] = __uint_as_float(a1[i]);
         }
       }
-      if (!kKV) {
-        // The scores are in registers: the next tile's S may overwrite them now.
-        tc_fence_before();
-        mbar_arrive(p_ready);
-      }
-      // P = 2^(S c - lse2) (lse2 of the column's query in the KV pass, of the row's otherwise)
-      if (kKV) {
+      // The scores are in registers: the next tile's S may overwrite them now.
+      tc_fence_before();
+      mbar_arrive(s_free);
+      // P = 2^(S c - lse2), lse2 of the column's query in the KV pass, of the row's otherwise;
+      // the workspace holds -lse2.  Column pairs (of every 8) below the polynomial share take
+      // the FMA-pipe exponential instead of the special-function unit.
+      {
+        const float2 c2 = make_float2(c, c);
+        auto exp_pair = [&](int i, float2 nl) {
+          const float2 x = fma2(make_float2(pv[i], pv[i + 1]), c2, nl);
+          float2 e;
+          if (((i >> 1) & 7) < bwd_poly_pairs_per8<D, kKV>()) {
+            e = exp2_poly2(x);
+          } else {
+            e.x = ex2_approx(x.x);
+            e.y = ex2_approx(x.y);
+          }
+          pv[i] = e.x;
+          pv[i + 1] = e.y;
+        };
+        if (kKV) {
 #pragma unroll
-        for (int i = 0; i < 64; i += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(vec + i);
-          pv[i] = ex2_approx(fmaf(pv[i], c, -l4.x));
-          pv[i + 1] = ex2_approx(fmaf(pv[i + 1], c, -l4.y));
-          pv[i + 2] = ex2_approx(fmaf(pv[i + 2], c, -l4.z));
-          pv[i + 3] = ex2_approx(fmaf(pv[i + 3], c, -l4.w));
+          for (int i = 0; i < 64; i += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(vec + i);
+            exp_pair(i, make_float2(l4.x, l4.y));
+            exp_pair(i + 2, make_float2(l4.z, l4.w));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; i += 2) exp_pair(i, make_float2(row_nlse2, row_nlse2));
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) pv[i] = ex2_approx(fmaf(pv[i], c, -row_lse2));
       }
       // Masks.  KV pass: row = key, column = query; the causal mask hides query < key
       // (diagonal block only), and key rows past N are zeroed.  Q pass: row = query,
@@ -444,9 +504,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (kKV) {
           const bool row_dead = row >= p.N;
           const bool diag = p.causal && cb == w.rb;
+          if (row_dead || diag) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (row_dead || (diag && col0 + i < row)) pv[i] = 0.f;
+            for (int i = 0; i < 64; ++i)
+              if (row_dead || col0 + i < row) pv[i] = 0.f;
+          }
         } else {
           const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;  // last allowed key
           if (col0 + 63 > lim) {
@@ -456,52 +518,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
       }
+      // dS = P o (dP - delta) (the workspace holds -delta), as bf16 pairs over the second 32
+      // of this half's dP columns; then (KV pass) P as bf16 pairs over the first 32.
+      if (!(ok = wait_phase(dp_full, par, abort_flag, kSiteBwdSoftDP))) break;
+      tc_fence_after();
+      {
+        uint32_t d0[32], d1[32];
+        tmem_ld32(t_dp, d0);
+        tmem_ld32(t_dp + 32, d1);
+        tmem_ld_wait();
+        reg_fence32(d0);
+        reg_fence32(d1);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const uint32_t* dv = ch ? d1 : d0;
+            float4 n4;
+            if (kKV) {
+              n4 = *reinterpret_cast<const float4*>(vec + kBlockN + 32 * ch + i);
+            } else {
+              n4 = make_float4(row_ndelta, row_ndelta, row_ndelta, row_ndelta);
+            }
+            const float2 e0 = mul2(make_float2(pv[32 * ch + i], pv[32 * ch + i + 1]),
+                                   add2(make_float2(__uint_as_float(dv[i]), __uint_as_float(dv[i + 1])),
+                                        make_float2(n4.x, n4.y)));
+            const float2 e1 = mul2(make_float2(pv[32 * ch + i + 2], pv[32 * ch + i + 3]),
+                                   add2(make_float2(__uint_as_float(dv[i + 2]), __uint_as_float(dv[i + 3])),
+                                        make_float2(n4.z, n4.w)));
+            pk[i / 2] = pack_bf16x2(e0.x, e0.y);
+            pk[i / 2 + 1] = pack_bf16x2(e1.x, e1.y);
+          }
+          tmem_st16(t_dp + 32 + 16 * ch, pk);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_ready);
       if (kKV) {
-        // P (bf16 pairs) over the first 32 of this half's score columns, for acc_p += P C1.
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pv[32 * ch + 2 * i], pv[32 * ch + 2 * i + 1]);
-          tmem_st16(t_s + 16 * ch, pk);
+          tmem_st16(t_dp + 16 * ch, pk);
         }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_ready);
       }
-      s_par ^= 1u;
-      // dS = P o (dP - delta) -> bf16 pairs over the first 32 of this half's dP columns.
-      if (!(ok = wait_phase(dp_full, (uint32_t)it & 1u, abort_flag, kSiteBwdSoftDP))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t dv[32];
-        tmem_ld32(t_dp + 32 * ch, dv);
-        tmem_ld_wait();
-        reg_fence32(dv);
-        uint32_t pk[16];
-        if (kKV) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 d4 = *reinterpret_cast<const float4*>(vec + kBlockN + 32 * ch + i);
-            const float e0 = pv[32 * ch + i] * (__uint_as_float(dv[i]) - d4.x);
-            const float e1 = pv[32 * ch + i + 1] * (__uint_as_float(dv[i + 1]) - d4.y);
-            const float e2 = pv[32 * ch + i + 2] * (__uint_as_float(dv[i + 2]) - d4.z);
-            const float e3 = pv[32 * ch + i + 3] * (__uint_as_float(dv[i + 3]) - d4.w);
-            pk[i / 2] = pack_bf16x2(e0, e1);
-            pk[i / 2 + 1] = pack_bf16x2(e2, e3);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; i += 2)
-            pk[i / 2] = pack_bf16x2(pv[32 * ch + i] * (__uint_as_float(dv[i]) - row_delta),
-                                    pv[32 * ch + i + 1] * (__uint_as_float(dv[i + 1]) - row_delta));
-        }
-        tmem_st16(t_dp + 16 * ch, pk);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(ds_ready);
       ring.advance<S>();
     }
 

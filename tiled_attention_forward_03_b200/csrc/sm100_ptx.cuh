@@ -326,6 +326,17 @@ ATTN_DEV float2 add2(float2 a, float2 b) {
   return d;
 }
 
+ATTN_DEV float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // 2^x for a pair, on the FMA pipe: x = n + f with n = round(x), |f| <= 1/2;
 // 2^f by a degree-3 polynomial (minimax relative error 7.5e-5 on [-1/2, 1/2],
 // coefficients fitted by csrc/fit_exp2_poly.py with the Remez exchange algorithm);
