@@ -30,7 +30,9 @@ Parity status: every forward function below is pinned by tests/test_oracle.py
 and by tests/test_oracle_mutants.py (planted mistakes must fail a pin).  The
 backward functions are pinned by tests/test_oracle_bwd.py (central differences
 of the forward, autograd through torch's fp64 SDPA, a scalar brute force through
-the softmax Jacobian, closed forms and invariants, planted mistakes).
+the softmax Jacobian, closed forms and invariants, planted mistakes).  The RoPE
+functions are pinned by tests/test_oracle_rope.py (hand-computed values, position 0,
+norm preservation, relative-position property, planted mistakes).
 """
 from __future__ import annotations
 
@@ -180,3 +182,35 @@ def attention_backward(q, k, v, do, causal: bool, scale: float):
             dk[b, kh] += gk
             dv[b, kh] += gv
     return dq, dk, dv
+
+
+# ----------------------------------------------------------------------------------------
+# Rotary position embedding (RoPE) applied to Q and K before attention.
+#
+# The pages list a rotary kernel among the kernels built with the tile library ("HipKittens:
+# fast and furious AMD kernels", section "Performance results") without its formula.  The
+# definition used (the "rotate-half" pairing): for position p (the token index) and
+# d < D/2, with theta = p * base^(-2d/D),
+#     x'_d       = x_d cos(theta) - x_{d+D/2} sin(theta)
+#     x'_{d+D/2} = x_{d+D/2} cos(theta) + x_d sin(theta)
+
+def rope_angles(N: int, D: int, base: float = 10000.0) -> np.ndarray:
+    """theta[p, d] = p * base^(-2d/D) for p < N, d < D/2, in fp64."""
+    p = np.arange(N, dtype=np.float64)[:, None]
+    d = np.arange(D // 2, dtype=np.float64)[None, :]
+    return p * base ** (-2.0 * d / D)
+
+
+def rope_rotate(x, base: float = 10000.0, angles=None):
+    """Rotate the last dimension of x [..., N, D] by the RoPE angles of positions 0..N-1."""
+    x = _as_f64(x)
+    N, D = x.shape[-2], x.shape[-1]
+    th = rope_angles(N, D, base) if angles is None else np.asarray(angles, dtype=np.float64)
+    c, s = np.cos(th), np.sin(th)
+    a, b = x[..., : D // 2], x[..., D // 2:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def attention_forward_rope(q, k, v, causal: bool, scale: float, base: float = 10000.0):
+    """Attention of RoPE(q), RoPE(k) and v (all fp64); returns (O, LSE) as attention_forward."""
+    return attention_forward(rope_rotate(q, base), rope_rotate(k, base), v, causal, scale)
