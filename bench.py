@@ -21,6 +21,9 @@ dK/dV and dQ launches), on the forward's o and lse computed once before timing; 
 FLOP count is 2.5x the forward's (the five N x N x D matmuls of the gradient), the
 usual convention.
 
+`--pass rope` times attn_fwd_rope (the rotary kernel on Q and K, then the forward) with the
+forward's FLOP count, and adds the rotary kernel alone against the HBM roofline.
+
 `--impl reference` times the fp64 CPU oracle instead (the only other
 implementation of this path): each step is a bounded sample of the workload's
 heads on the host cores.
@@ -45,6 +48,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 DEFAULT_WORKLOAD = "cfg2"
 METRIC = "attention fwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
+METRIC_ROPE = "attention fwd with RoPE of Q and K TFLOP/s (bf16, 1 B200; forward FLOP count) and % of dense BF16 tensor peak"
 METRIC_BWD = "attention bwd TFLOP/s (bf16, 1 B200; 2.5x the forward FLOP count) and % of dense BF16 tensor peak"
 BWD_FLOP_RATIO = 2.5      # counted backward FLOPs / forward FLOPs (five matmuls against two)
 BWD_EXECUTED_RATIO = 7 / 5  # matmuls the kernels execute / matmuls counted (S and dP run twice)
@@ -204,12 +208,13 @@ def cpu_threads():
     return len(os.sched_getaffinity(0))
 
 
-def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = False):
+def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = False, rope: bool = False):
     """Run the fp64 oracle on whole heads of workload w for about `seconds` (or `heads` heads);
-    the forward, or with `backward` the gradients of one query head.
+    the forward (of RoPE-rotated q and k with `rope`), or with `backward` the gradients of one
+    query head.
 
     Returns (TFLOP/s, FLOPs done, seconds, heads done, sample description)."""
-    from oracle import head_backward, head_forward
+    from oracle import head_backward, head_forward, rope_rotate
     from tiled_attention_forward_03_b200.synth import make_dout, make_qkv
 
     q, k, v = make_qkv(1, w.Hq, w.Hkv, w.N, w.D, w.seed)  # one batch row holds all heads
@@ -222,6 +227,8 @@ def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = Fa
         h = done % w.Hq
         if backward:
             head_backward(q[0, h], k[0, h // g], v[0, h // g], do[0, h], w.causal, w.softmax_scale)
+        elif rope:
+            head_forward(rope_rotate(q[0, h]), rope_rotate(k[0, h // g]), v[0, h // g], w.causal, w.softmax_scale)
         else:
             head_forward(q[0, h], k[0, h // g], v[0, h // g], w.causal, w.softmax_scale)
         done += 1
@@ -231,7 +238,7 @@ def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = Fa
         if heads is None and el >= seconds:
             break
     tflops = per_head * done / el / 1e12
-    what = "gradients" if backward else "forward"
+    what = "gradients" if backward else ("RoPE + forward" if rope else "forward")
     sample = (f"{what} of {done} heads, cycling over the {w.Hq} query heads of one batch row of {w.name} "
               f"(each head's full {w.N}x{w.N} fp64 score matrix), {el:.1f} s")
     return tflops, per_head * done, el, done, sample
@@ -269,6 +276,11 @@ def run_ours(args, w):
         def step():
             attn.backward(qd, kd, vd, o, lse, dod, causal=w.causal, scale=scale, dq=dq, dk=dk, dv=dv,
                           stream=stream)
+    elif args.pass_ == "rope":
+        cos_t, sin_t = attn.rope_tables(w.N, w.D, device=device)
+
+        def step():
+            attn.forward_rope(qd, kd, vd, cos_t, sin_t, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
     else:
         def step():
             attn.forward(qd, kd, vd, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
@@ -320,12 +332,16 @@ def run_ours(args, w):
         oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
         lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
 
+        tables = (cos_t, sin_t) if args.pass_ == "rope" else None
+
         def e2e_call():
             attn.forward_from_host(qh, kh, vh, causal=w.causal, scale=scale, device=device, out_host=oh,
-                                   lse_host=lh, stream=stream)
+                                   lse_host=lh, stream=stream, rope_tables=tables)
         h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-        e2e_path = "forward_from_host: pinned host q,k,v -> device, attn_fwd, o,lse -> pinned host"
+        e2e_path = ("forward_from_host: pinned host q,k,v -> device, "
+                    + ("attn_fwd_rope (device-resident cos/sin tables)" if tables else "attn_fwd")
+                    + ", o,lse -> pinned host")
     for _ in range(2):
         e2e_call()
     barrier(dist, device)
@@ -339,6 +355,22 @@ def run_ours(args, w):
     torch.cuda.synchronize(device)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
     barrier(dist, device)
+
+    rope_ms = None
+    if args.pass_ == "rope":
+        # the rotary kernel alone (attn_rope_qk), L2 flushed between launches
+        qo, ko = torch.empty_like(qd), torch.empty_like(kd)
+        for _ in range(3):
+            attn.rope(qd, kd, cos_t, sin_t, q_out=qo, k_out=ko, stream=stream)
+        rs = [torch.cuda.Event(enable_timing=True) for _ in range(20)]
+        re_ = [torch.cuda.Event(enable_timing=True) for _ in range(20)]
+        for i in range(20):
+            flush.zero_()
+            rs[i].record(stream)
+            attn.rope(qd, kd, cos_t, sin_t, q_out=qo, k_out=ko, stream=stream)
+            re_[i].record(stream)
+        torch.cuda.synchronize(device)
+        rope_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(rs, re_))
 
     if rank != 0:
         if dist is not None:
@@ -358,12 +390,15 @@ def run_ours(args, w):
         q_side = w.B * w.Hq * w.N * w.D * 2
         kv_side = w.B * w.Hkv * w.N * w.D * 2
         algo_bytes = 4 * q_side + 4 * kv_side + 4 * w.B * w.Hq * w.N
+    elif args.pass_ == "rope":
+        kernel = f"attn_fwd_rope call: attn_rope_qk + attn_fwd_sm100<{w.D}>, timed together"
+        algo_bytes = w.algorithmic_bytes
     else:
         kernel = f"attn_fwd_sm100<{w.D}>"
         algo_bytes = w.algorithmic_bytes
 
     line = {
-        "metric": METRIC_BWD if backward else METRIC,
+        "metric": METRIC_BWD if backward else (METRIC_ROPE if args.pass_ == "rope" else METRIC),
         "value": round(value, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -375,7 +410,7 @@ def run_ours(args, w):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {**w.describe(), "pass": "backward" if backward else "forward",
+        "config": {**w.describe(), "pass": {"fwd": "forward", "bwd": "backward", "rope": "forward with RoPE"}[args.pass_],
                    "l2": "flushed between timed steps (512 MB write)",
                    "parallelism": f"replicas{world}: each rank its own batch, no collective on the data path"},
         "pct_of_dense_bf16_peak": round(100.0 * value / world / DATASHEET_BF16_TFLOPS, 2),
@@ -384,7 +419,7 @@ def run_ours(args, w):
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "path": e2e_path},
-        "gpu_launches": args.steps * (3 if backward else 1),
+        "gpu_launches": args.steps * {"fwd": 1, "bwd": 3, "rope": 2}[args.pass_],
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_burst,
                      "unit": "TFLOP/s", "frac": round(achieved / peak_burst, 4), "traffic": traffic,
                      "peak_kind": f"{peak_kind} bf16 matmul, burst (kernel timed alone)",
@@ -394,8 +429,16 @@ def run_ours(args, w):
         line["roofline"]["executed_tflops"] = round(achieved * BWD_EXECUTED_RATIO, 2)
         line["roofline"]["executed_note"] = ("the kernels run 7 N x N x D matmuls where 5 are counted "
                                              "(scores and dP are formed in both the dK/dV and dQ kernels)")
+    if rope_ms is not None:
+        # read q, k once, write their rotations once (the 2 x N x D/2 fp32 tables stay in L2)
+        rope_bytes = 2 * 2 * (w.B * w.Hq + w.B * w.Hkv) * w.N * w.D
+        gbs = rope_bytes / (rope_ms * 1e-3) / 1e9
+        line["rope_kernel"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                               "frac": round(gbs / hbm, 4), "us_per_launch": round(rope_ms * 1e3, 2),
+                               "algorithmic_bytes": rope_bytes, "kernel": "attn_rope_qk",
+                               "peak_kind": "measured HBM copy bandwidth"}
     if world == 1 and not args.no_cpu_baseline:
-        tf, _, el, done, sample = time_oracle(w, CPU_SAMPLE_SECONDS, backward=backward)
+        tf, _, el, done, sample = time_oracle(w, CPU_SAMPLE_SECONDS, backward=backward, rope=args.pass_ == "rope")
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                                 "sample": sample}
     if dist is not None:
@@ -412,7 +455,7 @@ def run_reference(args, w):
     backward = args.pass_ == "bwd"
     per_step = []
     for i in range(args.warmup + args.steps):
-        tf, flops, el, done, sample = time_oracle(w, 0.0, heads=1, backward=backward)
+        tf, flops, el, done, sample = time_oracle(w, 0.0, heads=1, backward=backward, rope=args.pass_ == "rope")
         if i >= args.warmup:
             per_step.append((flops, el))
     flops = sum(f for f, _ in per_step)
@@ -423,7 +466,7 @@ def run_reference(args, w):
     sample = f"{what} of {w.name} per step (full {w.N}x{w.N} fp64 score matrix), {args.steps} steps"
     return {
         "impl": "reference",
-        "metric": METRIC_BWD if backward else METRIC,
+        "metric": METRIC_BWD if backward else (METRIC_ROPE if args.pass_ == "rope" else METRIC),
         "value": value,
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -435,7 +478,7 @@ def run_reference(args, w):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {**w.describe(), "pass": "backward" if backward else "forward"},
+        "config": {**w.describe(), "pass": {"fwd": "forward", "bwd": "backward", "rope": "forward with RoPE"}[args.pass_]},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -450,8 +493,9 @@ def main(argv=None):
                     help="cfg1..cfg4, a sweep point name (e.g. sweep_D128_N8192_causal), or 'all'")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
-                    help="fwd: the attention forward (default); bwd: the backward pass (attn_bwd)")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "rope"], default="fwd",
+                    help="fwd: the attention forward (default); bwd: the backward pass (attn_bwd); "
+                         "rope: RoPE of Q and K then the forward (attn_fwd_rope)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -1,5 +1,5 @@
 /*
- * attn.h -- C ABI of the B200 (sm_100a) bf16 attention library (forward and backward).
+ * attn.h -- C ABI of the B200 (sm_100a) bf16 attention library (forward, backward, RoPE).
  *
  * The operation is the tiled attention forward pass named by "HipKittens:
  * fast and furious AMD kernels" (section "Performance results": an attention
@@ -182,6 +182,52 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
  * -1 on invalid sizes.
  */
 long long attn_bwd_workspace_bytes(int B, int Hq, int N);
+
+/*
+ * attn_rope_qk -- rotary position embedding (RoPE) of Q and K, one pass over HBM.
+ *
+ * The pages list a rotary kernel among those built with the tile library ("HipKittens: fast
+ * and furious AMD kernels", section "Performance results") without a formula.  Rotate-half
+ * pairing: for the row of position p (its index 0..N-1 within the head) and d < D/2,
+ *     x'_d       = x_d cos_t[p][d] - x_{d+D/2} sin_t[p][d]
+ *     x'_{d+D/2} = x_{d+D/2} cos_t[p][d] + x_d sin_t[p][d]
+ * (usually cos_t, sin_t = cos, sin of p * base^(-2d/D); the caller chooses the angles).
+ *
+ * Arguments (DEVICE pointers, caller-owned; all 16-byte aligned):
+ *   q, k          bf16 [B, Hq, N, D] and [B, Hkv, N, D], contiguous.               read
+ *   cos_t, sin_t  fp32 [N, D/2], contiguous.                                        read
+ *   q_out, k_out  bf16, same shapes as q, k; written (every element).  May equal q, k
+ *                 (in place).
+ *   B, Hq, Hkv, N, D  as in attn_fwd (D in {32, 64, 96, 128}).
+ *   stream        cudaStream_t (void*); asynchronous.
+ * Errors: host checks as in attn_fwd, before any CUDA call (ATTN_ERR_MISALIGNED for any
+ * pointer not 16-byte aligned); ATTN_ERR_UNSUPPORTED when B*(Hq+Hkv)*N*D/16 > 2^38.
+ * Numerics: fp32 arithmetic on the bf16 inputs and fp32 tables, rounded to bf16 (nearest even).
+ */
+int attn_rope_qk(const void* q, const void* k, const float* cos_t, const float* sin_t,
+                 void* q_out, void* k_out, int B, int Hq, int Hkv, int N, int D, void* stream);
+
+/*
+ * attn_fwd_rope -- attention forward of RoPE(Q), RoPE(K) and V in one call: attn_rope_qk into
+ * the caller's workspace, then the forward kernel on the rotated tensors (both enqueued on
+ * `stream`).  Arguments as attn_fwd plus the tables of attn_rope_qk and
+ *   workspace        device pointer, 256-byte aligned, at least
+ *                    attn_fwd_rope_workspace_bytes() bytes (fewer, but at least the two rotated
+ *                    tensors, also works: the forward then makes no split); after the call it
+ *                    holds RoPE(Q) at offset 0 and RoPE(K) at offset round_up(B*Hq*N*D*2, 256).
+ * Errors as attn_fwd and attn_rope_qk (ATTN_ERR_INVALID_ARG for a null or too small
+ * workspace).  The result equals attn_fwd on the outputs of attn_rope_qk.
+ */
+int attn_fwd_rope(const void* q, const void* k, const void* v, const float* cos_t, const float* sin_t,
+                  void* o, float* lse, int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_fwd_rope_workspace_bytes -- workspace attn_fwd_rope uses for these sizes on the current
+ * device: the rotated Q and K (each rounded up to 256 bytes) plus the non-causal split
+ * workspace of attn_fwd_workspace_bytes().  -1 on invalid sizes or a CUDA error.
+ */
+long long attn_fwd_rope_workspace_bytes(int B, int Hq, int Hkv, int N, int D);
 
 /* Human-readable name of an attn_status_t value (static string, never null). */
 const char* attn_status_string(int status);

@@ -150,3 +150,46 @@ def test_backward_workspace_bytes():
     assert attn.attn_bwd_workspace_bytes(2, 4, 0) == 0
     assert attn.attn_bwd_workspace_bytes(-1, 4, 100) == -1
     assert attn.attn_bwd_workspace_bytes(1, 0, 100) == -1
+
+
+# ---------------------------------------------------------------- RoPE entry points
+
+def call_rope(**kw):
+    args = dict(q=P, k=P, c=P, s=P, qo=P, ko=P, B=1, Hq=2, Hkv=1, N=128, D=128)
+    args.update(kw)
+    return attn.attn_rope_qk(args["q"], args["k"], args["c"], args["s"], args["qo"], args["ko"], args["B"],
+                             args["Hq"], args["Hkv"], args["N"], args["D"], None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(q=None), INVALID), (dict(k=None), INVALID), (dict(c=None), INVALID), (dict(s=None), INVALID),
+    (dict(qo=None), INVALID), (dict(ko=None), INVALID), (dict(B=-1), INVALID), (dict(Hq=3, Hkv=2), INVALID),
+    (dict(D=80), UNSUPPORTED), (dict(D=256), UNSUPPORTED), (dict(q=P + 8), MISALIGNED),
+    (dict(c=P + 4), MISALIGNED), (dict(ko=P + 2), MISALIGNED),
+    (dict(B=1 << 20, Hq=1 << 10, Hkv=1 << 10, N=1 << 20), UNSUPPORTED),
+])
+def test_rope_rejected_before_any_cuda_call(kw, expected):
+    assert call_rope(**kw) == expected
+
+
+def test_rope_empty_problem_is_ok():
+    assert call_rope(B=0) == OK
+    assert call_rope(N=0, q=None, k=None, c=None, s=None, qo=None, ko=None) == OK
+
+
+def call_fwd_rope(**kw):
+    args = dict(q=P, k=P, v=P, c=P, s=P, o=P, lse=P, B=1, Hq=2, Hkv=1, N=128, D=128, causal=0, scale=0.125,
+                ws=P, nbytes=1 << 24)
+    args.update(kw)
+    return attn.attn_fwd_rope(args["q"], args["k"], args["v"], args["c"], args["s"], args["o"], args["lse"],
+                              args["B"], args["Hq"], args["Hkv"], args["N"], args["D"], args["causal"],
+                              args["scale"], args["ws"], args["nbytes"], None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(v=None), INVALID), (dict(ws=None), INVALID), (dict(nbytes=1024), INVALID), (dict(o=None), INVALID),
+    (dict(scale=math.nan), INVALID), (dict(D=48), UNSUPPORTED), (dict(ws=P + 64), MISALIGNED),
+    (dict(lse=P + 2), MISALIGNED), (dict(s=P + 8), MISALIGNED),
+])
+def test_fwd_rope_rejected_before_any_cuda_call(kw, expected):
+    assert call_fwd_rope(**kw) == expected

@@ -1,0 +1,105 @@
+"""GPU parity: RoPE of Q and K, and the attention forward of the rotated tensors, against the
+fp64 oracle (needs a B200).
+
+The rotation alone: the kernel works in fp32 on the bf16 inputs and fp32 tables and rounds to
+bf16 (nearest even), so each element is within half a bf16 step of the exact rotation plus
+fp32 rounding: |x' - ref| <= 2^-8 |ref| + 1e-6 (2^-8 = one bf16 step, twice the rounding bound).
+The rotated Q and K are bf16 tensors (the tensor core's operand type and attn_rope_qk's
+output type), so the attention is held to the forward's own tolerances (max |dO| <= 2e-2,
+mean |dO| <= 2e-3, max |dLSE| <= 1e-3) against the oracle's fp64 rotation rounded to bf16
+(nearest even, by the test) and then fp64 attention.  Against the unrounded fp64 rotation the
+LSE moves by the rounding of the rotated operands, up to ~2e-3 at D = 128 (measured 1.6e-3 at
+N = 256); that comparison is kept with LSE bound 5e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention_forward, attention_forward_rope, attention_rows, rope_rotate
+from tiled_attention_forward_03_b200.synth import CFG2, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def attn():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import tiled_attention_forward_03_b200 as mod
+    return mod
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,base", [
+    (1, 2, 1, 300, 128, 10000.0), (2, 4, 4, 129, 64, 10000.0), (1, 3, 1, 77, 96, 500.0), (1, 2, 2, 1, 32, 10000.0),
+    (1, 2, 1, 16384, 128, 10000.0),
+])
+def test_rope_rotation(attn, B, Hq, Hkv, N, D, base):
+    q, k, _ = make_qkv(B, Hq, Hkv, N, D, 4000 + N)
+    cos_t, sin_t = attn.rope_tables(N, D, base, device="cuda")
+    qo, ko = attn.rope(q.cuda(), k.cuda(), cos_t, sin_t)
+    torch.cuda.synchronize()
+    for got, x in ((qo, q), (ko, k)):
+        ref = rope_rotate(x, base)
+        g = got.float().cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6), float(np.max(np.abs(g - ref)))
+
+
+def test_rope_in_place(attn):
+    q, k, _ = make_qkv(1, 2, 2, 256, 128, 4100)
+    cos_t, sin_t = attn.rope_tables(256, 128, device="cuda")
+    a = attn.rope(q.cuda(), k.cuda(), cos_t, sin_t)
+    qd, kd = q.cuda(), k.cuda()
+    attn.rope(qd, kd, cos_t, sin_t, q_out=qd, k_out=kd)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], qd) and torch.equal(a[1], kd)
+
+
+def check_forward_rope(attn, q, k, v, causal, scale, base=10000.0):
+    N, D = q.shape[2], q.shape[3]
+    cos_t, sin_t = attn.rope_tables(N, D, base, device="cuda")
+    o, lse = attn.forward_rope(q.cuda(), k.cuda(), v.cuda(), cos_t, sin_t, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    st, site = attn.device_status()
+    assert st == attn.ATTN_OK, f"kernel wait gave up at site {site}"
+    return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def assert_fwd_close(o, lse, o_ref, lse_ref, what, lse_tol=1e-3):
+    d, dl = np.abs(o - o_ref), np.abs(lse - lse_ref)
+    msg = f"{what}: max|dO|={d.max():.3e} mean|dO|={d.mean():.3e} max|dLSE|={dl.max():.3e}"
+    assert d.max() <= 2e-2 and d.mean() <= 2e-3 and dl.max() <= lse_tol, msg
+
+
+def rot_bf16(x, base=10000.0):
+    """The oracle's fp64 rotation, rounded to bf16 (nearest even) as the kernel's operands are."""
+    return torch.from_numpy(rope_rotate(x, base)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,causal", [
+    (1, 2, 2, 256, 128, False), (1, 4, 2, 513, 128, True), (2, 2, 1, 300, 64, True), (1, 2, 2, 1000, 64, False),
+    (1, 2, 2, 200, 96, True), (1, 2, 1, 129, 32, False),
+])
+def test_forward_rope_small(attn, B, Hq, Hkv, N, D, causal):
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, 4200 + N)
+    scale = D ** -0.5
+    o, lse = check_forward_rope(attn, q, k, v, causal, scale)
+    what = f"rope B{B} Hq{Hq} Hkv{Hkv} N{N} D{D} c{causal}"
+    o_ref, lse_ref = attention_forward(rot_bf16(q), rot_bf16(k), v, causal, scale)
+    assert_fwd_close(o, lse, o_ref, lse_ref, what)
+    o_ref, lse_ref = attention_forward_rope(q, k, v, causal, scale)
+    assert_fwd_close(o, lse, o_ref, lse_ref, what + " (unrounded rotation)", lse_tol=5e-3)
+
+
+def test_forward_rope_cfg2_sampled(attn):
+    """cfg2 size (B4 H16 N2048 D128): sampled rows against the oracle's rotation of the sampled heads."""
+    w = CFG2
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.D, w.seed)
+    o, lse = check_forward_rope(attn, q, k, v, w.causal, w.softmax_scale)
+    rng = np.random.default_rng(17)
+    for (b, h) in [(0, 0), (w.B - 1, w.Hq - 1)]:
+        qr = rot_bf16(q[b:b + 1, h:h + 1])
+        kr = rot_bf16(k[b:b + 1, h:h + 1])
+        rows = [(0, 0, int(i)) for i in sorted(set(rng.integers(0, w.N, 64)) | {0, 127, 128, w.N - 1})]
+        o_ref, l_ref = attention_rows(qr, kr, v[b:b + 1, h:h + 1], rows, w.causal, w.softmax_scale)
+        idx = [r[2] for r in rows]
+        assert_fwd_close(o[b, h, idx], lse[b, h, idx], o_ref, l_ref, f"cfg2 rope head {(b, h)}")

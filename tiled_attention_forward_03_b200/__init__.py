@@ -1,4 +1,4 @@
-"""bf16 attention on B200 (sm_100a), forward and backward: Python binding of the C ABI in include/attn.h.
+"""bf16 attention on B200 (sm_100a) -- forward, backward, RoPE: Python binding of the C ABI in include/attn.h.
 
 The binding only marshals arguments: every step of the computation runs in the
 CUDA kernel inside ``libattn_fwd.so``.  There is no CPU fallback; if the library
@@ -7,6 +7,8 @@ cannot be loaded, importing this package raises.
     import tiled_attention_forward_03_b200 as attn
     o, lse = attn.forward(q, k, v, causal=True)        # q,k,v: CUDA bf16 [B, H, N, D]
     dq, dk, dv = attn.backward(q, k, v, o, lse, do, causal=True)
+    cos_t, sin_t = attn.rope_tables(N, D, device="cuda")
+    o, lse = attn.forward_rope(q, k, v, cos_t, sin_t, causal=True)   # attention of RoPE(q), RoPE(k)
 """
 from __future__ import annotations
 
@@ -23,7 +25,8 @@ __all__ = [
     "attn_status_string", "attn_last_cuda_error", "attn_device_status", "attn_num_units",
     "attn_version", "attn_selftest_exp2_poly", "attn_selftest_wait_timeout", "forward",
     "forward_from_host", "device_status", "attn_bwd", "attn_bwd_workspace_bytes", "backward",
-    "backward_from_host",
+    "backward_from_host", "attn_rope_qk", "attn_fwd_rope", "attn_fwd_rope_workspace_bytes", "rope_tables",
+    "rope", "forward_rope",
 ]
 
 ATTN_OK = 0
@@ -64,6 +67,12 @@ def _load() -> ctypes.CDLL:
     L.attn_bwd.restype = i
     L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
     L.attn_bwd_workspace_bytes.restype = ctypes.c_longlong
+    L.attn_rope_qk.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    L.attn_rope_qk.restype = i
+    L.attn_fwd_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, ctypes.c_size_t, vp]
+    L.attn_fwd_rope.restype = i
+    L.attn_fwd_rope_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.attn_fwd_rope_workspace_bytes.restype = ctypes.c_longlong
     L.attn_fwd_ws.restype = i
     L.attn_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
     L.attn_fwd_workspace_bytes.restype = ctypes.c_longlong
@@ -120,6 +129,22 @@ def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, causal, scale,
 
 def attn_bwd_workspace_bytes(B: int, Hq: int, N: int) -> int:
     return lib.attn_bwd_workspace_bytes(B, Hq, N)
+
+
+def attn_rope_qk(q, k, cos_t, sin_t, q_out, k_out, B, Hq, Hkv, N, D, stream) -> int:
+    """Direct call of the RoPE entry point (pointers and stream as integers)."""
+    return lib.attn_rope_qk(q, k, cos_t, sin_t, q_out, k_out, B, Hq, Hkv, N, D, stream)
+
+
+def attn_fwd_rope(q, k, v, cos_t, sin_t, o, lse, B, Hq, Hkv, N, D, causal, scale, workspace, workspace_bytes,
+                  stream) -> int:
+    """Direct call of the RoPE + forward entry point."""
+    return lib.attn_fwd_rope(q, k, v, cos_t, sin_t, o, lse, B, Hq, Hkv, N, D, int(bool(causal)), float(scale),
+                             workspace, workspace_bytes, stream)
+
+
+def attn_fwd_rope_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> int:
+    return lib.attn_fwd_rope_workspace_bytes(B, Hq, Hkv, N, D)
 
 
 def attn_fwd_noalloc_scratch_bytes() -> int:
@@ -238,11 +263,13 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
 
 
 def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None, device=None,
-                      out_host=None, lse_host=None, stream=None):
+                      out_host=None, lse_host=None, stream=None, rope_tables=None):
     """End-to-end call on host (ideally pinned) bf16 tensors: copy in, attention, copy out.
 
     Returns host tensors (o, lse).  The copies and the kernel are enqueued on one
-    stream; the call returns after the device-to-host copies have completed.
+    stream; the call returns after the device-to-host copies have completed.  With
+    ``rope_tables`` = (cos_t, sin_t) (device tables from rope_tables()), the attention is that
+    of RoPE(q), RoPE(k) and v (forward_rope).
     """
     import torch
 
@@ -252,7 +279,10 @@ def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None,
         qd = q.to(dev, non_blocking=True)
         kd = k.to(dev, non_blocking=True)
         vd = v.to(dev, non_blocking=True)
-        o, lse = forward(qd, kd, vd, causal=causal, scale=scale, stream=s)
+        if rope_tables is not None:
+            o, lse = forward_rope(qd, kd, vd, rope_tables[0], rope_tables[1], causal=causal, scale=scale, stream=s)
+        else:
+            o, lse = forward(qd, kd, vd, causal=causal, scale=scale, stream=s)
         if out_host is None:
             out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
         if lse_host is None:
@@ -323,6 +353,77 @@ def backward_from_host(q, k, v, o, lse, dout, causal: bool = False, scale: float
             h.copy_(g, non_blocking=True)
     s.synchronize()
     return tuple(out_host)
+
+
+def rope_tables(N: int, D: int, base: float = 10000.0, device=None):
+    """cos and sin tables [N, D/2] (fp32, computed in fp64) of the angles p * base^(-2d/D)."""
+    import torch
+
+    p = torch.arange(N, dtype=torch.float64)[:, None]
+    d = torch.arange(D // 2, dtype=torch.float64)[None, :]
+    theta = p * torch.pow(torch.tensor(float(base), dtype=torch.float64), -2.0 * d / D)
+    cos_t, sin_t = torch.cos(theta).to(torch.float32), torch.sin(theta).to(torch.float32)
+    if device is not None:
+        cos_t, sin_t = cos_t.to(device), sin_t.to(device)
+    return cos_t.contiguous(), sin_t.contiguous()
+
+
+def rope(q, k, cos_t, sin_t, q_out=None, k_out=None, stream=None):
+    """RoPE of CUDA bf16 q [B, Hq, N, D] and k [B, Hkv, N, D] with tables [N, D/2] (fp32, on the
+    device); returns (q_out, k_out).  Pass q_out=q, k_out=k to rotate in place."""
+    import torch
+
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    _check(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _check(k, "k", torch.bfloat16, (B, Hkv, N, D))
+    _check(cos_t, "cos_t", torch.float32, (N, D // 2))
+    _check(sin_t, "sin_t", torch.float32, (N, D // 2))
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    _check(q_out, "q_out", torch.bfloat16, (B, Hq, N, D))
+    _check(k_out, "k_out", torch.bfloat16, (B, Hkv, N, D))
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = attn_rope_qk(q.data_ptr(), k.data_ptr(), cos_t.data_ptr(), sin_t.data_ptr(), q_out.data_ptr(),
+                          k_out.data_ptr(), B, Hq, Hkv, N, D, s.cuda_stream)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_rope_qk")
+    return q_out, k_out
+
+
+def forward_rope(q, k, v, cos_t, sin_t, causal: bool = False, scale: float | None = None, out=None, lse=None,
+                 stream=None):
+    """Attention forward of RoPE(q), RoPE(k), v in one call (attn_fwd_rope); returns (o, lse).
+    The workspace (rotated q and k, split tail) is cached per device; calls sharing it are
+    ordered on one stream."""
+    import torch
+
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    _check(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _check(k, "k", torch.bfloat16, (B, Hkv, N, D))
+    _check(v, "v", torch.bfloat16, (B, Hkv, N, D))
+    _check(cos_t, "cos_t", torch.float32, (N, D // 2))
+    _check(sin_t, "sin_t", torch.float32, (N, D // 2))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(out, "out", torch.bfloat16, (B, Hq, N, D))
+    _check(lse, "lse", torch.float32, (B, Hq, N))
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        nbytes = attn_fwd_rope_workspace_bytes(B, Hq, Hkv, N, D)
+        if nbytes < 0:
+            raise AttnError(ATTN_ERR_CUDA, "attn_fwd_rope_workspace_bytes")
+        ws = _workspace(q.device, max(nbytes, 256), "rope")
+        st = attn_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), cos_t.data_ptr(), sin_t.data_ptr(),
+                           out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, D, causal, scale, ws.data_ptr(),
+                           ws.numel(), s.cuda_stream)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_rope")
+    return out, lse
 
 
 def device_status(stream=None):

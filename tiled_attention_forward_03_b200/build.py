@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libattn_fwd.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = ["attn_api.cu"]
-HEADERS = ["attn_fwd_kernel.cuh", "attn_bwd_kernel.cuh", "sm100_ptx.cuh"]
+HEADERS = ["attn_fwd_kernel.cuh", "attn_bwd_kernel.cuh", "attn_rope_kernel.cuh", "sm100_ptx.cuh"]
 EXPECTED_REGS = 168
 
 NVCC_FLAGS = [

@@ -17,6 +17,7 @@
 #include "attn.h"
 #include "attn_fwd_kernel.cuh"
 #include "attn_bwd_kernel.cuh"
+#include "attn_rope_kernel.cuh"
 
 #define ATTN_VERSION_STRING "b200-attn 0.1 (sm_100a, tcgen05/TMA/TMEM)"
 
@@ -559,7 +560,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const long long rows = (long long)B * Hq * p.Npad;
   const int prep_threads = 256;
-  const long long prep_blocks = (rows + prep_threads / 16 - 1) / (prep_threads / 16);
+  const long long rows_per_block = prep_threads / 16 * attn::kPrepRows;
+  const long long prep_blocks = (rows + rows_per_block - 1) / rows_per_block;
   attn::attn_bwd_prep<<<(unsigned)prep_blocks, prep_threads, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), lse, nlse2, ndelta,
       rows, N, p.Npad, D);
@@ -576,6 +578,95 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Rotary position embedding (RoPE) of Q and K, alone and ahead of the forward pass.
+
+namespace {
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Host checks shared by the RoPE entry points (no CUDA call).
+int rope_checks(const void* q, const void* k, const float* cos_t, const float* sin_t, int B, int Hq, int Hkv,
+                int N, int D) {
+  if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0) return ATTN_ERR_INVALID_ARG;
+  if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
+  // one thread per 8 rotation pairs, 256 per block, on a 1-D grid (< 2^31 blocks)
+  if ((long long)B * (Hq + Hkv) * (long long)N * (D / 16) > (1LL << 38)) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return ATTN_OK;
+  if (!q || !k || !cos_t || !sin_t) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(cos_t, 16) || !aligned(sin_t, 16)) return ATTN_ERR_MISALIGNED;
+  return ATTN_OK;
+}
+
+int launch_rope(const void* q, const void* k, const float* cos_t, const float* sin_t, void* q_out, void* k_out,
+                int B, int Hq, int Hkv, int N, int D, cudaStream_t s) {
+  const long long q_rows = (long long)B * Hq * N, k_rows = (long long)B * Hkv * N;
+  const long long items = (q_rows + k_rows) * (D / 16);
+  const int threads = 256;
+  const long long per_block = (long long)threads * attn::kRopeItems;
+  attn::attn_rope_qk<<<(unsigned)((items + per_block - 1) / per_block), threads, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k), cos_t, sin_t,
+      reinterpret_cast<__nv_bfloat16*>(q_out), reinterpret_cast<__nv_bfloat16*>(k_out), q_rows, k_rows, N, D);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    record_cuda_error("rope kernel launch", e);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_rope_qk(const void* q, const void* k, const float* cos_t, const float* sin_t, void* q_out, void* k_out,
+                 int B, int Hq, int Hkv, int N, int D, void* stream) {
+  int st = rope_checks(q, k, cos_t, sin_t, B, Hq, Hkv, N, D);
+  if (st != ATTN_OK || B == 0 || N == 0) return st;
+  if (!q_out || !k_out) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q_out, 16) || !aligned(k_out, 16)) return ATTN_ERR_MISALIGNED;
+  return launch_rope(q, k, cos_t, sin_t, q_out, k_out, B, Hq, Hkv, N, D, reinterpret_cast<cudaStream_t>(stream));
+}
+
+long long attn_fwd_rope_workspace_bytes(int B, int Hq, int Hkv, int N, int D) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || N < 0 || !supported_head_dim(D)) return -1;
+  if (B == 0 || N == 0) return 0;
+  const long long split = attn_fwd_workspace_bytes(B, Hq, N, D, 0);
+  if (split < 0) return -1;
+  return (long long)(round256((size_t)B * Hq * N * D * 2) + round256((size_t)B * Hkv * N * D * 2)) + split;
+}
+
+int attn_fwd_rope(const void* q, const void* k, const void* v, const float* cos_t, const float* sin_t, void* o,
+                  float* lse, int B, int Hq, int Hkv, int N, int D, int causal, float scale, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  int st = rope_checks(q, k, cos_t, sin_t, B, Hq, Hkv, N, D);
+  if (st != ATTN_OK) return st;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return ATTN_OK;
+  if (!v || !o || !lse || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) || !aligned(workspace, 256)) return ATTN_ERR_MISALIGNED;
+  const size_t q_part = round256((size_t)B * Hq * N * D * 2), k_part = round256((size_t)B * Hkv * N * D * 2);
+  if (workspace_bytes < q_part + k_part) return ATTN_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    record_cuda_error("cudaGetDevice", e);
+    return ATTN_ERR_CUDA;
+  }
+  // the split-tail workspace, if the rest of the caller's workspace holds it
+  const long long need = attn_fwd_workspace_bytes(B, Hq, N, D, causal);
+  if (need < 0) return ATTN_ERR_CUDA;
+  const size_t rest = workspace_bytes - q_part - k_part;
+  void* split_ws = (need > 0 && (size_t)need <= rest) ? ws + q_part + k_part : nullptr;
+  if ((st = launch_rope(q, k, cos_t, sin_t, ws, ws + q_part, B, Hq, Hkv, N, D, s)) != ATTN_OK) return st;
+  return launch_forward(ws, ws + q_part, v, o, lse, B, Hq, Hkv, N, D, causal, scale, split_ws,
+                        split_ws ? rest : 0, stream);
 }
 
 }  // extern "C"

@@ -124,42 +124,57 @@ struct BwdParams {
   uint32_t idesc_acc;   // 128 x D x 128, A from TMEM, B MN-major
 };
 
-// -delta_i = -sum_d dO_id O_id (fp32 sums of the bf16 products) and -lse2_i = -LSE_i log2(e),
-// one 16-thread group per row of the padded [B*Hq][Npad] layout; pad rows get 0.  (Stored
-// negated so that the kernels add them with paired fp32 instructions.)
+// -delta_i = -sum_d dO_id O_id (fp32 sums of the bf16 products) and -lse2_i = -LSE_i log2(e)
+// over the padded [B*Hq][Npad] layout (pad rows get 0); stored negated so that the kernels add
+// them with paired fp32 instructions.  A 16-lane group takes kPrepRows consecutive rows (D <= 128:
+// one 16-byte piece of O and of dO per lane and row) and issues all their loads before using
+// any, to keep enough bytes in flight for HBM.
+constexpr int kPrepRows = 4;
 __global__ void attn_bwd_prep(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                               const float* __restrict__ lse, float* __restrict__ nlse2,
                               float* __restrict__ ndelta, long long rows, int N, int Npad, int D) {
-  const long long row = (long long)blockIdx.x * (blockDim.x >> 4) + (threadIdx.x >> 4);
+  const long long row0 = ((long long)blockIdx.x * (blockDim.x >> 4) + (threadIdx.x >> 4)) * kPrepRows;
   const int l16 = threadIdx.x & 15;
-  if (row >= rows) return;  // whole 16-lane groups leave together
-  const long long bh = row / Npad;
-  const int qi = (int)(row - bh * Npad);
-  float acc = 0.f;
-  if (qi < N) {
-    const size_t base = ((size_t)bh * N + qi) * D;
-    for (int d = l16 * 8; d < D; d += 128) {
-      const uint4 a = *reinterpret_cast<const uint4*>(o + base + d);
-      const uint4 b = *reinterpret_cast<const uint4*>(dout + base + d);
-      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+  if (row0 >= rows) return;  // whole 16-lane groups leave together (rows is a multiple of 128)
+  uint4 a[kPrepRows], b[kPrepRows];
+  bool live[kPrepRows];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 fa = __bfloat1622float2(pa[e]);
-        const float2 fb = __bfloat1622float2(pb[e]);
-        acc = fmaf(fa.x, fb.x, acc);
-        acc = fmaf(fa.y, fb.y, acc);
-      }
+  for (int k = 0; k < kPrepRows; ++k) {
+    const long long row = row0 + k;
+    const long long bh = row / Npad;
+    const int qi = (int)(row - bh * Npad);
+    live[k] = qi < N && l16 * 8 < D;
+    a[k] = b[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (live[k]) {
+      const size_t off = ((size_t)bh * N + qi) * D + l16 * 8;
+      a[k] = *reinterpret_cast<const uint4*>(o + off);
+      b[k] = *reinterpret_cast<const uint4*>(dout + off);
     }
   }
   const unsigned mask = 0xffffu << (threadIdx.x & 16);
-  acc += __shfl_xor_sync(mask, acc, 8, 16);
-  acc += __shfl_xor_sync(mask, acc, 4, 16);
-  acc += __shfl_xor_sync(mask, acc, 2, 16);
-  acc += __shfl_xor_sync(mask, acc, 1, 16);
-  if (l16 == 0) {
-    ndelta[row] = -acc;
-    nlse2[row] = qi < N ? -lse[(size_t)bh * N + qi] * kLog2e : 0.f;
+#pragma unroll
+  for (int k = 0; k < kPrepRows; ++k) {
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a[k]);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b[k]);
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fa = __bfloat1622float2(pa[e]);
+      const float2 fb = __bfloat1622float2(pb[e]);
+      acc = fmaf(fa.x, fb.x, acc);
+      acc = fmaf(fa.y, fb.y, acc);
+    }
+    acc += __shfl_xor_sync(mask, acc, 8, 16);
+    acc += __shfl_xor_sync(mask, acc, 4, 16);
+    acc += __shfl_xor_sync(mask, acc, 2, 16);
+    acc += __shfl_xor_sync(mask, acc, 1, 16);
+    if (l16 == k) {
+      const long long row = row0 + k;
+      const long long bh = row / Npad;
+      const int qi = (int)(row - bh * Npad);
+      ndelta[row] = -acc;
+      nlse2[row] = qi < N ? -lse[(size_t)bh * N + qi] * kLog2e : 0.f;
+    }
   }
 }
 
