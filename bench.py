@@ -24,6 +24,9 @@ usual convention.
 `--pass rope` times attn_fwd_rope (the rotary kernel on Q and K, then the forward) with the
 forward's FLOP count, and adds the rotary kernel alone against the HBM roofline.
 
+`--pass fp8` times attn_fwd_fp8 on E4M3 inputs (N(0,1) x 16 rounded to E4M3, descale 1/16) with
+the forward's FLOP count, against the measured bf16 peak x 2 (the nominal E4M3/bf16 ratio).
+
 `--impl reference` times the fp64 CPU oracle instead (the only other
 implementation of this path): each step is a bounded sample of the workload's
 heads on the host cores.
@@ -48,8 +51,11 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 DEFAULT_WORKLOAD = "cfg2"
 METRIC = "attention fwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
+METRIC_FP8 = "attention fwd E4M3 (FP8) TFLOP/s (1 B200) and % of dense FP8 tensor peak"
+FP8_OVER_BF16 = 2.0  # nominal dense E4M3 / bf16 tensor rate (4.5 / 2.25 PFLOP/s)
 METRIC_ROPE = "attention fwd with RoPE of Q and K TFLOP/s (bf16, 1 B200; forward FLOP count) and % of dense BF16 tensor peak"
 METRIC_BWD = "attention bwd TFLOP/s (bf16, 1 B200; 2.5x the forward FLOP count) and % of dense BF16 tensor peak"
+PASS_NAMES = {"fwd": "forward", "bwd": "backward", "rope": "forward with RoPE", "fp8": "forward, E4M3 inputs"}
 BWD_FLOP_RATIO = 2.5      # counted backward FLOPs / forward FLOPs (five matmuls against two)
 BWD_EXECUTED_RATIO = 7 / 5  # matmuls the kernels execute / matmuls counted (S and dP run twice)
 L2_FLUSH_BYTES = 512 << 20
@@ -215,7 +221,7 @@ def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = Fa
 
     Returns (TFLOP/s, FLOPs done, seconds, heads done, sample description)."""
     from oracle import head_backward, head_forward, rope_rotate
-    from tiled_attention_forward_03_b200.synth import make_dout, make_qkv
+    from tiled_attention_forward_03_b200.synth import make_dout, make_qkv, make_qkv_e4m3
 
     q, k, v = make_qkv(1, w.Hq, w.Hkv, w.N, w.D, w.seed)  # one batch row holds all heads
     do = make_dout(1, w.Hq, w.N, w.D, w.seed + 500) if backward else None
@@ -256,11 +262,15 @@ def run_ours(args, w):
     dist = init_dist(world, "nccl")
 
     import tiled_attention_forward_03_b200 as attn
-    from tiled_attention_forward_03_b200.synth import make_dout, make_qkv
+    from tiled_attention_forward_03_b200.synth import make_dout, make_qkv, make_qkv_e4m3
 
-    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.D, rank_seed(w.seed, rank))
+    fp8 = args.pass_ == "fp8"
+    if fp8:
+        q, k, v, ds = make_qkv_e4m3(w.B, w.Hq, w.Hkv, w.N, w.D, rank_seed(w.seed, rank))
+    else:
+        q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.N, w.D, rank_seed(w.seed, rank))
     qd, kd, vd = (x.to(device) for x in (q, k, v))
-    o = torch.empty_like(qd)
+    o = torch.empty(qd.shape, dtype=torch.bfloat16, device=device)
     lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
@@ -276,6 +286,9 @@ def run_ours(args, w):
         def step():
             attn.backward(qd, kd, vd, o, lse, dod, causal=w.causal, scale=scale, dq=dq, dk=dk, dv=dv,
                           stream=stream)
+    elif fp8:
+        def step():
+            attn.forward_fp8(qd, kd, vd, ds, ds, ds, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
     elif args.pass_ == "rope":
         cos_t, sin_t = attn.rope_tables(w.N, w.D, device=device)
 
@@ -333,14 +346,16 @@ def run_ours(args, w):
         lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
 
         tables = (cos_t, sin_t) if args.pass_ == "rope" else None
+        descales = (ds, ds, ds) if fp8 else None
 
         def e2e_call():
             attn.forward_from_host(qh, kh, vh, causal=w.causal, scale=scale, device=device, out_host=oh,
-                                   lse_host=lh, stream=stream, rope_tables=tables)
+                                   lse_host=lh, stream=stream, rope_tables=tables, fp8_descales=descales)
         h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
         e2e_path = ("forward_from_host: pinned host q,k,v -> device, "
-                    + ("attn_fwd_rope (device-resident cos/sin tables)" if tables else "attn_fwd")
+                    + ("attn_fwd_rope (device-resident cos/sin tables)" if tables else
+                       ("attn_fwd_fp8 (E4M3 inputs)" if fp8 else "attn_fwd"))
                     + ", o,lse -> pinned host")
     for _ in range(2):
         e2e_call()
@@ -393,12 +408,18 @@ def run_ours(args, w):
     elif args.pass_ == "rope":
         kernel = f"attn_fwd_rope call: attn_rope_qk + attn_fwd_sm100<{w.D}>, timed together"
         algo_bytes = w.algorithmic_bytes
+    elif fp8:
+        kernel = f"attn_fwd_sm100<{w.D}, E4M3>"
+        # q, k, v one byte per element; o bf16, lse fp32
+        algo_bytes = (w.B * w.Hq + 2 * w.B * w.Hkv) * w.N * w.D + 2 * w.B * w.Hq * w.N * w.D + 4 * w.B * w.Hq * w.N
+        peak_burst = peak_burst * FP8_OVER_BF16
+        peak_kind = f"{peak_kind} bf16 matmul x {FP8_OVER_BF16:g} (nominal E4M3/bf16 ratio)"
     else:
         kernel = f"attn_fwd_sm100<{w.D}>"
         algo_bytes = w.algorithmic_bytes
 
     line = {
-        "metric": METRIC_BWD if backward else (METRIC_ROPE if args.pass_ == "rope" else METRIC),
+        "metric": {"fwd": METRIC, "bwd": METRIC_BWD, "rope": METRIC_ROPE, "fp8": METRIC_FP8}[args.pass_],
         "value": round(value, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -408,18 +429,19 @@ def run_ours(args, w):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "e4m3" if fp8 else "bf16",
         "data": "synthetic",
-        "config": {**w.describe(), "pass": {"fwd": "forward", "bwd": "backward", "rope": "forward with RoPE"}[args.pass_],
+        "config": {**w.describe(), "pass": PASS_NAMES[args.pass_],
                    "l2": "flushed between timed steps (512 MB write)",
                    "parallelism": f"replicas{world}: each rank its own batch, no collective on the data path"},
-        "pct_of_dense_bf16_peak": round(100.0 * value / world / DATASHEET_BF16_TFLOPS, 2),
-        "pct_of_measured_bf16_peak": round(100.0 * value / world / peak_burst, 2),
+        "pct_of_dense_bf16_peak" if not fp8 else "pct_of_dense_fp8_peak":
+            round(100.0 * value / world / (DATASHEET_BF16_TFLOPS * (FP8_OVER_BF16 if fp8 else 1.0)), 2),
+        "pct_of_measured_bf16_peak" if not fp8 else "pct_of_measured_fp8_peak": round(100.0 * value / world / peak_burst, 2),
         "hbm_gbs_algorithmic": round(algo_bytes / (statistics.mean(kernel_ms) * 1e-3) / 1e9, 1),
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "path": e2e_path},
-        "gpu_launches": args.steps * {"fwd": 1, "bwd": 3, "rope": 2}[args.pass_],
+        "gpu_launches": args.steps * {"fwd": 1, "bwd": 3, "rope": 2, "fp8": 1}[args.pass_],
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_burst,
                      "unit": "TFLOP/s", "frac": round(achieved / peak_burst, 4), "traffic": traffic,
                      "peak_kind": f"{peak_kind} bf16 matmul, burst (kernel timed alone)",
@@ -466,7 +488,7 @@ def run_reference(args, w):
     sample = f"{what} of {w.name} per step (full {w.N}x{w.N} fp64 score matrix), {args.steps} steps"
     return {
         "impl": "reference",
-        "metric": METRIC_BWD if backward else (METRIC_ROPE if args.pass_ == "rope" else METRIC),
+        "metric": {"fwd": METRIC, "bwd": METRIC_BWD, "rope": METRIC_ROPE, "fp8": METRIC_FP8}[args.pass_],
         "value": value,
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -478,7 +500,7 @@ def run_reference(args, w):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {**w.describe(), "pass": {"fwd": "forward", "bwd": "backward", "rope": "forward with RoPE"}[args.pass_]},
+        "config": {**w.describe(), "pass": PASS_NAMES[args.pass_]},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -493,9 +515,10 @@ def main(argv=None):
                     help="cfg1..cfg4, a sweep point name (e.g. sweep_D128_N8192_causal), or 'all'")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "rope"], default="fwd",
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "rope", "fp8"], default="fwd",
                     help="fwd: the attention forward (default); bwd: the backward pass (attn_bwd); "
-                         "rope: RoPE of Q and K then the forward (attn_fwd_rope)")
+                         "rope: RoPE of Q and K then the forward (attn_fwd_rope); fp8: the E4M3 forward "
+                         "(attn_fwd_fp8)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

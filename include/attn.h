@@ -229,6 +229,31 @@ int attn_fwd_rope(const void* q, const void* k, const void* v, const float* cos_
  */
 long long attn_fwd_rope_workspace_bytes(int B, int Hq, int Hkv, int N, int D);
 
+/*
+ * attn_fwd_fp8 -- the attention forward on E4M3 (8-bit float) Q, K and V.
+ *
+ * The pages stress the low-precision tensor-core rates (FP8 GEMM in "HipKittens: fast and
+ * furious AMD kernels", sections "State of the AMD ecosystem" and "Performance results") but
+ * give no FP8 attention recipe.  The library computes the same definition as attn_fwd on the
+ * dequantized inputs  Q = q_descale * q,  K = k_descale * k,  V = v_descale * v:
+ *     O = softmax(scale * Q K^T (+ causal mask)) V,   LSE = ln sum_j exp(scale * Q_i . K_j)
+ *   q, k, v      E4M3 (float8_e4m3fn: 1 sign, 4 exponent, 3 mantissa bits, max 448) bytes,
+ *                [B, Hq, N, D] / [B, Hkv, N, D], contiguous, 16-byte aligned.       read
+ *   o, lse       bf16 [B, Hq, N, D] and fp32 [B, Hq, N], as attn_fwd.              written
+ *   q_descale, k_descale, v_descale   per-tensor factors (finite; q and k non-zero).
+ *   D            64 or 128 (ATTN_ERR_UNSUPPORTED otherwise).
+ *   workspace, workspace_bytes   optional split-tail workspace, as attn_fwd_ws.
+ * Numerics: Q K^T on the E4M3 tensor cores (kind::f8f6f4) with fp32 accumulation; base-2 online
+ * softmax in fp32; probabilities rounded to E4M3 (nearest even; p <= 2^8 by the lazy rescale,
+ * inside E4M3's range) for P V, also E4M3 with fp32 accumulation; row sums of the fp32
+ * probabilities; O rounded to bf16.  Deterministic.  Errors as attn_fwd_ws, plus
+ * ATTN_ERR_INVALID_ARG for non-finite or zero descales.
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+                 float q_descale, float k_descale, float v_descale,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Human-readable name of an attn_status_t value (static string, never null). */
 const char* attn_status_string(int status);
 

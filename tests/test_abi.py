@@ -193,3 +193,29 @@ def call_fwd_rope(**kw):
 ])
 def test_fwd_rope_rejected_before_any_cuda_call(kw, expected):
     assert call_fwd_rope(**kw) == expected
+
+
+# ---------------------------------------------------------------- E4M3 forward
+
+def call_fp8(**kw):
+    args = dict(q=P, k=P, v=P, o=P, lse=P, B=1, Hq=2, Hkv=1, N=128, D=128, causal=0, scale=0.125, qd=0.1, kd=0.1,
+                vd=0.1, ws=None, nbytes=0)
+    args.update(kw)
+    return attn.attn_fwd_fp8(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["Hq"],
+                             args["Hkv"], args["N"], args["D"], args["causal"], args["scale"], args["qd"],
+                             args["kd"], args["vd"], args["ws"], args["nbytes"], None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(q=None), INVALID), (dict(o=None), INVALID), (dict(qd=0.0), INVALID), (dict(kd=math.nan), INVALID),
+    (dict(vd=math.inf), INVALID), (dict(scale=math.nan), INVALID), (dict(Hq=3, Hkv=2), INVALID),
+    (dict(D=32), UNSUPPORTED), (dict(D=96), UNSUPPORTED), (dict(D=80), UNSUPPORTED),
+    (dict(v=P + 8), MISALIGNED), (dict(ws=P + 64, nbytes=4096), MISALIGNED), (dict(ws=None, nbytes=64), INVALID),
+])
+def test_fp8_rejected_before_any_cuda_call(kw, expected):
+    assert call_fp8(**kw) == expected
+
+
+def test_fp8_empty_problem_is_ok():
+    assert call_fp8(B=0) == OK
+    assert call_fp8(N=0, q=None, k=None, v=None, o=None, lse=None) == OK

@@ -26,7 +26,7 @@ __all__ = [
     "attn_version", "attn_selftest_exp2_poly", "attn_selftest_wait_timeout", "forward",
     "forward_from_host", "device_status", "attn_bwd", "attn_bwd_workspace_bytes", "backward",
     "backward_from_host", "attn_rope_qk", "attn_fwd_rope", "attn_fwd_rope_workspace_bytes", "rope_tables",
-    "rope", "forward_rope",
+    "rope", "forward_rope", "attn_fwd_fp8", "forward_fp8",
 ]
 
 ATTN_OK = 0
@@ -67,6 +67,8 @@ def _load() -> ctypes.CDLL:
     L.attn_bwd.restype = i
     L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
     L.attn_bwd_workspace_bytes.restype = ctypes.c_longlong
+    L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, vp, ctypes.c_size_t, vp]
+    L.attn_fwd_fp8.restype = i
     L.attn_rope_qk.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     L.attn_rope_qk.restype = i
     L.attn_fwd_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, ctypes.c_size_t, vp]
@@ -129,6 +131,13 @@ def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, causal, scale,
 
 def attn_bwd_workspace_bytes(B: int, Hq: int, N: int) -> int:
     return lib.attn_bwd_workspace_bytes(B, Hq, N)
+
+
+def attn_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, q_descale, k_descale, v_descale, workspace,
+                 workspace_bytes, stream) -> int:
+    """Direct call of the E4M3 forward entry point (pointers, sizes and stream as integers)."""
+    return lib.attn_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, D, int(bool(causal)), float(scale), float(q_descale),
+                            float(k_descale), float(v_descale), workspace, workspace_bytes, stream)
 
 
 def attn_rope_qk(q, k, cos_t, sin_t, q_out, k_out, B, Hq, Hkv, N, D, stream) -> int:
@@ -263,13 +272,14 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
 
 
 def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None, device=None,
-                      out_host=None, lse_host=None, stream=None, rope_tables=None):
+                      out_host=None, lse_host=None, stream=None, rope_tables=None, fp8_descales=None):
     """End-to-end call on host (ideally pinned) bf16 tensors: copy in, attention, copy out.
 
     Returns host tensors (o, lse).  The copies and the kernel are enqueued on one
     stream; the call returns after the device-to-host copies have completed.  With
     ``rope_tables`` = (cos_t, sin_t) (device tables from rope_tables()), the attention is that
-    of RoPE(q), RoPE(k) and v (forward_rope).
+    of RoPE(q), RoPE(k) and v (forward_rope).  With ``fp8_descales`` = (q_descale, k_descale,
+    v_descale), q, k, v are float8_e4m3fn and the call is forward_fp8.
     """
     import torch
 
@@ -281,6 +291,8 @@ def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None,
         vd = v.to(dev, non_blocking=True)
         if rope_tables is not None:
             o, lse = forward_rope(qd, kd, vd, rope_tables[0], rope_tables[1], causal=causal, scale=scale, stream=s)
+        elif fp8_descales is not None:
+            o, lse = forward_fp8(qd, kd, vd, *fp8_descales, causal=causal, scale=scale, stream=s)
         else:
             o, lse = forward(qd, kd, vd, causal=causal, scale=scale, stream=s)
         if out_host is None:
@@ -353,6 +365,41 @@ def backward_from_host(q, k, v, o, lse, dout, causal: bool = False, scale: float
             h.copy_(g, non_blocking=True)
     s.synchronize()
     return tuple(out_host)
+
+
+def forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float, causal: bool = False,
+                scale: float | None = None, out=None, lse=None, stream=None, split: bool = True):
+    """Attention forward on CUDA float8_e4m3fn q, k, v [B, H, N, D] with per-tensor descales
+    (the inputs' values are descale * stored value); returns (o bf16, lse fp32 [B, Hq, N]).
+    Workspace handling as forward()."""
+    import torch
+
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, N, D]")
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    f8 = torch.float8_e4m3fn
+    _check(q, "q", f8, (B, Hq, N, D))
+    _check(k, "k", f8, (B, Hkv, N, D))
+    _check(v, "v", f8, (B, Hkv, N, D))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = torch.empty((B, Hq, N, D), dtype=torch.bfloat16, device=q.device) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(out, "out", torch.bfloat16, (B, Hq, N, D))
+    _check(lse, "lse", torch.float32, (B, Hq, N))
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        ws_bytes = attn_fwd_workspace_bytes(B, Hq, N, D, causal) if split else 0
+        if ws_bytes < 0:
+            raise AttnError(ATTN_ERR_CUDA, "attn_fwd_workspace_bytes")
+        ws = _workspace(q.device, ws_bytes) if ws_bytes > 0 else None
+        st = attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N,
+                          D, causal, scale, q_descale, k_descale, v_descale, ws.data_ptr() if ws is not None else None,
+                          ws.numel() if ws is not None else 0, s.cuda_stream)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_fp8")
+    return out, lse
 
 
 def rope_tables(N: int, D: int, base: float = 10000.0, device=None):

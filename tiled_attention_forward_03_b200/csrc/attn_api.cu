@@ -79,6 +79,8 @@ bool device_setup(int dev, int* num_sms) {
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64>), attn::SmemPlan<64>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<96>), attn::SmemPlan<96>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<128>), attn::SmemPlan<128>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, true>), attn::SmemPlan<64, true>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<128, true>), attn::SmemPlan<128, true>::kAlloc);
     d.err = e;
     d.attrs_ok = (e == cudaSuccess);
     if (d.attrs_ok && !regs_ok) {
@@ -100,19 +102,21 @@ bool device_setup(int dev, int* num_sms) {
   return true;
 }
 
-// [heads, N, D] bf16 tensor viewed by TMA as 3-D (D fastest), boxes of 64 x 128 x 1
-// with 128-byte swizzle; rows past N read as zero.
-int encode_map(CUtensorMap* map, const void* base, long long heads, int N, int D) {
+// [heads, N, D] tensor of bf16 (elem_bytes 2) or E4M3 bytes (1) viewed by TMA as 3-D (D
+// fastest), boxes of one 128-byte row chunk x 128 rows x 1 head with 128-byte swizzle; rows past
+// N (and columns past D) read as zero.
+int encode_map(CUtensorMap* map, const void* base, long long heads, int N, int D, int elem_bytes = 2) {
   auto enc = tensor_map_encoder();
   if (!enc) {
     std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled entry point unavailable");
     return ATTN_ERR_CUDA;
   }
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * (cuuint64_t)D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)attn::kBlockM, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)D * elem_bytes, (cuuint64_t)N * (cuuint64_t)D * elem_bytes};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / elem_bytes), (cuuint32_t)attn::kBlockM, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -168,9 +172,11 @@ unsigned next_epoch() {
   return e;
 }
 
+// e4m3: q, k, v hold E4M3 bytes whose values are multiplied by qk_descale (in the scores) and
+// o_scale (in the output); otherwise bf16 and both factors 1.
 int launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                    int N, int D, int causal, float scale, void* workspace, size_t workspace_bytes,
-                   void* stream);
+                   void* stream, bool e4m3 = false, float qk_descale = 1.f, float o_scale = 1.f);
 
 }  // namespace
 
@@ -221,18 +227,31 @@ long long attn_fwd_workspace_bytes(int B, int Hq, int N, int D, int causal) {
   return (long long)plan_schedule(units, units, nb, num_sms, 0, D, true).ws_bytes();
 }
 
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                 int D, int causal, float scale, float q_descale, float k_descale, float v_descale, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  if (workspace == nullptr && workspace_bytes != 0) return ATTN_ERR_INVALID_ARG;
+  if (workspace != nullptr && !aligned(workspace, 256)) return ATTN_ERR_MISALIGNED;
+  if (!std::isfinite(q_descale) || !std::isfinite(k_descale) || !std::isfinite(v_descale) || q_descale == 0.f ||
+      k_descale == 0.f)
+    return ATTN_ERR_INVALID_ARG;
+  return launch_forward(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, workspace, workspace_bytes, stream,
+                        true, q_descale * k_descale, v_descale);
+}
+
 }  // extern "C"
 
 namespace {
 
 int launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                    int N, int D, int causal, float scale, void* workspace, size_t workspace_bytes,
-                   void* stream) {
+                   void* stream, bool e4m3, float qk_descale, float o_scale) {
 
   // ---- host-side validation (no CUDA call before this block passes)
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
     return ATTN_ERR_INVALID_ARG;
-  if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
+  if (!supported_head_dim(D) || (e4m3 && D != 64 && D != 128)) return ATTN_ERR_UNSUPPORTED;
+  if (e4m3 && (!std::isfinite(qk_descale) || !std::isfinite(o_scale) || qk_descale == 0.f)) return ATTN_ERR_INVALID_ARG;
   if ((long long)B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return ATTN_OK;  // empty problem: nothing to compute or write
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
@@ -250,9 +269,10 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
 
   CUtensorMap mq, mk, mv;
   int st;
-  if ((st = encode_map(&mq, q, (long long)B * Hq, N, D)) != ATTN_OK) return st;
-  if ((st = encode_map(&mk, k, (long long)B * Hkv, N, D)) != ATTN_OK) return st;
-  if ((st = encode_map(&mv, v, (long long)B * Hkv, N, D)) != ATTN_OK) return st;
+  const int eb = e4m3 ? 1 : 2;
+  if ((st = encode_map(&mq, q, (long long)B * Hq, N, D, eb)) != ATTN_OK) return st;
+  if ((st = encode_map(&mk, k, (long long)B * Hkv, N, D, eb)) != ATTN_OK) return st;
+  if ((st = encode_map(&mv, v, (long long)B * Hkv, N, D, eb)) != ATTN_OK) return st;
 
   attn::FwdParams p;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
@@ -269,9 +289,14 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   p.num_steps = p.causal ? (long long)B * Hq * ((p.num_pairs + 1) / 2) : p.num_units;
   // c > 0 always: masked scores are -inf and -inf * c must stay -inf.  For scale == 0 every
   // allowed score gives 2^(tiny) == 1 in fp32, the same softmax as c == 0.
-  p.c = std::fmax(std::fabs(scale) * 1.44269504088896340736f, 1e-30f);
-  p.idesc_s = attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, scale < 0.f);
-  p.idesc_pv = attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
+  // (E4M3: the scores carry the product of the Q and K descales; its sign joins scale's.)
+  const float s_eff = scale * qk_descale;
+  p.c = std::fmax(std::fabs(s_eff) * 1.44269504088896340736f, 1e-30f);
+  p.o_scale = o_scale;
+  p.idesc_s = e4m3 ? attn::idesc_e4m3_f32(attn::kBlockM, attn::kBlockN, false, false, s_eff < 0.f)
+                   : attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, s_eff < 0.f);
+  p.idesc_pv = e4m3 ? attn::idesc_e4m3_f32(attn::kBlockM, D, false, true, false)
+                    : attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
 
   // Split the last wave only when a workspace big enough for it was given.
   const Schedule plan0 = plan_schedule(p.num_units, p.num_steps, p.num_blocks, num_sms, p.causal, D, true);
@@ -287,7 +312,14 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   p.epoch = split ? next_epoch() : 0u;
   const long long grid = sc.grid;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  switch (D) {
+  if (e4m3) {
+    if (D == 64)
+      attn::attn_fwd_sm100<64, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64, true>::kAlloc, s>>>(
+          mq, mk, mv, p);
+    else
+      attn::attn_fwd_sm100<128, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128, true>::kAlloc, s>>>(
+          mq, mk, mv, p);
+  } else switch (D) {
     case 32:
       attn::attn_fwd_sm100<32><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32>::kAlloc, s>>>(mq, mk, mv, p);
       break;

@@ -77,10 +77,14 @@ enum : unsigned {
 
 __device__ unsigned int g_attn_fault_site = 0;
 
-template <int D>
+// kF8: Q, K, V are E4M3 bytes (one 128-byte swizzle chunk holds 128 columns) instead of bf16.
+template <int D, bool kF8 = false>
 struct SmemPlan {
   static_assert(D == 32 || D == 64 || D == 96 || D == 128, "head dim must be 32, 64, 96 or 128");
-  static constexpr int kChunks = (D + 63) / 64;             // 64-column (128 B) swizzle chunks per row
+  static_assert(!kF8 || D == 64 || D == 128, "E4M3 head dim must be 64 or 128");
+  static constexpr int kElemBytes = kF8 ? 1 : 2;
+  static constexpr int kRowElems = 128 / kElemBytes;        // columns per 128-byte swizzle row
+  static constexpr int kChunks = (D + kRowElems - 1) / kRowElems;  // 128-byte swizzle chunks per row
   static constexpr int kChunkBytes = kBlockM * 128;         // one chunk of a tile: 16 KB
   // one 128-row tile; a partly used last chunk (D = 32, 96) is zero-filled by TMA
   static constexpr int kTileBytes = kChunks * kChunkBytes;
@@ -117,7 +121,8 @@ struct FwdParams {
   float* ws_ml;       // first range's (m, l) [tail_units][2 tiles][128 rows] float2
   unsigned* ws_cnt;   // [tail_units][2 tiles][2]: finished ranges ((epoch << 8) | count), ready flag (epoch)
   unsigned epoch;     // launch tag (24 bits, non-zero): counts of other launches read as 0
-  float c;           // |scale| * log2(e)
+  float c;           // |scale| * log2(e) (times the Q and K descales for E4M3 inputs)
+  float o_scale;     // multiplies the normalised output (the V descale for E4M3 inputs, else 1)
   uint32_t idesc_s;  // S = Q K^T instruction descriptor (negates A when scale < 0)
   uint32_t idesc_pv; // O += P V instruction descriptor
 };
@@ -271,11 +276,15 @@ struct Ring {
   }
 };
 
-template <int D>
+template <int D, bool kF8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
-  using Plan = SmemPlan<D>;
+  using Plan = SmemPlan<D, kF8>;
+  // 32-byte K steps of the tensor-core instructions: 16 bf16 or 32 E4M3 elements each
+  constexpr int kSSteps = D * Plan::kElemBytes / 32;
+  constexpr int kPVSteps = kBlockN * Plan::kElemBytes / 32;
+  constexpr uint32_t kPVStepBytes = (32 / Plan::kElemBytes) * 128;  // K rows of V per step x 128 B
   constexpr int S = Plan::kStages;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled TMA tiles and UMMA descriptors need 1024-byte aligned tiles.
@@ -347,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            uint64_t pol) {
 #pragma unroll
         for (int ch = 0; ch < Plan::kChunks; ++ch)
-          tma_load_3d(dst + ch * Plan::kChunkBytes, map, bar, ch * 64, row, head, pol);
+          tma_load_3d(dst + ch * Plan::kChunkBytes, map, bar, ch * Plan::kRowElems, row, head, pol);
       };
       auto load_kv = [&](const CUtensorMap* map, int row, int head) -> bool {
         if (!wait_phase(&kv_empty[ring.stage], ring.phase ^ 1u, abort_flag, kSiteProducerKV)) return false;
@@ -403,27 +412,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // Adds a byte offset to a descriptor's start-address field (bits 0-13, in 16-byte units).
       auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
-      // S_t = Q_t K^T over D in steps of 16 (K-major A and B, 128-byte swizzle).
+      // S_t = Q_t K^T over D in 32-byte steps (K-major A and B, 128-byte swizzle).
       auto issue_s = [&](int t, uint32_t stage) {
         const uint64_t da = adv(desc_q, t * Plan::kTileBytes);
         const uint64_t db = adv(desc_k, stage * Plan::kTileBytes);
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < kSSteps; ++kk) {
             const uint32_t off = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
-            mma_ss(tmem + t * 128, adv(da, off), adv(db, off), idesc_s, kk > 0 ? 1u : 0u);
+            if constexpr (kF8)
+              mma_ss_f8(tmem + t * 128, adv(da, off), adv(db, off), idesc_s, kk > 0 ? 1u : 0u);
+            else
+              mma_ss(tmem + t * 128, adv(da, off), adv(db, off), idesc_s, kk > 0 ? 1u : 0u);
           }
         }
         __syncwarp();
       };
-      // O_t += P_t V over the 128 keys in steps of 16 (P from TMEM, V MN-major in smem).
+      // O_t += P_t V over the 128 keys in 32-byte steps (P from TMEM: 8 columns per step;
+      // V MN-major in smem).
       auto issue_pv = [&](int t, uint32_t stage, bool accumulate) {
         const uint64_t dv = adv(desc_v, stage * Plan::kTileBytes);
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kBlockN / 16; ++kk)
-            mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, adv(dv, kk * 2048), idesc_pv,
-                   (accumulate || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kPVSteps; ++kk) {
+            if constexpr (kF8)
+              mma_ts_f8(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, adv(dv, kk * kPVStepBytes), idesc_pv,
+                        (accumulate || kk > 0) ? 1u : 0u);
+            else
+              mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, adv(dv, kk * kPVStepBytes), idesc_pv,
+                     (accumulate || kk > 0) ? 1u : 0u);
+          }
         }
         __syncwarp();
       };
@@ -573,8 +591,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           return fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]);
         };
-        // P = 2^(s*c - m_use) in two halves of 64 keys; each half is packed to bf16 pairs and
-        // written over the (already loaded) score columns it came from.  Returns the row
+        // P = 2^(s*c - m_use) in two halves of 64 keys; each half is packed (bf16 pairs, or
+        // four E4M3 bytes per column for E4M3 inputs: p <= 2^8 < 448 fits) and written over
+        // the (already loaded) score columns it came from.  Returns the row
         // sum of the fp32 values.  Masked keys hold s = -inf, so their p is 0 from the
         // special-function unit and 2^-125 (negligible) from the polynomial (c > 0 always).
         // poly_pairs_per8<D>() of every 8 column pairs use the FMA-pipe polynomial instead
@@ -587,6 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t pk[32];
+            float prev = 0.f;  // E4M3: the first value of a group of four
+            float prev2 = 0.f;
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
               const int col = half * 64 + i;
@@ -599,9 +620,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pr.y = ex2_approx(x.y);
               }
               acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], pr);
-              pk[i >> 1] = pack_bf16x2(pr.x, pr.y);
+              if constexpr (kF8) {
+                if ((i & 2) == 0) {
+                  prev = pr.x;
+                  prev2 = pr.y;
+                } else {
+                  pk[i >> 2] = pack_e4m3x4(prev, prev2, pr.x, pr.y);
+                }
+              } else {
+                pk[i >> 1] = pack_bf16x2(pr.x, pr.y);
+              }
             }
-            tmem_st32(t_s + half * 32, pk);
+            if constexpr (kF8) {
+              uint32_t pk16[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk16[i] = pk[i];
+              tmem_st16(t_s + half * 16, pk16);
+            } else {
+              tmem_st32(t_s + half * 32, pk);
+            }
           }
           const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
           return a.x + a.y;
@@ -656,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = row < p.N;
       __nv_bfloat16* orow = p.o + ((size_t)w.head_q * p.N + (row_ok ? row : 0)) * D;
       if (w.parts == 1) {
-        const float inv_l = 1.f / l;
+        const float inv_l = (kF8 ? p.o_scale : 1.f) / l;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t ov[32];
@@ -739,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float mt = fmaxf(m0, m1);
             const float w0 = ex2_approx(m0 - mt), w1 = ex2_approx(m1 - mt);
             const float lt = fmaf(l1, w1, l0 * w0);
-            const float inv_l = 1.f / lt;
+            const float inv_l = (kF8 ? p.o_scale : 1.f) / lt;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
               float4 other[8];

@@ -106,6 +106,23 @@ def make_dout(B: int, Hq: int, N: int, D: int, seed: int):
     return torch.randn((B, Hq, N, D), generator=g, dtype=torch.float32).to(torch.bfloat16)
 
 
+E4M3_AMPLITUDE = 16.0  # inputs are drawn N(0,1), multiplied by this and rounded to E4M3
+
+
+def make_qkv_e4m3(B: int, Hq: int, Hkv: int, N: int, D: int, seed: int):
+    """Draw (q, k, v) as for make_qkv (same generator and order, fp32 N(0,1)), multiply by
+    E4M3_AMPLITUDE and round to float8_e4m3fn (nearest even).  Returns the three CPU E4M3
+    tensors and the descale factor 1 / E4M3_AMPLITUDE that maps them back to the inputs'
+    scale (the values |x| * 16 >= 2^-6 are normal E4M3 numbers)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    out = []
+    for shape in ((B, Hq, N, D), (B, Hkv, N, D), (B, Hkv, N, D)):
+        x = torch.randn(shape, generator=g, dtype=torch.float32) * E4M3_AMPLITUDE
+        out.append(x.to(torch.float8_e4m3fn))
+    return out[0], out[1], out[2], 1.0 / E4M3_AMPLITUDE
+
+
 def make_workload_inputs(w: Workload):
     return make_qkv(w.B, w.Hq, w.Hkv, w.N, w.D, w.seed)
 
