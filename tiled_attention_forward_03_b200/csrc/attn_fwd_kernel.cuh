@@ -54,7 +54,7 @@ constexpr float kRescaleLog2 = 8.0f;
 // Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial instead of the
 // special-function unit; measured best on B200: 2 at D=128, 1 at D=64 (more polynomial work
 // costs issue slots that the MMA-issuing warp shares with the softmax warps).
-template <int D>
+template <int D, bool kF8 = false>
 __host__ __device__ constexpr int poly_pairs_per8() { return D == 128 ? 2 : 1; }
 // (D = 32 and 96 take 1 of 8, like D = 64: their tensor work per block is smaller than at
 // D = 128, so the exponentials weigh more and fewer issue slots can go to the polynomial.)
@@ -613,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int col = half * 64 + i;
               const float2 x = fma2(make_float2(s[col], s[col + 1]), c2, nm2);
               float2 pr;
-              if (((col >> 1) & 7) < poly_pairs_per8<D>()) {
+              if (((col >> 1) & 7) < poly_pairs_per8<D, kF8>()) {
                 pr = exp2_poly2(x);
               } else {
                 pr.x = ex2_approx(x.x);
