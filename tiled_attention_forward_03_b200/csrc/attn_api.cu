@@ -486,10 +486,10 @@ BwdDeviceInfo g_bwd_dev[kMaxDevices];
 template <int D>
 cudaError_t bwd_setup_dim() {
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_bwd_sm100<D, true>),
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, attn::BwdPlan<D>::kAlloc);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, attn::BwdPlan<D, true>::kAlloc);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_bwd_sm100<D, false>),
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, attn::BwdPlan<D>::kAlloc);
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, attn::BwdPlan<D, false>::kAlloc);
   return e;
 }
 
@@ -520,9 +520,9 @@ size_t bwd_part_bytes(long long B, int Hq, int N) {
 template <int D>
 void launch_bwd_dim(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                     const attn::BwdParams& p, long long grid_kv, long long grid_q, cudaStream_t s) {
-  attn::attn_bwd_sm100<D, true><<<(unsigned)grid_kv, attn::kBwdThreads, attn::BwdPlan<D>::kAlloc, s>>>(
+  attn::attn_bwd_sm100<D, true><<<(unsigned)grid_kv, attn::kBwdThreads, attn::BwdPlan<D, true>::kAlloc, s>>>(
       mk, mv, mq, mdo, p);
-  attn::attn_bwd_sm100<D, false><<<(unsigned)grid_q, attn::kBwdThreads, attn::BwdPlan<D>::kAlloc, s>>>(
+  attn::attn_bwd_sm100<D, false><<<(unsigned)grid_q, attn::kBwdThreads, attn::BwdPlan<D, false>::kAlloc, s>>>(
       mq, mdo, mk, mv, p);
 }
 

@@ -51,7 +51,8 @@
 // t+1 overlap all of tile t's gradient matmuls; dP(t+1) overwrites dS(t) and P(t) only
 // after the MMAs reading them.  C0 and C1 tiles have rings of their own, each stage
 // refilled as soon as its last reader has completed (C0 after acc_ds, C1 after acc_p, or
-// after dP in the Q pass), so the next tiles are in flight while the current ones are used.
+// after dP in the Q pass), so the next tiles are in flight while the current ones are used
+// (D = 128: 2 + 2 stages in the KV pass, 3 + 2 in the Q pass; 4 + 4 at D <= 64).
 //
 // Every wait is bounded, as in the forward kernel.
 #pragma once
@@ -90,21 +91,26 @@ ATTN_DEV void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t*
                : "memory");
 }
 
-template <int D>
+template <int D, bool kKV>
 struct BwdPlan {
   static_assert(D == 32 || D == 64 || D == 96 || D == 128, "head dim must be 32, 64, 96 or 128");
   static constexpr int kChunks = (D + 63) / 64;
   static constexpr int kChunkBytes = kBlockM * 128;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = (kChunks == 2) ? 2 : 4;   // column-tile ring depth
-  static constexpr int kROff = 0;                          // R0, R1
-  static constexpr int kCOff = 2 * kTileBytes;             // per stage: C0, C1
-  static constexpr int kVecOff = kCOff + kStages * 2 * kTileBytes;  // per stage: lse2[128], delta[128]
-  static constexpr int kVecBytes = 2 * kBlockN * 4;
-  static constexpr int kBarOff = kVecOff + kStages * kVecBytes;
-  // r_full c0_full[S] c0_empty[S] c1_full[S] c1_empty[S] s_full s_free dp_full p_ready ds_ready
+  // Ring depths of the C0 tiles (Q, or K in the Q pass; they are read first, by S, and last, by
+  // acc_ds) and the C1 tiles (dO or V).  At D = 128 the Q pass, which needs no per-query
+  // vectors, fits a third C0 stage (64 + 96 + 64 KB); the KV pass does not.
+  static constexpr int kStages0 = (kChunks == 2) ? (kKV ? 2 : 3) : 4;
+  static constexpr int kStages1 = (kChunks == 2) ? 2 : 4;
+  static constexpr int kROff = 0;                                  // R0, R1
+  static constexpr int kC0Off = 2 * kTileBytes;                    // C0 ring
+  static constexpr int kC1Off = kC0Off + kStages0 * kTileBytes;    // C1 ring
+  static constexpr int kVecBytes = kKV ? 2 * kBlockN * 4 : 0;      // per C0 stage: -lse2[128], -delta[128]
+  static constexpr int kVecOff = kC1Off + kStages1 * kTileBytes;
+  static constexpr int kBarOff = kVecOff + kStages0 * kVecBytes;
+  // r_full c0_full[S0] c0_empty[S0] c1_full[S1] c1_empty[S1] s_full s_free dp_full p_ready ds_ready
   // acc_full drain
-  static constexpr int kNumBars = 1 + 4 * kStages + 7;
+  static constexpr int kNumBars = 1 + 2 * kStages0 + 2 * kStages1 + 7;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -228,22 +234,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_sm100(const __grid_constant__ CUtensorMap tmap_r0, const __grid_constant__ CUtensorMap tmap_r1,
                    const __grid_constant__ CUtensorMap tmap_c0, const __grid_constant__ CUtensorMap tmap_c1,
                    const BwdParams p) {
-  using Plan = BwdPlan<D>;
-  constexpr int S = Plan::kStages;
+  using Plan = BwdPlan<D, kKV>;
+  constexpr int S0 = Plan::kStages0;
+  constexpr int S1 = Plan::kStages1;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
 
   uint8_t* sR = smem + Plan::kROff;
-  uint8_t* sC = smem + Plan::kCOff;
+  uint8_t* sC0 = smem + Plan::kC0Off;
+  uint8_t* sC1 = smem + Plan::kC1Off;
   float* sVec = reinterpret_cast<float*>(smem + Plan::kVecOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kBarOff);
   uint64_t* r_full = bars;
   uint64_t* c0_full = bars + 1;
-  uint64_t* c0_empty = c0_full + S;
-  uint64_t* c1_full = c0_full + 2 * S;
-  uint64_t* c1_empty = c0_full + 3 * S;
-  uint64_t* s_full = c0_full + 4 * S;
+  uint64_t* c0_empty = c0_full + S0;
+  uint64_t* c1_full = c0_full + 2 * S0;
+  uint64_t* c1_empty = c1_full + S1;
+  uint64_t* s_full = c1_full + 2 * S1;
   uint64_t* s_free = s_full + 1;
   uint64_t* dp_full = s_full + 2;
   uint64_t* p_ready = s_full + 3;
@@ -259,9 +267,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(r_full, 1);
-    for (int i = 0; i < S; ++i) {
+    for (int i = 0; i < S0; ++i) {
       mbar_init(&c0_full[i], 1);
       mbar_init(&c0_empty[i], 1);
+    }
+    for (int i = 0; i < S1; ++i) {
       mbar_init(&c1_full[i], 1);
       mbar_init(&c1_empty[i], 1);
     }
@@ -305,41 +315,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive_expect_tx(r_full, 2 * Plan::kTileBytes);
       load_tile(&tmap_r0, sR, r_full, w.rb * kBlockM, w.row_head, pol_once);
       load_tile(&tmap_r1, sR + Plan::kTileBytes, r_full, w.rb * kBlockM, w.row_head, pol_once);
-      Ring ring;
-      uint32_t filled = 0u, fill_par = 0u;
+      Ring r0, r1;
+      uint32_t filled0 = 0u, par0 = 0u, filled1 = 0u, par1 = 0u;  // per stage: ever filled / parity of last fill
       for (int it = 0; it < w.n; ++it) {
         int cb, chead;
         bwd_col<kKV>(p, w, it, cb, chead);
-        uint8_t* dst = sC + ring.stage * 2 * Plan::kTileBytes;
-        if (!wait_phase(&c0_empty[ring.stage], ring.phase ^ 1u, abort_flag, kSiteBwdProducer)) break;
-        uint64_t* bar0 = &c0_full[ring.stage];
-        mbar_arrive_expect_tx(bar0, Plan::kTileBytes + (kKV ? Plan::kVecBytes : 0));
-        load_tile(&tmap_c0, dst, bar0, cb * kBlockN, chead, pol_shared);
+        if (!wait_phase(&c0_empty[r0.stage], r0.phase ^ 1u, abort_flag, kSiteBwdProducer)) break;
+        uint64_t* bar0 = &c0_full[r0.stage];
+        mbar_arrive_expect_tx(bar0, Plan::kTileBytes + Plan::kVecBytes);
+        load_tile(&tmap_c0, sC0 + r0.stage * Plan::kTileBytes, bar0, cb * kBlockN, chead, pol_shared);
         if (kKV) {
           const size_t off = (size_t)chead * p.Npad + (size_t)cb * kBlockN;
-          float* vec = sVec + ring.stage * 2 * kBlockN;
+          float* vec = sVec + r0.stage * 2 * kBlockN;
           bulk_load_1d(vec, p.nlse2 + off, kBlockN * 4, bar0);
           bulk_load_1d(vec + kBlockN, p.ndelta + off, kBlockN * 4, bar0);
         }
-        if (!wait_phase(&c1_empty[ring.stage], ring.phase ^ 1u, abort_flag, kSiteBwdProducer)) {
-          filled |= 1u << ring.stage;
-          fill_par = (fill_par & ~(1u << ring.stage)) | (ring.phase << ring.stage);
-          break;
-        }
-        uint64_t* bar1 = &c1_full[ring.stage];
+        filled0 |= 1u << r0.stage;
+        par0 = (par0 & ~(1u << r0.stage)) | (r0.phase << r0.stage);
+        r0.advance<S0>();
+        if (!wait_phase(&c1_empty[r1.stage], r1.phase ^ 1u, abort_flag, kSiteBwdProducer)) break;
+        uint64_t* bar1 = &c1_full[r1.stage];
         mbar_arrive_expect_tx(bar1, Plan::kTileBytes);
-        load_tile(&tmap_c1, dst + Plan::kTileBytes, bar1, cb * kBlockN, chead, pol_shared);
-        filled |= 1u << (S + ring.stage);
-        filled |= 1u << ring.stage;
-        fill_par = (fill_par & ~(1u << ring.stage)) | (ring.phase << ring.stage);
-        ring.advance<S>();
+        load_tile(&tmap_c1, sC1 + r1.stage * Plan::kTileBytes, bar1, cb * kBlockN, chead, pol_shared);
+        filled1 |= 1u << r1.stage;
+        par1 = (par1 & ~(1u << r1.stage)) | (r1.phase << r1.stage);
+        r1.advance<S1>();
       }
       // Drain: every issued copy lands before the CTA may exit.
       drain_phase(r_full, 0u, abort_flag);
-      for (int s = 0; s < S; ++s) {
-        if (filled & (1u << s)) drain_phase(&c0_full[s], (fill_par >> s) & 1u, abort_flag);
-        if (filled & (1u << (S + s))) drain_phase(&c1_full[s], (fill_par >> s) & 1u, abort_flag);
-      }
+      for (int s = 0; s < S0; ++s)
+        if (filled0 & (1u << s)) drain_phase(&c0_full[s], (par0 >> s) & 1u, abort_flag);
+      for (int s = 0; s < S1; ++s)
+        if (filled1 & (1u << s)) drain_phase(&c1_full[s], (par1 >> s) & 1u, abort_flag);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -353,8 +360,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_base, 0);
     const uint64_t desc_r0 = smem_desc_kmajor_sw128(smem_u32(sR));
     const uint64_t desc_r1 = smem_desc_kmajor_sw128(smem_u32(sR + Plan::kTileBytes));
-    const uint64_t desc_c_k = smem_desc_kmajor_sw128(smem_u32(sC));
-    const uint64_t desc_c_mn = smem_desc_mnmajor_sw128(smem_u32(sC), Plan::kChunkBytes);
+    const uint64_t desc_c0_k = smem_desc_kmajor_sw128(smem_u32(sC0));
+    const uint64_t desc_c1_k = smem_desc_kmajor_sw128(smem_u32(sC1));
+    const uint64_t desc_c0_mn = smem_desc_mnmajor_sw128(smem_u32(sC0), Plan::kChunkBytes);
+    const uint64_t desc_c1_mn = smem_desc_mnmajor_sw128(smem_u32(sC1), Plan::kChunkBytes);
     auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
     // D = A B^T over the head dim (both K-major): S (R0, C0) or dP (R1, C1).
     auto issue_rc = [&](uint32_t d_col, uint64_t da, uint64_t db) {
@@ -386,53 +395,55 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool mine = wait_phase(bar, parity, abort_flag, site);
       return __all_sync(0xffffffffu, mine);
     };
-    auto c0_bytes = [](uint32_t st) -> uint32_t { return st * 2 * Plan::kTileBytes; };
-    auto c1_bytes = [](uint32_t st) -> uint32_t { return st * 2 * Plan::kTileBytes + Plan::kTileBytes; };
+    auto st_bytes = [](uint32_t st) -> uint32_t { return st * Plan::kTileBytes; };
 
     bool ok = wait_all(r_full, 0u, kSiteBwdMmaRow);
-    Ring ring;
+    Ring r0, r1;  // ring positions of the current tile's C0 and C1
     if (ok && w.n > 0) ok = wait_all(&c0_full[0], 0u, kSiteBwdMmaCol);
     if (ok && w.n > 0) {
       tc_fence_after();
-      issue_rc(0, desc_r0, adv(desc_c_k, c0_bytes(0)));
+      issue_rc(0, desc_r0, desc_c0_k);
       commit(s_full);
       ok = wait_all(&c1_full[0], 0u, kSiteBwdMmaCol);
     }
     if (ok && w.n > 0) {
       tc_fence_after();
-      issue_rc(128, desc_r1, adv(desc_c_k, c1_bytes(0)));
+      issue_rc(128, desc_r1, desc_c1_k);
       commit(dp_full);
       if (!kKV) commit(&c1_empty[0]);
     }
     for (int it = 0; it < w.n && ok; ++it) {
-      const uint32_t st = ring.stage;
       const uint32_t par = (uint32_t)it & 1u;
-      ring.advance<S>();
+      Ring n0 = r0, n1 = r1;  // the next tile's
+      n0.advance<S0>();
+      n1.advance<S1>();
       const bool has_next = it + 1 < w.n;
       if (!(ok = wait_all(s_free, par, kSiteBwdMmaP))) break;
       if (has_next) {
-        if (!(ok = wait_all(&c0_full[ring.stage], ring.phase, kSiteBwdMmaCol))) break;
+        if (!(ok = wait_all(&c0_full[n0.stage], n0.phase, kSiteBwdMmaCol))) break;
         tc_fence_after();
-        issue_rc(0, desc_r0, adv(desc_c_k, c0_bytes(ring.stage)));
+        issue_rc(0, desc_r0, adv(desc_c0_k, st_bytes(n0.stage)));
         commit(s_full);
       }
       if (!(ok = wait_all(ds_ready, par, kSiteBwdMmaDS))) break;
       tc_fence_after();
-      issue_acc(384, 128 + 32, adv(desc_c_mn, c0_bytes(st)), it > 0);
-      commit(&c0_empty[st]);
+      issue_acc(384, 128 + 32, adv(desc_c0_mn, st_bytes(r0.stage)), it > 0);
+      commit(&c0_empty[r0.stage]);
       if (kKV) {
         if (!(ok = wait_all(p_ready, par, kSiteBwdMmaP))) break;
         tc_fence_after();
-        issue_acc(256, 128, adv(desc_c_mn, c1_bytes(st)), it > 0);
-        commit(&c1_empty[st]);
+        issue_acc(256, 128, adv(desc_c1_mn, st_bytes(r1.stage)), it > 0);
+        commit(&c1_empty[r1.stage]);
       }
       if (has_next) {
-        if (!(ok = wait_all(&c1_full[ring.stage], ring.phase, kSiteBwdMmaCol))) break;
+        if (!(ok = wait_all(&c1_full[n1.stage], n1.phase, kSiteBwdMmaCol))) break;
         tc_fence_after();
-        issue_rc(128, desc_r1, adv(desc_c_k, c1_bytes(ring.stage)));
+        issue_rc(128, desc_r1, adv(desc_c1_k, st_bytes(n1.stage)));
         commit(dp_full);
-        if (!kKV) commit(&c1_empty[ring.stage]);
+        if (!kKV) commit(&c1_empty[n1.stage]);
       }
+      r0 = n0;
+      r1 = n1;
     }
     if (ok) commit(acc_full);
     // Drain: all MMAs issued by this warp complete before TMEM is released.
@@ -456,7 +467,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       row_ndelta = p.ndelta[off];
     }
     bool ok = true;
-    Ring ring;
+    Ring ring;  // position of the current tile's C0 (and per-query vectors)
     for (int it = 0; it < w.n && ok; ++it) {
       int cb, chead;
       bwd_col<kKV>(p, w, it, cb, chead);
@@ -583,7 +594,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(p_ready);
       }
-      ring.advance<S>();
+      ring.advance<S0>();
     }
 
     // Epilogue: this thread's row of acc_p / acc_ds, 32-column chunks alternating between
