@@ -193,7 +193,7 @@ def profile_traffic(workload_name: str, which: str = "fwd"):
         return None
     from tiled_attention_forward_03_b200.build import kernel_source_digest
 
-    if d.get("kernel_source_sha256") != kernel_source_digest():
+    if d.get("kernel_source_sha256") != kernel_source_digest(which):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -397,7 +397,9 @@ def run_ours(args, w):
     value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
     achieved = flops_step / (statistics.mean(kernel_ms) * 1e-3) / 1e12
     e2e_value = world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
-    traffic = profile_traffic(w.name, "bwd" if backward else "fwd")
+    # DRAM traffic from a committed ncu record of this path and workload (bf16 forward and
+    # backward only), if the record's kernel sources are the current ones
+    traffic = profile_traffic(w.name, args.pass_) if args.pass_ in ("fwd", "bwd") else None
     if backward:
         kernel = (f"attn_bwd call: attn_bwd_prep + attn_bwd_sm100<{w.D}, dK/dV> + attn_bwd_sm100<{w.D}, dQ>, "
                   f"timed together")

@@ -98,12 +98,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 
 
-def kernel_source_digest() -> str:
-    """SHA-256 over the CUDA sources and headers (identifies the kernel an ncu capture measured)."""
-    import hashlib
+# The files that define each measured path's kernels and their launch: a traffic record taken
+# with ncu stays valid while these files are unchanged.
+DIGEST_FILES = {
+    "fwd": ["attn_fwd_kernel.cuh", "sm100_ptx.cuh", "attn_api.cu"],
+    "bwd": ["attn_bwd_kernel.cuh", "attn_fwd_kernel.cuh", "sm100_ptx.cuh", "attn_api.cu"],
+    "all": SOURCES + HEADERS,
+}
 
+
+def kernel_source_digest(which: str = "all") -> str:
+    """SHA-256 over the CUDA sources of one path ("fwd", "bwd") or of all ("all"); identifies
+    the kernels an ncu capture measured."""
+    import hashlib
     h = hashlib.sha256()
-    for name in SOURCES + HEADERS:
+    for name in DIGEST_FILES[which]:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
