@@ -155,7 +155,7 @@ size_t attn_fwd_noalloc_scratch_bytes(void);
  *   dk    bf16 [B, Hkv, N, D], contiguous.                           written (every element)
  *   dv    bf16 [B, Hkv, N, D], contiguous.                           written (every element)
  *   B, Hq, Hkv, N, D, causal, scale   as in attn_fwd (same limits; additionally
- *         B * Hq * ceil(N / 128) <= 2^31-1).
+ *         B * Hq * ceil(N / 128) <= 2^30, else ATTN_ERR_UNSUPPORTED).
  *   workspace        device pointer, 256-byte aligned, of at least
  *                    attn_bwd_workspace_bytes(B, Hq, N) bytes (per-row delta and
  *                    LSE * log2(e)); needs no initialisation; calls sharing it must be

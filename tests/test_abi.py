@@ -219,3 +219,8 @@ def test_fp8_rejected_before_any_cuda_call(kw, expected):
 def test_fp8_empty_problem_is_ok():
     assert call_fp8(B=0) == OK
     assert call_fp8(N=0, q=None, k=None, v=None, o=None, lse=None) == OK
+
+
+def test_backward_grid_limit():
+    # B * Hq * ceil(N/128) above 2^30 is refused on the host
+    assert call_bwd(B=1 << 16, Hq=1 << 8, Hkv=1 << 8, N=128 * ((1 << 6) + 1)) == UNSUPPORTED

@@ -1,0 +1,36 @@
+"""bench.py on the CPU: the argument checks and the reference arm (the fp64 oracle) for every
+pass, on the smallest workload (no GPU needed)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def run_bench(*args, timeout=600):
+    proc = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True, text=True,
+                          timeout=timeout, cwd=ROOT)
+    return proc
+
+
+@pytest.mark.parametrize("pass_", ["fwd", "bwd", "rope", "fp8"])
+def test_reference_arm_prints_one_json_line(pass_):
+    proc = run_bench("--impl", "reference", "--pass", pass_, "--workload", "cfg1", "--steps", "2", "--warmup", "3")
+    assert proc.returncode == 0, proc.stderr
+    lines = [l for l in proc.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference"
+    assert line["value"] > 0 and line["unit"] == "TFLOP/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["config"]["workload"].startswith("cfg1")
+
+
+def test_warmup_below_three_is_refused():
+    proc = run_bench("--impl", "reference", "--warmup", "2", "--steps", "1")
+    assert proc.returncode != 0
+    assert "--warmup" in proc.stderr

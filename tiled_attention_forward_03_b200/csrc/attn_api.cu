@@ -543,7 +543,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
     return ATTN_ERR_INVALID_ARG;
   if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
-  if ((long long)B * Hq * (((long long)N + attn::kBlockN - 1) / attn::kBlockN) > 0x7fffffffLL)
+  // the dQ grid has B*Hq*ceil(N/128) CTAs and the prep grid twice that many blocks (< 2^31)
+  if ((long long)B * Hq * (((long long)N + attn::kBlockN - 1) / attn::kBlockN) > (1LL << 30))
     return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return ATTN_OK;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
