@@ -222,6 +222,19 @@ def test_side_stream_and_host_path(attn):
     assert_close(o_h.float().numpy().astype(np.float64), l_h.numpy().astype(np.float64), o_ref, l_ref, "host path")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,pieces", [(3, 4, 2, 4), (1, 8, 2, 4), (2, 2, 2, 1)])
+def test_host_path_in_pieces_equals_device_call(attn, B, Hq, Hkv, pieces):
+    """forward_from_host cuts the problem into batch rows (or KV-head groups when B == 1) and
+    pipelines the copies; every piece is checked against the oracle.  (A small piece may take
+    the split last wave, whose merge rounds differently from one whole call, so the pieces are
+    not compared bit for bit with a single device call.)"""
+    q, k, v = make_qkv(B, Hq, Hkv, 700, 128, seed=4011 + B)
+    o_h, l_h = attn.forward_from_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), causal=False, pieces=pieces)
+    o_ref, l_ref = attention_forward(q, k, v, False, 128 ** -0.5)
+    assert_close(o_h.float().numpy().astype(np.float64), l_h.numpy().astype(np.float64), o_ref, l_ref,
+                 f"host path in {pieces} pieces")
+
+
 def test_misaligned_device_pointer_rejected(attn):
     q, k, v = (x.cuda() for x in make_qkv(1, 1, 1, 128, 64, seed=4010))
     o = torch.empty(1 * 128 * 64 + 8, dtype=torch.bfloat16, device="cuda")

@@ -179,3 +179,19 @@ def test_backward_cfg3_sampled_head(attn):
 def test_backward_cfg4_sampled_kv_head(attn):
     # one KV head of the GQA workload: its 4 query heads at N = 8192
     check_heads(attn, CFG4, [(3, 6)])
+
+
+@pytest.mark.parametrize("B,Hq,Hkv", [(3, 4, 2), (1, 8, 2)])
+def test_backward_host_path_in_pieces_equals_device_call(attn, B, Hq, Hkv):
+    """backward_from_host pipelines batch rows (or whole KV-head groups when B == 1); the
+    gradients equal one device call bit for bit."""
+    q, k, v = make_qkv(B, Hq, Hkv, 384, 128, 3400 + B)
+    do = make_dout(B, Hq, 384, 128, 3401 + B)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    o, lse = attn.forward(qd, kd, vd, causal=True)
+    ref = attn.backward(qd, kd, vd, o, lse, dod, causal=True)
+    torch.cuda.synchronize()
+    got = attn.backward_from_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), o.cpu().pin_memory(),
+                                  lse.cpu().pin_memory(), do.pin_memory(), causal=True)
+    for g, r in zip(got, ref):
+        assert torch.equal(g, r.cpu())

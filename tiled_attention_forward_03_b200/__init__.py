@@ -271,12 +271,58 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     return out, lse
 
 
-def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None, device=None,
-                      out_host=None, lse_host=None, stream=None, rope_tables=None, fp8_descales=None):
-    """End-to-end call on host (ideally pinned) bf16 tensors: copy in, attention, copy out.
+def _pieces(B: int, Hq: int, Hkv: int, n: int):
+    """Up to n independent pieces of a [B, H, ...] attention problem, as (batch slice, query-head
+    slice, KV-head slice): ranges of batch rows, or for B == 1 ranges of whole KV-head groups.
+    Each piece is a contiguous block of every tensor."""
+    if B >= 2 or Hkv == 1:
+        n = max(1, min(n, B))
+        e = [B * i // n for i in range(n + 1)]
+        return [(slice(e[i], e[i + 1]), slice(None), slice(None)) for i in range(n) if e[i] < e[i + 1]]
+    g = Hq // Hkv
+    n = max(1, min(n, Hkv))
+    e = [Hkv * i // n for i in range(n + 1)]
+    return [(slice(0, 1), slice(e[i] * g, e[i + 1] * g), slice(e[i], e[i + 1])) for i in range(n) if e[i] < e[i + 1]]
 
-    Returns host tensors (o, lse).  The copies and the kernel are enqueued on one
-    stream; the call returns after the device-to-host copies have completed.  With
+
+def _pipelined(dev, stream, pieces, inputs, outputs, compute):
+    """Run `compute(piece)` for each piece with its inputs copied in and its outputs copied out,
+    the copies on two side streams so that piece i+1's upload and piece i-1's download overlap
+    piece i's kernels.  inputs / outputs: lists of (host tensor, device tensor, piece -> index).
+    Returns after every copy has completed."""
+    import torch
+
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_in.wait_stream(stream)
+    for pc in pieces:
+        with torch.cuda.stream(s_in):
+            for host, devt, idx in inputs:
+                devt[idx(pc)].copy_(host[idx(pc)], non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(s_in)
+        stream.wait_event(ev_in)
+        with torch.cuda.stream(stream):
+            compute(pc)
+            ev_c = torch.cuda.Event()
+            ev_c.record(stream)
+        s_out.wait_event(ev_c)
+        with torch.cuda.stream(s_out):
+            for host, devt, idx in outputs:
+                host[idx(pc)].copy_(devt[idx(pc)], non_blocking=True)
+    s_out.synchronize()
+    stream.synchronize()
+    s_in.synchronize()
+
+
+def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None, device=None,
+                      out_host=None, lse_host=None, stream=None, rope_tables=None, fp8_descales=None,
+                      pieces: int = 4):
+    """End-to-end call on host (ideally pinned) tensors: copy in, attention, copy out.
+
+    Returns host tensors (o, lse).  The problem is cut into up to ``pieces`` independent parts
+    (batch rows, or KV-head groups when B == 1); each part's upload, kernel and download are
+    enqueued so that the copies of neighbouring parts overlap the kernels (copies on two side
+    streams, kernels on ``stream``).  The call returns after the last download.  With
     ``rope_tables`` = (cos_t, sin_t) (device tables from rope_tables()), the attention is that
     of RoPE(q), RoPE(k) and v (forward_rope).  With ``fp8_descales`` = (q_descale, k_descale,
     v_descale), q, k, v are float8_e4m3fn and the call is forward_fp8.
@@ -285,23 +331,30 @@ def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None,
 
     dev = torch.device(device if device is not None else "cuda")
     s = stream if stream is not None else torch.cuda.current_stream(dev)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
     with torch.cuda.stream(s):
-        qd = q.to(dev, non_blocking=True)
-        kd = k.to(dev, non_blocking=True)
-        vd = v.to(dev, non_blocking=True)
+        qd, kd, vd = (torch.empty(x.shape, dtype=x.dtype, device=dev) for x in (q, k, v))
+        od = torch.empty((B, Hq, N, D), dtype=torch.bfloat16, device=dev)
+        ld = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    if out_host is None:
+        out_host = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
+    if lse_host is None:
+        lse_host = torch.empty(ld.shape, dtype=ld.dtype, pin_memory=True)
+    qi = lambda pc: (pc[0], pc[1])
+    ki = lambda pc: (pc[0], pc[2])
+
+    def compute(pc):
+        a, b, c, o, lse = qd[qi(pc)], kd[ki(pc)], vd[ki(pc)], od[qi(pc)], ld[qi(pc)]
         if rope_tables is not None:
-            o, lse = forward_rope(qd, kd, vd, rope_tables[0], rope_tables[1], causal=causal, scale=scale, stream=s)
+            forward_rope(a, b, c, rope_tables[0], rope_tables[1], causal=causal, scale=scale, out=o, lse=lse, stream=s)
         elif fp8_descales is not None:
-            o, lse = forward_fp8(qd, kd, vd, *fp8_descales, causal=causal, scale=scale, stream=s)
+            forward_fp8(a, b, c, *fp8_descales, causal=causal, scale=scale, out=o, lse=lse, stream=s)
         else:
-            o, lse = forward(qd, kd, vd, causal=causal, scale=scale, stream=s)
-        if out_host is None:
-            out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        if lse_host is None:
-            lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-        out_host.copy_(o, non_blocking=True)
-        lse_host.copy_(lse, non_blocking=True)
-    s.synchronize()
+            forward(a, b, c, causal=causal, scale=scale, out=o, lse=lse, stream=s)
+
+    _pipelined(dev, s, _pieces(B, Hq, Hkv, pieces), [(q, qd, qi), (k, kd, ki), (v, vd, ki)],
+               [(out_host, od, qi), (lse_host, ld, qi)], compute)
     return out_host, lse_host
 
 
@@ -348,22 +401,35 @@ def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
 
 
 def backward_from_host(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None, device=None,
-                       out_host=None, stream=None):
+                       out_host=None, stream=None, pieces: int = 4):
     """End-to-end backward on host (ideally pinned) tensors: copy q, k, v, o, lse and dout in,
     run attn_bwd, copy dq, dk, dv out.  Returns host tensors (dq, dk, dv); ``out_host`` may
-    hold three preallocated host tensors for them.  Returns after the copies completed."""
+    hold three preallocated host tensors for them.  Pipelined in up to ``pieces`` independent
+    parts as forward_from_host (batch rows, or whole KV-head groups when B == 1, so that each
+    KV head's gradient is complete within one part).  Returns after the last download."""
     import torch
 
     dev = torch.device(device if device is not None else "cuda")
     s = stream if stream is not None else torch.cuda.current_stream(dev)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    host_in = (q, k, v, o, lse, dout)
     with torch.cuda.stream(s):
-        qd, kd, vd, od, ld, dd = (x.to(dev, non_blocking=True) for x in (q, k, v, o, lse, dout))
-        grads = backward(qd, kd, vd, od, ld, dd, causal=causal, scale=scale, stream=s)
-        if out_host is None:
-            out_host = tuple(torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads)
-        for h, g in zip(out_host, grads):
-            h.copy_(g, non_blocking=True)
-    s.synchronize()
+        dev_in = tuple(torch.empty(x.shape, dtype=x.dtype, device=dev) for x in host_in)
+        grads = tuple(torch.empty(x.shape, dtype=x.dtype, device=dev) for x in (q, k, v))
+    if out_host is None:
+        out_host = tuple(torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads)
+    qi = lambda pc: (pc[0], pc[1])
+    ki = lambda pc: (pc[0], pc[2])
+    in_idx = (qi, ki, ki, qi, qi, qi)
+
+    def compute(pc):
+        qd, kd, vd, od, ld, dd = (x[f(pc)] for x, f in zip(dev_in, in_idx))
+        backward(qd, kd, vd, od, ld, dd, causal=causal, scale=scale, dq=grads[0][qi(pc)], dk=grads[1][ki(pc)],
+                 dv=grads[2][ki(pc)], stream=s)
+
+    _pipelined(dev, s, _pieces(B, Hq, Hkv, pieces), list(zip(host_in, dev_in, in_idx)),
+               list(zip(out_host, grads, (qi, ki, ki))), compute)
     return tuple(out_host)
 
 
