@@ -1,5 +1,7 @@
 /*
- * attn.h -- C ABI of the B200 (sm_100a) bf16 attention library (forward, backward, RoPE).
+ * attn.h -- C ABI of the B200 (sm_100a) attention library: the forward pass in bf16
+ * (attn_fwd, attn_fwd_ws, attn_fwd_noalloc) and E4M3 (attn_fwd_fp8), its gradients
+ * (attn_bwd), and rotary position embedding of Q and K (attn_rope_qk, attn_fwd_rope).
  *
  * The operation is the tiled attention forward pass named by "HipKittens:
  * fast and furious AMD kernels" (section "Performance results": an attention
@@ -30,7 +32,8 @@ typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = 1, /* null pointer, negative size, Hq % Hkv != 0, non-finite scale */
   ATTN_ERR_UNSUPPORTED = 2, /* head dim D other than 32, 64, 96 or 128, or a size beyond the limits below */
-  ATTN_ERR_MISALIGNED = 3,  /* a q/k/v/o pointer not 16-byte aligned, or lse not 4-byte aligned */
+  ATTN_ERR_MISALIGNED = 3,  /* a tensor pointer not 16-byte aligned, lse not 4-byte aligned, or a
+                               workspace not 256-byte aligned (per entry point below) */
   ATTN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
   ATTN_ERR_TIMEOUT = 5      /* a kernel wait gave up (reported by attn_device_status) */
 } attn_status_t;
@@ -269,8 +272,11 @@ const char* attn_last_cuda_error(void);
  * whether any kernel of this library, on the current device, gave up on a
  * bounded wait since the previous call.  Returns ATTN_OK or ATTN_ERR_TIMEOUT
  * (and clears the record), or ATTN_ERR_CUDA if the synchronisation failed.
- * If `site` is non-null it receives the code of the wait that gave up (0 if
- * none).
+ * If `site` is non-null it receives the code of the first wait that gave up (0 if
+ * none): 1-9 the forward kernel's roles (producer, MMA issuer, softmax, drain),
+ * 10 the wait self-test, 11 the forward's split-tail merge, 12-19 the backward
+ * kernels' roles, 20 a backward kernel that found its shared memory base
+ * unaligned.
  */
 int attn_device_status(void* stream, int* site);
 
