@@ -275,8 +275,7 @@ const char* attn_last_cuda_error(void);
  * If `site` is non-null it receives the code of the first wait that gave up (0 if
  * none): 1-9 the forward kernel's roles (producer, MMA issuer, softmax, drain),
  * 10 the wait self-test, 11 the forward's split-tail merge, 12-19 the backward
- * kernels' roles, 20 a backward kernel that found its shared memory base
- * unaligned.
+ * kernels' roles.
  */
 int attn_device_status(void* stream, int* site);
 
