@@ -285,14 +285,30 @@ def _pieces(B: int, Hq: int, Hkv: int, n: int):
     return [(slice(0, 1), slice(e[i] * g, e[i + 1] * g), slice(e[i], e[i + 1])) for i in range(n) if e[i] < e[i + 1]]
 
 
+_streams: dict = {}
+
+
+def _side_streams(dev):
+    """The two copy streams of the host-buffer calls, created once per device."""
+    import torch
+
+    key = (dev.type, dev.index if dev.index is not None else torch.cuda.current_device())
+    pair = _streams.get(key)
+    if pair is None:
+        pair = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+        _streams[key] = pair
+    return pair
+
+
 def _pipelined(dev, stream, pieces, inputs, outputs, compute):
     """Run `compute(piece)` for each piece with its inputs copied in and its outputs copied out,
     the copies on two side streams so that piece i+1's upload and piece i-1's download overlap
     piece i's kernels.  inputs / outputs: lists of (host tensor, device tensor, piece -> index).
-    Returns after every copy has completed."""
+    Returns after every copy has completed.  The side streams are shared by all calls on a
+    device: calls from several host threads at once must not overlap."""
     import torch
 
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_in, s_out = _side_streams(dev)
     s_in.wait_stream(stream)
     for pc in pieces:
         with torch.cuda.stream(s_in):
