@@ -43,6 +43,8 @@
 //   [128,256) dP fp32; once loaded, each softmax warpgroup writes into its 64 columns
 //             P (bf16 pairs, KV pass) over the first 32 and dS (bf16 pairs) over the second 32
 //   [256,256+D) acc_p (dV);  [384,384+D) acc_ds (dK or dQ)
+//   (D <= 64: a second dP buffer at [256,384), acc_p at [384,448), acc_ds at [448,512); dP
+//   alternates between the buffers by tile parity)
 // The two warpgroups never touch each other's columns.
 //
 // MMA order per column tile t (tcgen05 MMAs of one CTA run in issue order):
@@ -108,9 +110,9 @@ struct BwdPlan {
   static constexpr int kVecBytes = kKV ? 2 * kBlockN * 4 : 0;      // per C0 stage: -lse2[128], -delta[128]
   static constexpr int kVecOff = kC1Off + kStages1 * kTileBytes;
   static constexpr int kBarOff = kVecOff + kStages0 * kVecBytes;
-  // r_full c0_full[S0] c0_empty[S0] c1_full[S1] c1_empty[S1] s_full s_free dp_full p_ready ds_ready
-  // acc_full drain
-  static constexpr int kNumBars = 1 + 2 * kStages0 + 2 * kStages1 + 7;
+  // r_full c0_full[S0] c0_empty[S0] c1_full[S1] c1_empty[S1] s_full s_free dp_full[2] p_ready
+  // ds_ready acc_full drain
+  static constexpr int kNumBars = 1 + 2 * kStages0 + 2 * kStages1 + 8;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -253,11 +255,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* c1_empty = c1_full + S1;
   uint64_t* s_full = c1_full + 2 * S1;
   uint64_t* s_free = s_full + 1;
-  uint64_t* dp_full = s_full + 2;
-  uint64_t* p_ready = s_full + 3;
-  uint64_t* ds_ready = s_full + 4;
-  uint64_t* acc_full = s_full + 5;
-  uint64_t* drain = s_full + 6;
+  uint64_t* dp_full = s_full + 2;   // [2]: one per dP buffer ([0] only at D = 128)
+  uint64_t* p_ready = s_full + 4;
+  uint64_t* ds_ready = s_full + 5;
+  uint64_t* acc_full = s_full + 6;
+  uint64_t* drain = s_full + 7;
+  // At D <= 64 tensor memory has room for a second dP buffer (S 128 + dP 2 x 128 + two
+  // accumulators of D <= 64 columns): dP(t+1) then goes into the other buffer as soon as S(t+1)
+  // is issued, instead of waiting for the MMAs that read P(t) and dS(t).
+  constexpr bool kDualDP = D <= 64;
+  constexpr uint32_t kAccP = kDualDP ? 384u : 256u;            // acc_p (dV) column
+  constexpr uint32_t kAccDS = kDualDP ? 384u + 64u : 384u;     // acc_ds (dK or dQ) column
+  auto dp_col = [](int t) -> uint32_t { return 128u + (kDualDP ? 128u * (uint32_t)(t & 1) : 0u); };
+  auto dp_bar = [](int t) -> int { return kDualDP ? (t & 1) : 0; };
+  auto dp_par = [](int t) -> uint32_t { return kDualDP ? (((uint32_t)t >> 1) & 1u) : ((uint32_t)t & 1u); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Plan::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Plan::kMiscOff + 4);
 
@@ -277,7 +288,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 256);
-    mbar_init(dp_full, 1);
+    mbar_init(&dp_full[0], 1);
+    mbar_init(&dp_full[1], 1);
     mbar_init(p_ready, 256);
     mbar_init(ds_ready, 256);
     mbar_init(acc_full, 1);
@@ -408,8 +420,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (ok && w.n > 0) {
       tc_fence_after();
-      issue_rc(128, desc_r1, desc_c1_k);
-      commit(dp_full);
+      issue_rc(dp_col(0), desc_r1, desc_c1_k);
+      commit(&dp_full[dp_bar(0)]);
       if (!kKV) commit(&c1_empty[0]);
     }
     for (int it = 0; it < w.n && ok; ++it) {
@@ -424,22 +436,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         issue_rc(0, desc_r0, adv(desc_c0_k, st_bytes(n0.stage)));
         commit(s_full);
+        if (kDualDP) {
+          // dP(t+1) into the other buffer, whose P(t-1) / dS(t-1) the previous MMAs have read
+          if (!(ok = wait_all(&c1_full[n1.stage], n1.phase, kSiteBwdMmaCol))) break;
+          tc_fence_after();
+          issue_rc(dp_col(it + 1), desc_r1, adv(desc_c1_k, st_bytes(n1.stage)));
+          commit(&dp_full[dp_bar(it + 1)]);
+          if (!kKV) commit(&c1_empty[n1.stage]);
+        }
       }
       if (!(ok = wait_all(ds_ready, par, kSiteBwdMmaDS))) break;
       tc_fence_after();
-      issue_acc(384, 128 + 32, adv(desc_c0_mn, st_bytes(r0.stage)), it > 0);
+      issue_acc(kAccDS, dp_col(it) + 32, adv(desc_c0_mn, st_bytes(r0.stage)), it > 0);
       commit(&c0_empty[r0.stage]);
       if (kKV) {
         if (!(ok = wait_all(p_ready, par, kSiteBwdMmaP))) break;
         tc_fence_after();
-        issue_acc(256, 128, adv(desc_c1_mn, st_bytes(r1.stage)), it > 0);
+        issue_acc(kAccP, dp_col(it), adv(desc_c1_mn, st_bytes(r1.stage)), it > 0);
         commit(&c1_empty[r1.stage]);
       }
-      if (has_next) {
+      if (!kDualDP && has_next) {
         if (!(ok = wait_all(&c1_full[n1.stage], n1.phase, kSiteBwdMmaCol))) break;
         tc_fence_after();
         issue_rc(128, desc_r1, adv(desc_c1_k, st_bytes(n1.stage)));
-        commit(dp_full);
+        commit(&dp_full[0]);
         if (!kKV) commit(&c1_empty[n1.stage]);
       }
       r0 = n0;
@@ -456,7 +476,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int h = warp >> 2;                    // column half
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem_base + lane_off + 64 * h;
-    const uint32_t t_dp = tmem_base + lane_off + 128 + 64 * h;
+    const uint32_t t_dp0 = tmem_base + lane_off + 64 * h;   // + dp_col(t): this thread's dP columns
     const float c = p.c;
     const int row = w.rb * kBlockM + r;         // global index of this thread's tile row
     // Q pass: the row's -lse2 and -delta are fixed for the whole unit.
@@ -546,8 +566,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       // dS = P o (dP - delta) (the workspace holds -delta), as bf16 pairs over the second 32
       // of this half's dP columns; then (KV pass) P as bf16 pairs over the first 32.
-      if (!(ok = wait_phase(dp_full, par, abort_flag, kSiteBwdSoftDP))) break;
+      if (!(ok = wait_phase(&dp_full[dp_bar(it)], dp_par(it), abort_flag, kSiteBwdSoftDP))) break;
       tc_fence_after();
+      const uint32_t t_dp = t_dp0 + dp_col(it);
       {
         uint32_t d0[32], d1[32];
         tmem_ld32(t_dp, d0);
@@ -620,10 +641,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
       if (kKV) {
-        store_acc(256, 1.f, p.dv);
-        store_acc(384, p.scale, p.dk);
+        store_acc(kAccP, 1.f, p.dv);
+        store_acc(kAccDS, p.scale, p.dk);
       } else {
-        store_acc(384, p.scale, p.dq);
+        store_acc(kAccDS, p.scale, p.dq);
       }
     }
   }
