@@ -31,7 +31,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = 1, /* null pointer, negative size, Hq % Hkv != 0, non-finite scale */
-  ATTN_ERR_UNSUPPORTED = 2, /* head dim D other than 32, 64, 96 or 128, or a size beyond the limits below */
+  ATTN_ERR_UNSUPPORTED = 2, /* a head dim D the entry point does not cover, or a size beyond the limits below */
   ATTN_ERR_MISALIGNED = 3,  /* a tensor pointer not 16-byte aligned, lse not 4-byte aligned, or a
                                workspace not 256-byte aligned (per entry point below) */
   ATTN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
@@ -53,7 +53,10 @@ typedef enum {
  *         B >= 0, N >= 0, Hq >= 1, Hkv >= 1, Hq % Hkv == 0.  B == 0 or N == 0
  *         is an empty problem: ATTN_OK is returned and nothing is launched
  *         (pointers may then be null).  Limits: B*Hq <= 2^31-1 and N <= 2^31-1.
- *   D     head dim of q, k, v and o: 32, 64, 96 or 128.
+ *   D     head dim of q, k, v and o: 32, 64, 96, 128, 192 or 256.  D <= 128 runs on the two-tile
+ *         kernel (two 128-row Q tiles per CTA ping-pong on the tensor core); 192 and 256 run on a
+ *         one-tile kernel that ping-pongs two score buffers instead (2 x (128 + D) tensor-memory
+ *         columns would exceed 512).
  *   causal  0: every key is visible; non-zero: key j is visible to query i
  *         iff j <= i (queries and keys share positions 0..N-1).
  *   scale   finite float multiplying q.k before the softmax (1/sqrt(D) is
@@ -102,7 +105,7 @@ int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse
 
 /*
  * attn_fwd_workspace_bytes -- workspace attn_fwd_ws needs for these sizes on the current
- * device (0 if it makes no split, e.g. causal problems or full last waves).  At most
+ * device (0 if it makes no split: causal problems, full last waves, D = 192 or 256).  At most
  * SMs/2 x 2 x 128 x (D + 2) x 4 bytes plus 16 bytes per split unit rounded up to 256
  * (about 9.9 MB on a 148-SM B200 at D=128).
  * Queries the current device's SM count; returns -1 on invalid sizes or a CUDA error.
@@ -157,8 +160,8 @@ size_t attn_fwd_noalloc_scratch_bytes(void);
  *   dq    bf16 [B, Hq,  N, D], contiguous.                           written (every element)
  *   dk    bf16 [B, Hkv, N, D], contiguous.                           written (every element)
  *   dv    bf16 [B, Hkv, N, D], contiguous.                           written (every element)
- *   B, Hq, Hkv, N, D, causal, scale   as in attn_fwd (same limits; additionally
- *         B * Hq * ceil(N / 128) <= 2^30, else ATTN_ERR_UNSUPPORTED).
+ *   B, Hq, Hkv, N, D, causal, scale   as in attn_fwd, but D in {32, 64, 96, 128}; additionally
+ *         B * Hq * ceil(N / 128) <= 2^30, else ATTN_ERR_UNSUPPORTED.
  *   workspace        device pointer, 256-byte aligned, of at least
  *                    attn_bwd_workspace_bytes(B, Hq, N) bytes (per-row delta and
  *                    LSE * log2(e)); needs no initialisation; calls sharing it must be

@@ -61,8 +61,8 @@ def call(**kw):
     (dict(o=None), INVALID), (dict(lse=None), INVALID),
     (dict(B=-1), INVALID), (dict(N=-5), INVALID), (dict(Hq=0), INVALID), (dict(Hkv=0), INVALID),
     (dict(Hq=3, Hkv=2), INVALID), (dict(scale=math.nan), INVALID), (dict(scale=math.inf), INVALID),
-    (dict(D=80), UNSUPPORTED), (dict(D=256), UNSUPPORTED), (dict(D=0), UNSUPPORTED), (dict(D=48), UNSUPPORTED),
-    (dict(q=P + 8), MISALIGNED), (dict(k=P + 2), MISALIGNED), (dict(v=P + 4), MISALIGNED),
+    (dict(D=80), UNSUPPORTED), (dict(D=384), UNSUPPORTED), (dict(D=0), UNSUPPORTED), (dict(D=48), UNSUPPORTED),
+    (dict(D=160), UNSUPPORTED), (dict(q=P + 8), MISALIGNED), (dict(k=P + 2), MISALIGNED), (dict(v=P + 4), MISALIGNED),
     (dict(o=P + 1), MISALIGNED), (dict(lse=P + 2), MISALIGNED),
 ])
 def test_rejected_before_any_cuda_call(kw, expected):
@@ -104,6 +104,12 @@ def test_workspace_entry_point_host_checks():
     assert call_ws(P, 1 << 20, D=80) == UNSUPPORTED        # the usual checks still apply first
     assert call_ws(P, 1 << 20, q=None) == INVALID
     assert call_ws(None, 0, B=0) == OK                     # empty problem
+
+
+def test_wide_head_dims_need_no_workspace():
+    # D = 192, 256 run on the one-tile kernel, which never splits its last wave
+    assert attn.attn_fwd_workspace_bytes(4, 16, 2048, 256, 0) == 0
+    assert attn.attn_fwd_workspace_bytes(4, 16, 2048, 192, 0) == 0
 
 
 def test_workspace_bytes_host_cases():
@@ -164,7 +170,7 @@ def call_rope(**kw):
 @pytest.mark.parametrize("kw,expected", [
     (dict(q=None), INVALID), (dict(k=None), INVALID), (dict(c=None), INVALID), (dict(s=None), INVALID),
     (dict(qo=None), INVALID), (dict(ko=None), INVALID), (dict(B=-1), INVALID), (dict(Hq=3, Hkv=2), INVALID),
-    (dict(D=80), UNSUPPORTED), (dict(D=256), UNSUPPORTED), (dict(q=P + 8), MISALIGNED),
+    (dict(D=80), UNSUPPORTED), (dict(D=384), UNSUPPORTED), (dict(q=P + 8), MISALIGNED),
     (dict(c=P + 4), MISALIGNED), (dict(ko=P + 2), MISALIGNED),
     (dict(B=1 << 20, Hq=1 << 10, Hkv=1 << 10, N=1 << 20), UNSUPPORTED),
 ])

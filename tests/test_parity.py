@@ -136,6 +136,35 @@ def test_head_dims_32_and_96(attn, shape):
     check_full(attn, q, k, v, causal, 1.0 / math.sqrt(D), str(shape))
 
 
+WIDE_HEAD_DIMS = [
+    # (B, Hq, Hkv, N, D, causal): head dims 192 and 256 (the one-tile, two-score-buffer kernel)
+    (1, 2, 2, 1, 192, False), (1, 2, 1, 129, 192, True), (2, 4, 4, 700, 192, False), (1, 4, 2, 1025, 192, True),
+    (1, 2, 2, 1, 256, True), (1, 2, 1, 255, 256, False), (2, 4, 4, 700, 256, True), (1, 4, 2, 1025, 256, False),
+    (1, 4, 4, 2048, 256, False), (1, 8, 2, 2048, 256, True), (1, 2, 2, 384, 256, False),
+]
+
+
+@pytest.mark.parametrize("shape", WIDE_HEAD_DIMS,
+                         ids=lambda s: "B{}_Hq{}_Hkv{}_N{}_D{}_{}".format(*s[:5], "c" if s[5] else "nc"))
+def test_head_dims_192_and_256(attn, shape):
+    B, Hq, Hkv, N, D, causal = shape
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, seed=3600 + N + D + Hq)
+    check_full(attn, q, k, v, causal, 1.0 / math.sqrt(D), str(shape))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_wide_head_dim_rescale_and_scales(attn, causal):
+    """D = 256 with keys whose norm grows along the sequence (the lazy O rescale runs between
+    the two score buffers) and with a negative and a zero scale."""
+    B, Hq, Hkv, N, D = 1, 2, 1, 900, 256
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, seed=3700 + causal)
+    growth = torch.linspace(0.2, 3.0, N).reshape(1, 1, N, 1)
+    k = (k.float() * growth).to(torch.bfloat16)
+    check_full(attn, q, k, v, causal, 1.0 / math.sqrt(D), "wide growing keys")
+    check_full(attn, q, k, v, causal, -0.05, "wide negative scale")
+    check_full(attn, q, k, v, causal, 0.0, "wide zero scale")
+
+
 @pytest.mark.parametrize("scale", [0.0, -0.0883883, 0.02, 0.5])
 @pytest.mark.parametrize("causal", [False, True])
 def test_scales(attn, scale, causal):

@@ -18,6 +18,7 @@
 #include "attn_fwd_kernel.cuh"
 #include "attn_bwd_kernel.cuh"
 #include "attn_rope_kernel.cuh"
+#include "attn_fwd_wide_kernel.cuh"
 
 #define ATTN_VERSION_STRING "b200-attn 0.1 (sm_100a, tcgen05/TMA/TMEM)"
 
@@ -81,6 +82,13 @@ bool device_setup(int dev, int* num_sms) {
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<128>), attn::SmemPlan<128>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, true>), attn::SmemPlan<64, true>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<128, true>), attn::SmemPlan<128, true>::kAlloc);
+    // the wide-head kernel has no register split: dynamic shared memory opt-in only
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_fwd_wide_sm100<192>),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, attn::WidePlan<192>::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_fwd_wide_sm100<256>),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, attn::WidePlan<256>::kAlloc);
     d.err = e;
     d.attrs_ok = (e == cudaSuccess);
     if (d.attrs_ok && !regs_ok) {
@@ -128,7 +136,9 @@ int encode_map(CUtensorMap* map, const void* base, long long heads, int N, int D
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-bool supported_head_dim(int D) { return D == 32 || D == 64 || D == 96 || D == 128; }
+// Forward (bf16): 32 ... 128 on the two-tile kernel, 192 and 256 on the wide-head kernel.
+bool supported_head_dim(int D) { return D == 32 || D == 64 || D == 96 || D == 128 || D == 192 || D == 256; }
+bool narrow_head_dim(int D) { return D == 32 || D == 64 || D == 96 || D == 128; }
 
 // How a non-causal problem is spread over the persistent grid.  Whole units run round
 // robin; if the last wave would be at most half full, each of its units is split into two
@@ -218,7 +228,7 @@ int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse
 
 long long attn_fwd_workspace_bytes(int B, int Hq, int N, int D, int causal) {
   if (B < 0 || Hq < 1 || N < 0 || !supported_head_dim(D)) return -1;
-  if (B == 0 || N == 0 || causal) return 0;
+  if (B == 0 || N == 0 || causal || !narrow_head_dim(D)) return 0;  // the wide-head kernel never splits
   int dev = 0, num_sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
   if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
@@ -274,6 +284,36 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   if ((st = encode_map(&mk, k, (long long)B * Hkv, N, D, eb)) != ATTN_OK) return st;
   if ((st = encode_map(&mv, v, (long long)B * Hkv, N, D, eb)) != ATTN_OK) return st;
 
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!narrow_head_dim(D)) {
+    // D = 192, 256: one CTA per 128-row Q tile on the wide-head kernel
+    attn::WideParams wp;
+    wp.o = reinterpret_cast<__nv_bfloat16*>(o);
+    wp.lse = lse;
+    wp.Hq = Hq;
+    wp.group = Hq / Hkv;
+    wp.N = N;
+    wp.num_blocks = (int)(((long long)N + attn::kBlockN - 1) / attn::kBlockN);
+    wp.causal = causal ? 1 : 0;
+    wp.c = std::fmax(std::fabs(scale) * 1.44269504088896340736f, 1e-30f);
+    wp.idesc_s = attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, scale < 0.f);
+    wp.idesc_pv = attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
+    const long long grid = (long long)B * Hq * wp.num_blocks;
+    if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (D == 192)
+      attn::attn_fwd_wide_sm100<192><<<(unsigned)grid, attn::kWideThreads, attn::WidePlan<192>::kAlloc, s>>>(
+          mq, mk, mv, wp);
+    else
+      attn::attn_fwd_wide_sm100<256><<<(unsigned)grid, attn::kWideThreads, attn::WidePlan<256>::kAlloc, s>>>(
+          mq, mk, mv, wp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      record_cuda_error("kernel launch", e);
+      return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+  }
+
   attn::FwdParams p;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -311,7 +351,6 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   p.ws_o = split ? reinterpret_cast<float*>(static_cast<char*>(workspace) + sc.cnt_bytes + sc.ml_bytes) : nullptr;
   p.epoch = split ? next_epoch() : 0u;
   const long long grid = sc.grid;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (e4m3) {
     if (D == 64)
       attn::attn_fwd_sm100<64, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64, true>::kAlloc, s>>>(
@@ -542,7 +581,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   // ---- host-side validation (no CUDA call before this block passes)
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
     return ATTN_ERR_INVALID_ARG;
-  if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
+  if (!narrow_head_dim(D)) return ATTN_ERR_UNSUPPORTED;  // the backward covers D <= 128
   // the dQ grid has B*Hq*ceil(N/128) CTAs and the prep grid twice that many blocks (< 2^31)
   if ((long long)B * Hq * (((long long)N + attn::kBlockN - 1) / attn::kBlockN) > (1LL << 30))
     return ATTN_ERR_UNSUPPORTED;

@@ -1,0 +1,410 @@
+// attn_fwd_wide_kernel.cuh -- attention forward for head dims 192 and 256 on B200 (sm_100a).
+//
+// The same computation as attn_fwd_kernel.cuh (the pages' tiled forward with an online
+// softmax: "HipKittens: fast and furious AMD kernels", section "Performance results", over
+// several head dims), for D too wide for its two-tile layout: two Q tiles would need
+// 2 x (128 + D) tensor-memory columns, more than the 512 there are.  Here a CTA holds one
+// 128-row Q tile and ping-pongs two score buffers instead:
+//
+//   tensor memory:  S_0 [0,128)  S_1 [128,256)  O [256,256+D)
+//   MMA order:      S(0) S(1) | P(0)V(0) S(2) | P(1)V(1) S(3) | ...
+//
+// S(j+1) is computed while the softmax works on S(j); S(j+2) goes into S(j)'s buffer after
+// P(j) V(j) has read P(j) from it (tcgen05 MMAs of one CTA run in issue order).  The lazy
+// rescale of O at block j waits for P(j-1) V(j-1) to have completed.
+//
+// Warp roles (256 threads, one CTA per SM; no register reallocation is needed):
+//   warps 0-3  softmax: TMEM lane = query row
+//   warp  4    TMA producer: Q once, then K_0, K_1, V_0, K_2, V_1, ... in MMA order
+//   warp  5    MMA issuer (one elected lane)
+//   warps 6-7  idle
+// One CTA per 128-row Q tile (grid = B * Hq * ceil(N/128)), heaviest tiles first when causal.
+// Every wait is bounded, as in the other kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "attn_fwd_kernel.cuh"
+
+namespace attn {
+
+constexpr int kWideThreads = 256;
+
+enum : unsigned {
+  kSiteWideProducer = 21,
+  kSiteWideMma = 22,
+  kSiteWideSoftmax = 23,
+};
+
+template <int D>
+struct WidePlan {
+  static_assert(D == 192 || D == 256, "wide head dim must be 192 or 256");
+  static constexpr int kChunks = D / 64;                 // 64-column (128 B) swizzle chunks per row
+  static constexpr int kChunkBytes = kBlockM * 128;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = D == 256 ? 2 : 3;       // K/V ring depth (tiles)
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  // q_full kv_full[S] kv_empty[S] s_full[2] p_full[2] pv_done o_full drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 4 + 3;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "wide forward shared memory plan exceeds 227 KB");
+};
+
+struct WideParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int Hq, group, N, num_blocks;
+  int causal;
+  float c;            // |scale| * log2(e)
+  uint32_t idesc_s;   // 128 x 128 x D
+  uint32_t idesc_pv;  // 128 x D x 128
+};
+
+template <int D>
+__global__ void __launch_bounds__(kWideThreads, 1)
+    attn_fwd_wide_sm100(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v, const WideParams p) {
+  using Plan = WidePlan<D>;
+  constexpr int S = Plan::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sQ = smem + Plan::kQOff;
+  uint8_t* sKV = smem + Plan::kKVOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + S;
+  uint64_t* s_full = kv_full + 2 * S;  // [2]
+  uint64_t* p_full = s_full + 2;       // [2]
+  uint64_t* pv_done = s_full + 4;      // one phase per P V
+  uint64_t* o_full = s_full + 5;
+  uint64_t* drain = s_full + 6;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Plan::kMiscOff);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Plan::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // The CTA's Q tile: heads in order, a head's tiles heaviest first when causal.
+  const int nb = p.num_blocks;
+  const int head_q = (int)(blockIdx.x / nb);
+  const int k = (int)(blockIdx.x - (long long)head_q * nb);
+  const int qt = p.causal ? nb - 1 - k : k;
+  const int head_kv = (head_q / p.Hq) * (p.Hq / p.group) + (head_q % p.Hq) / p.group;
+  const int n = p.causal ? qt + 1 : nb;  // KV blocks this tile sees
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kBlockM);
+    }
+    mbar_init(pv_done, 1);
+    mbar_init(o_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const uint64_t pol_q = l2_policy_evict_first();
+      auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int row, int head, uint64_t pol) {
+#pragma unroll
+        for (int ch = 0; ch < Plan::kChunks; ++ch)
+          tma_load_3d(dst + ch * Plan::kChunkBytes, map, bar, ch * 64, row, head, pol);
+      };
+      mbar_arrive_expect_tx(q_full, Plan::kTileBytes);
+      load_tile(&tmap_q, sQ, q_full, qt * kBlockM, head_q, pol_q);
+      Ring ring;
+      uint32_t filled = 0u, fill_par = 0u;
+      bool ok = true;
+      // Tiles in the order the MMAs read them: K_0, K_1, V_0, K_2, V_1, ..., V_{n-1}.
+      const int total = 2 * n;
+      for (int i = 0; i < total && ok; ++i) {
+        bool is_k;
+        int j;
+        if (i < 2) {
+          is_k = (i == 0) || n > 1;
+          j = (i == 0) ? 0 : (n > 1 ? 1 : 0);
+        } else {
+          const int q2 = (i - 2) >> 1;   // pairs (V_q2, K_{q2+2}) after the first two K
+          const bool second = ((i - 2) & 1) != 0;
+          if (!second) {
+            is_k = false;
+            j = q2;
+          } else {
+            is_k = q2 + 2 < n;
+            j = is_k ? q2 + 2 : q2 + 1;
+          }
+        }
+        if (!(ok = wait_phase(&kv_empty[ring.stage], ring.phase ^ 1u, abort_flag, kSiteWideProducer))) break;
+        mbar_arrive_expect_tx(&kv_full[ring.stage], Plan::kTileBytes);
+        load_tile(is_k ? &tmap_k : &tmap_v, sKV + ring.stage * Plan::kTileBytes, &kv_full[ring.stage],
+                  j * kBlockN, head_kv, pol_kv);
+        filled |= 1u << ring.stage;
+        fill_par = (fill_par & ~(1u << ring.stage)) | (ring.phase << ring.stage);
+        ring.advance<S>();
+      }
+      drain_phase(q_full, 0u, abort_flag);
+      for (int s = 0; s < S; ++s)
+        if (filled & (1u << s)) drain_phase(&kv_full[s], (fill_par >> s) & 1u, abort_flag);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_base, 0);
+    const uint64_t desc_q = smem_desc_kmajor_sw128(smem_u32(sQ));
+    const uint64_t desc_k = smem_desc_kmajor_sw128(smem_u32(sKV));
+    const uint64_t desc_v = smem_desc_mnmajor_sw128(smem_u32(sKV), Plan::kChunkBytes);
+    auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) tc_commit(bar);
+      __syncwarp();
+    };
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      const bool mine = wait_phase(bar, parity, abort_flag, kSiteWideMma);
+      return __all_sync(0xffffffffu, mine);
+    };
+    Ring ring;
+    // Takes the next ring tile (waits for it); returns its stage.
+    auto next_tile = [&](bool& ok) -> uint32_t {
+      const uint32_t st = ring.stage;
+      ok = wait_all(&kv_full[st], ring.phase);
+      ring.advance<S>();
+      return st;
+    };
+    auto issue_s = [&](int b, uint32_t st) {
+      const uint64_t db = adv(desc_k, st * Plan::kTileBytes);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
+          mma_ss(tmem + b * 128, adv(desc_q, off), adv(db, off), p.idesc_s, kk > 0 ? 1u : 0u);
+        }
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int b, uint32_t st, bool accumulate) {
+      const uint64_t dv = adv(desc_v, st * Plan::kTileBytes);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk)
+          mma_ts(tmem + 256, tmem + b * 128 + kk * 8, adv(dv, kk * 2048), p.idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+    };
+    bool ok = wait_all(q_full, 0u);
+    if (ok) {
+      uint32_t st = next_tile(ok);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, st);
+        commit(s_full);
+        commit(&kv_empty[st]);
+      }
+    }
+    if (ok && n > 1) {
+      uint32_t st = next_tile(ok);
+      if (ok) {
+        tc_fence_after();
+        issue_s(1, st);
+        commit(&s_full[1]);
+        commit(&kv_empty[st]);
+      }
+    }
+    for (int j = 0; j < n && ok; ++j) {
+      const int b = j & 1;
+      if (!(ok = wait_all(&p_full[b], ((uint32_t)j >> 1) & 1u))) break;
+      const uint32_t vst = next_tile(ok);
+      if (!ok) break;
+      tc_fence_after();
+      issue_pv(b, vst, j > 0);
+      commit(pv_done);
+      commit(&kv_empty[vst]);
+      if (j + 2 < n) {
+        const uint32_t kst = next_tile(ok);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(b, kst);
+        commit(&s_full[b]);
+        commit(&kv_empty[kst]);
+      }
+    }
+    if (ok) commit(o_full);
+    commit(drain);
+    drain_phase(drain, 0u, abort_flag);
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ softmax warpgroup
+    const int r = threadIdx.x;                     // query row within the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t t_o = tmem_base + lane_off + 256;
+    const float c = p.c;
+    const int row = qt * kBlockM + r;
+    const int key_lim = p.causal ? min(row, p.N - 1) : (p.N - 1);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n && ok; ++j) {
+      const int b = j & 1;
+      const uint32_t t_s = tmem_base + lane_off + b * 128;
+      if (!(ok = wait_phase(&s_full[b], ((uint32_t)j >> 1) & 1u, abort_flag, kSiteWideSoftmax))) break;
+      tc_fence_after();
+      float s[kBlockN];
+      {
+        uint32_t a0[32], a1[32], a2[32], a3[32];
+        tmem_ld32(t_s + 0, a0);
+        tmem_ld32(t_s + 32, a1);
+        tmem_ld32(t_s + 64, a2);
+        tmem_ld32(t_s + 96, a3);
+        tmem_ld_wait();
+        reg_fence32(a0);
+        reg_fence32(a1);
+        reg_fence32(a2);
+        reg_fence32(a3);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(a0[i]);
+          s[32 + i] = __uint_as_float(a1[i]);
+          s[64 + i] = __uint_as_float(a2[i]);
+          s[96 + i] = __uint_as_float(a3[i]);
+        }
+      }
+      const int k0 = j * kBlockN;
+      if (k0 + kBlockN - 1 > key_lim) {
+#pragma unroll
+        for (int i = 0; i < kBlockN; ++i)
+          if (k0 + i > key_lim) s[i] = -INFINITY;
+      }
+      float mx[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx[e] = max3f(s[e], s[4 + e], s[8 + e]);
+#pragma unroll
+      for (int i = 12; i < kBlockN; i += 8) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[i + e], s[i + 4 + e]);
+      }
+      const float m_new = fmaxf(m, fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]) * c);
+      // Lazy rescale (as in the narrow kernel): the running max moves only when the row's
+      // maximum grew by more than kRescaleLog2, and O (holding blocks < j once P(j-1) V has
+      // completed) and l are then scaled by 2^(m - m_new).
+      bool any_rescale = false;
+      float alpha = 1.f;
+      if (j == 0) {
+        m = m_new;
+      } else {
+        const bool need = m_new > m + kRescaleLog2;
+        any_rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+          alpha = ex2_approx(m - m_new);
+          l *= alpha;
+          m = m_new;
+        }
+      }
+      if (any_rescale) {
+        // P(j-1) V has been issued before S(j+1) and S(j) needed P(j-2) V first, so at most
+        // this one P V is outstanding: its phase is j-1.
+        if (!(ok = wait_phase(pv_done, ((uint32_t)j - 1u) & 1u, abort_flag, kSiteWideSoftmax))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t ov[32];
+          tmem_ld32(t_o + ch * 32, ov);
+          tmem_ld_wait();
+          reg_fence32(ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(t_o + ch * 32, ov);
+        }
+      }
+      // P = 2^(s c - m) -> bf16 pairs over the first 64 columns of S; row sum in fp32.
+      {
+        const float2 c2 = make_float2(c, c);
+        const float2 nm2 = make_float2(-m, -m);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 64; i += 2) {
+            const int col = half * 64 + i;
+            const float2 x = fma2(make_float2(s[col], s[col + 1]), c2, nm2);
+            float2 pr;
+            if (((col >> 1) & 7) < 2) {
+              pr = exp2_poly2(x);
+            } else {
+              pr.x = ex2_approx(x.x);
+              pr.y = ex2_approx(x.y);
+            }
+            acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], pr);
+            pk[i >> 1] = pack_bf16x2(pr.x, pr.y);
+          }
+          tmem_st32(t_s + half * 32, pk);
+        }
+        const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+        l += a.x + a.y;
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    // Epilogue: O / l -> bf16, LSE = (m + log2 l) ln 2.
+    if (ok && wait_phase(o_full, 0u, abort_flag, kSiteWideSoftmax)) {
+      tc_fence_after();
+      const bool row_ok = row < p.N;
+      __nv_bfloat16* orow = p.o + ((size_t)head_q * p.N + (row_ok ? row : 0)) * D;
+      const float inv_l = 1.f / l;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t ov[32];
+        tmem_ld32(t_o + ch * 32, ov);
+        tmem_ld_wait();
+        reg_fence32(ov);
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          packed[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+      if (row_ok) p.lse[(size_t)head_q * p.N + row] = (m + log2f(l)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace attn
