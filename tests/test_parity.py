@@ -13,7 +13,7 @@ import torch
 
 from oracle import attention_forward, attention_rows, head_forward
 from tiled_attention_forward_03_b200.synth import (
-    CFG1, CFG2, CFG3, CFG4, make_qkv, make_workload_inputs, sample_rows, sweep_points)
+    CFG1, CFG2, CFG3, CFG4, make_qkv, make_workload_inputs, sample_rows, sweep_points, wide_points)
 
 pytestmark = pytest.mark.gpu
 
@@ -99,6 +99,14 @@ def test_sweep_point(attn, w):
         check_full(attn, q, k, v, w.causal, w.softmax_scale, w.name)
     else:
         check_sampled(attn, w, q, k, v, count=128, full_heads=())
+
+
+@pytest.mark.parametrize("w", [w for w in wide_points() if w.N == 8192 or not w.causal], ids=lambda w: w.name)
+def test_wide_point_sampled(attn, w):
+    """Head dims 192 and 256 at the benchmark sizes: sampled rows (every tile edge of one head
+    and seeded draws), each computed by the oracle on its own."""
+    q, k, v = make_workload_inputs(w)
+    check_sampled(attn, w, q, k, v, count=96, full_heads=())
 
 
 # ------------------------------------------------------------------ edge shapes

@@ -80,7 +80,20 @@ def sweep_points() -> list[Workload]:
     return pts
 
 
-WORKLOADS = {w.name: w for w in (CFG1, CFG2, CFG3, CFG4, *sweep_points())}
+def wide_points() -> list[Workload]:
+    """Head dims 192 and 256 (beyond the sweep's 64 and 128), same token count per batch."""
+    pts = []
+    i = 0
+    for D in (192, 256):
+        for N in (2048, 8192):
+            for causal in (True, False):
+                tag = "causal" if causal else "noncausal"
+                pts.append(Workload(f"wide_D{D}_N{N}_{tag}", SWEEP_TOKENS // N, 16, 16, N, D, causal, 3000 + i))
+                i += 1
+    return pts
+
+
+WORKLOADS = {w.name: w for w in (CFG1, CFG2, CFG3, CFG4, *sweep_points(), *wide_points())}
 ALIASES = {"cfg1": CFG1.name, "cfg2": CFG2.name, "cfg3": CFG3.name, "cfg4": CFG4.name}
 
 
