@@ -77,7 +77,7 @@ def rot_bf16(x, base=10000.0):
 
 @pytest.mark.parametrize("B,Hq,Hkv,N,D,causal", [
     (1, 2, 2, 256, 128, False), (1, 4, 2, 513, 128, True), (2, 2, 1, 300, 64, True), (1, 2, 2, 1000, 64, False),
-    (1, 2, 2, 200, 96, True), (1, 2, 1, 129, 32, False),
+    (1, 2, 2, 200, 96, True), (1, 2, 1, 129, 32, False), (1, 2, 1, 300, 256, True), (1, 2, 2, 257, 192, False),
 ])
 def test_forward_rope_small(attn, B, Hq, Hkv, N, D, causal):
     q, k, v = make_qkv(B, Hq, Hkv, N, D, 4200 + N)

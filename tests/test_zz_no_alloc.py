@@ -51,6 +51,7 @@ def _close(o, lse, o_ref, lse_ref):
     (4, 16, 16, 2048, 128, False),   # last wave split: the static array holds the partial rows
     (1, 4, 2, 1100, 64, False),      # split, GQA, empty second tile in the last pair
     (2, 8, 2, 1000, 128, True),      # causal: no split, no scratch use
+    (1, 4, 2, 700, 256, False),      # wide head dim: the one-tile kernel, no scratch use
 ])
 def test_noalloc_matches_existing_entry_points_twice(attn, shape):
     B, Hq, Hkv, N, D, causal = shape
