@@ -187,9 +187,12 @@ __device__ __forceinline__ bool unit_at(const FwdParams& p, long long step, int 
 
 // Counts one finished KV range of a split unit and returns how many had finished before
 // it in this launch.  The word holds (epoch << 8) | count; a word left by another launch
-// (different epoch) counts as zero, so the workspace never needs clearing.  Each failed
-// compare-and-swap means another range's update succeeded, so the loop ends after at
-// most `parts` attempts.
+// (different epoch) counts as zero, so the workspace never needs clearing.  The merging
+// range zeroes the words once it has read them, so a launch that completes leaves none
+// behind: the epoch then guards against fresh memory and launches that gave up, and the
+// 24-bit epoch wrapping round, or another copy of the library sharing the workspace, cannot
+// make a stale word look current.  Each failed compare-and-swap means another range's
+// update succeeded, so the loop ends after at most `parts` attempts.
 __device__ __forceinline__ unsigned count_finished(unsigned* cnt, unsigned epoch) {
   unsigned old = atomicAdd(cnt, 0u);
   while (true) {
@@ -763,6 +766,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             *order = have ? 1u : 2u;
+            // Both ranges have counted themselves and the first has published, so nothing
+            // else reads these two words in this launch: they are left at 0 (never an
+            // epoch), and no later launch can take them for its own, whatever its epoch.
+            if (have) {
+              *reinterpret_cast<volatile unsigned*>(cnt) = 0u;
+              *reinterpret_cast<volatile unsigned*>(ready) = 0u;
+            }
           }
           named_bar_sync(1 + t, kBlockM);
           if (*order == 2u) {
