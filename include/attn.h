@@ -96,7 +96,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  *   workspace        device pointer, 256-byte aligned, or NULL (then no split is made)
  *   workspace_bytes  its size; must be >= attn_fwd_workspace_bytes() for the problem
  *                    whenever a split is planned, else ATTN_ERR_INVALID_ARG
- * The workspace needs no initialisation and is left in a state any later call accepts.
+ * The workspace needs no initialisation and is left in a state any later call accepts
+ * (a call from another loaded copy of this library included).
  * Calls that share a workspace must not run concurrently (same stream, or ordered).
  */
 int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse,
