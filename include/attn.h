@@ -297,6 +297,15 @@ const char* attn_version(void);
 /* ---- self-test entry points (used by the library's tests; no part of the forward pass) ---- */
 
 /*
+ * attn_selftest_fast_div -- floor(n / d) computed on the host the way the forward kernel's
+ * scheduler divides by its launch-constant divisors: the high 64 bits of n * m with the
+ * precomputed reciprocal m = ceil(2^64 / d) (Granlund and Montgomery, "Division by
+ * invariant integers using multiplication"; m = 0 stands for d = 1).  No CUDA call.
+ * Returns 0 for d == 0.
+ */
+unsigned int attn_selftest_fast_div(unsigned int n, unsigned int d);
+
+/*
  * attn_selftest_exp2_poly -- evaluate, on the device, the polynomial 2^x that the
  * softmax uses for part of its exponentials (round-to-nearest range reduction,
  * degree-3 minimax polynomial on [-1/2, 1/2], exponent-field scaling; inputs below

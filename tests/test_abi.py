@@ -230,3 +230,28 @@ def test_fp8_empty_problem_is_ok():
 def test_backward_grid_limit():
     # B * Hq * ceil(N/128) above 2^30 is refused on the host
     assert call_bwd(B=1 << 16, Hq=1 << 8, Hkv=1 << 8, N=128 * ((1 << 6) + 1)) == UNSUPPORTED
+
+
+def test_fast_div_equals_floor_division():
+    """The scheduler's division by launch-constant divisors (multiply-high by
+    ceil(2^64 / d)) against exact integer division: every small divisor, powers of two and
+    their neighbours, large divisors, and dividends at 0, around multiples of d and at the
+    top of the 32-bit range (the kernel's counts stay below 2^31)."""
+    import random
+
+    rng = random.Random(11)
+    divisors = list(range(1, 300))
+    for e in range(1, 32):
+        divisors += [(1 << e) - 1, 1 << e, (1 << e) + 1]
+    divisors += [rng.randrange(2, 1 << 32) for _ in range(200)] + [(1 << 32) - 1, (1 << 31) - 1, 3 * 5 * 7 * 11 * 13]
+    top = (1 << 32) - 1
+    for d in divisors:
+        if d > top:
+            continue
+        ns = {0, 1, d - 1, d, d + 1, 2 * d - 1, top, top - 1, (1 << 31) - 1, (top // d) * d, (top // d) * d - 1}
+        ns |= {rng.randrange(0, 1 << 32) for _ in range(40)}
+        ns |= {k * d + r for k in (rng.randrange(0, max(1, top // d)),) for r in (0, d - 1)}
+        for n in ns:
+            if 0 <= n <= top:
+                assert attn.attn_selftest_fast_div(n, d) == n // d, (n, d)
+    assert attn.attn_selftest_fast_div(5, 0) == 0

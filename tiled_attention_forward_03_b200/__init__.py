@@ -92,6 +92,8 @@ def _load() -> ctypes.CDLL:
     L.attn_num_units.restype = ctypes.c_longlong
     L.attn_version.argtypes = []
     L.attn_version.restype = ctypes.c_char_p
+    L.attn_selftest_fast_div.argtypes = [ctypes.c_uint, ctypes.c_uint]
+    L.attn_selftest_fast_div.restype = ctypes.c_uint
     L.attn_selftest_exp2_poly.argtypes = [vp, vp, i, vp]
     L.attn_selftest_exp2_poly.restype = i
     L.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
@@ -184,6 +186,10 @@ def attn_num_units(B: int, Hq: int, N: int) -> int:
 
 def attn_version() -> str:
     return lib.attn_version().decode()
+
+
+def attn_selftest_fast_div(n: int, d: int) -> int:
+    return lib.attn_selftest_fast_div(n, d)
 
 
 def attn_selftest_exp2_poly(x_ptr, y_ptr, n: int, stream) -> int:

@@ -263,6 +263,8 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   if (!supported_head_dim(D) || (e4m3 && D != 64 && D != 128)) return ATTN_ERR_UNSUPPORTED;
   if (e4m3 && (!std::isfinite(qk_descale) || !std::isfinite(o_scale) || qk_descale == 0.f)) return ATTN_ERR_INVALID_ARG;
   if ((long long)B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  // the scheduler indexes work units (256 query rows of one head) in 32 bits
+  if (attn_num_units(B, Hq, N) > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return ATTN_OK;  // empty problem: nothing to compute or write
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
@@ -327,6 +329,10 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   p.causal = causal ? 1 : 0;
   p.units_per_step = p.causal ? 2 : 1;
   p.num_steps = p.causal ? (long long)B * Hq * ((p.num_pairs + 1) / 2) : p.num_units;
+  p.div_pairs = attn::make_fast_div((uint32_t)p.num_pairs);
+  p.div_steps = attn::make_fast_div((uint32_t)((p.num_pairs + 1) / 2));
+  p.div_hq = attn::make_fast_div((uint32_t)Hq);
+  p.div_group = attn::make_fast_div((uint32_t)p.group);
   // c > 0 always: masked scores are -inf and -inf * c must stay -inf.  For scale == 0 every
   // allowed score gives 2^(tiny) == 1 in fp32, the same softmax as c == 0.
   // (E4M3: the scores carry the product of the Q and K descales; its sign joins scale's.)
@@ -479,6 +485,12 @@ int attn_device_status(void* stream, int* site) {
   }
   if (site) *site = (int)value;
   return value ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+unsigned int attn_selftest_fast_div(unsigned int n, unsigned int d) {
+  if (d == 0u) return 0u;
+  const attn::FastDiv f = attn::make_fast_div(d);
+  return f.m ? (unsigned int)(((unsigned __int128)n * f.m) >> 64) : n;
 }
 
 int attn_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {

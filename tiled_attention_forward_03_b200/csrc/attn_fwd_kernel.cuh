@@ -100,6 +100,29 @@ struct SmemPlan {
   static constexpr int kAlloc = kBytes + 1024;              // slack for 1024-byte alignment
 };
 
+// Division by a divisor fixed for the launch, as a multiply-high by a precomputed reciprocal
+// (T. Granlund and P. L. Montgomery, "Division by invariant integers using multiplication",
+// PLDI 1994): with m = ceil(2^64 / d), floor(n / d) is the high 64 bits of n * m for every
+// n < 2^32 and 2 <= d < 2^32, since n * m / 2^64 = n / d + n * (m - 2^64 / d) / 2^64 and the
+// second term is below 2^-32 <= 1 / d.  m = 0 stands for d = 1.  The scheduler evaluates
+// its work items with these: on the MMA warp a new unit waits for that arithmetic, where a
+// 64-bit division costs hundreds of cycles.
+struct FastDiv {
+  unsigned long long m;
+  uint32_t d;
+};
+
+inline FastDiv make_fast_div(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.m = d > 1u ? ~0ull / d + 1ull : 0ull;
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+  return f.m ? (uint32_t)__umul64hi((unsigned long long)n, f.m) : n;
+}
+
 struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
@@ -121,6 +144,11 @@ struct FwdParams {
   float* ws_ml;       // first range's (m, l) [tail_units][2 tiles][128 rows] float2
   unsigned* ws_cnt;   // [tail_units][2 tiles][2]: finished ranges ((epoch << 8) | count), ready flag (epoch)
   unsigned epoch;     // launch tag (24 bits, non-zero): counts of other launches read as 0
+  // divisors of the schedule (all counts below 2^31: checked on the host)
+  FastDiv div_pairs;  // num_pairs
+  FastDiv div_steps;  // (num_pairs + 1) / 2: causal scheduling steps per head
+  FastDiv div_hq;     // Hq
+  FastDiv div_group;  // group
   float c;           // |scale| * log2(e) (times the Q and K descales for E4M3 inputs)
   float o_scale;     // multiplies the normalised output (the V descale for E4M3 inputs, else 1)
   uint32_t idesc_s;  // S = Q K^T instruction descriptor (negates A when scale < 0)
@@ -140,13 +168,13 @@ struct Unit {
   int tail;        // index of the split unit among the tail units
 };
 
-__device__ __forceinline__ Unit make_unit(const FwdParams& p, long long head, int pair) {
+__device__ __forceinline__ Unit make_unit(const FwdParams& p, uint32_t head, int pair) {
   Unit w;
-  const int hq = (int)(head % p.Hq);
-  const int b = (int)(head / p.Hq);
+  const uint32_t b = fast_div(head, p.div_hq);
+  const uint32_t hq = head - b * (uint32_t)p.Hq;
   w.q0 = pair * 2 * kBlockM;
   w.head_q = (int)head;
-  w.head_kv = b * p.Hkv + hq / p.group;
+  w.head_kv = (int)(b * (uint32_t)p.Hkv + fast_div(hq, p.div_group));
   w.valid1 = (w.q0 + kBlockM) < p.N;
   if (p.causal) {
     w.n0 = min(p.num_blocks, 2 * pair + 1);
@@ -170,15 +198,14 @@ __device__ __forceinline__ Unit make_unit(const FwdParams& p, long long head, in
 // one head (and the heads of one GQA group are consecutive), so K/V tiles are shared
 // through L2 by the CTAs running at the same time.  Returns false if the step has no
 // such unit (the middle pair of a head with an odd pair count).
-__device__ __forceinline__ bool unit_at(const FwdParams& p, long long step, int part, Unit& w) {
+__device__ __forceinline__ bool unit_at(const FwdParams& p, uint32_t step, int part, Unit& w) {
   if (!p.causal) {
-    const long long head = step / p.num_pairs;
-    w = make_unit(p, head, (int)(step - head * p.num_pairs));
+    const uint32_t head = fast_div(step, p.div_pairs);
+    w = make_unit(p, head, (int)(step - head * (uint32_t)p.num_pairs));
     return true;
   }
-  const int steps_per_head = (p.num_pairs + 1) / 2;
-  const long long head = step / steps_per_head;
-  const int s = (int)(step - head * steps_per_head);
+  const uint32_t head = fast_div(step, p.div_steps);
+  const int s = (int)(step - head * p.div_steps.d);
   const int pair = part == 0 ? p.num_pairs - 1 - s : s;
   if (part == 1 && pair == p.num_pairs - 1 - s) return false;
   w = make_unit(p, head, pair);
@@ -212,26 +239,27 @@ __device__ __forceinline__ int item_at(const FwdParams& p, int it, Unit& w) {
   if (p.causal) {
     const long long step = blockIdx.x + (long long)(it >> 1) * gridDim.x;
     if (step >= p.num_steps) return 0;
-    return unit_at(p, step, it & 1, w) ? 1 : 2;
+    return unit_at(p, (uint32_t)step, it & 1, w) ? 1 : 2;
   }
   if (p.parts <= 1 || it < p.whole_per_cta) {
     const long long u = blockIdx.x + (long long)it * gridDim.x;
     if (u >= p.num_units) return 0;
-    const long long head = u / p.num_pairs;
-    w = make_unit(p, head, (int)(u - head * p.num_pairs));
+    const uint32_t head = fast_div((uint32_t)u, p.div_pairs);
+    w = make_unit(p, head, (int)((uint32_t)u - head * (uint32_t)p.num_pairs));
     return 1;
   }
   if (it > p.whole_per_cta) return 0;
-  const int q = blockIdx.x;
-  if (q >= p.tail_units * p.parts) return 0;
-  const long long u = (long long)p.whole_per_cta * gridDim.x + q / p.parts;
-  const long long head = u / p.num_pairs;
-  w = make_unit(p, head, (int)(u - head * p.num_pairs));
+  const uint32_t q = blockIdx.x;
+  const uint32_t parts = (uint32_t)p.parts;
+  if (q >= (uint32_t)p.tail_units * parts) return 0;
+  const uint32_t u = (uint32_t)p.whole_per_cta * gridDim.x + q / parts;
+  const uint32_t head = fast_div(u, p.div_pairs);
+  w = make_unit(p, head, (int)(u - head * (uint32_t)p.num_pairs));
   w.parts = p.parts;
-  w.part = q % p.parts;
-  w.tail = q / p.parts;
-  w.jb = (int)((long long)w.part * p.num_blocks / p.parts);
-  w.n0 = w.n1 = w.nmax = (int)((long long)(w.part + 1) * p.num_blocks / p.parts);
+  w.part = (int)(q % parts);
+  w.tail = (int)(q / parts);
+  w.jb = (int)((uint32_t)w.part * (uint32_t)p.num_blocks / parts);
+  w.n0 = w.n1 = w.nmax = (int)((uint32_t)(w.part + 1) * (uint32_t)p.num_blocks / parts);
   return 1;
 }
 
