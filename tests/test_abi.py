@@ -255,3 +255,11 @@ def test_fast_div_equals_floor_division():
             if 0 <= n <= top:
                 assert attn.attn_selftest_fast_div(n, d) == n // d, (n, d)
     assert attn.attn_selftest_fast_div(5, 0) == 0
+
+
+def test_work_unit_count_limit():
+    """The scheduler indexes work units (256 query rows of one head) in 32 bits: a problem with
+    2^31 or more of them is refused before any CUDA call, even when B*Hq itself fits."""
+    B, Hq = 1 << 20, 1 << 10                      # B*Hq = 2^30
+    assert call(B=B, Hq=Hq, Hkv=Hq, N=2048) == UNSUPPORTED   # 2^30 heads x 8 units
+    assert call(B=B, Hq=Hq, Hkv=Hq, N=512) == UNSUPPORTED    # exactly 2^31 units
