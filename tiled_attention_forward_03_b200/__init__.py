@@ -220,9 +220,12 @@ def _check(t, name, dtype, shape):
 _workspaces: dict = {}
 
 
-def _workspace(device, nbytes: int, purpose: str = "fwd"):
+def _workspace(device, nbytes: int, purpose: str = "fwd", stream=None):
     """A cached device buffer of at least nbytes, per device and purpose ("fwd": the
-    split-tail schedule, "bwd": the backward pass's per-row delta and LSE)."""
+    split-tail schedule, "bwd": the backward pass's per-row delta and LSE, "rope": the
+    rotated q and k).  The buffer is marked as used on ``stream``, so that when a larger one
+    replaces it, torch's allocator does not hand its memory to another stream's allocation
+    before the kernels enqueued on ``stream`` have finished with it."""
     import torch
 
     key = (device.type, device.index, purpose)
@@ -230,6 +233,8 @@ def _workspace(device, nbytes: int, purpose: str = "fwd"):
     if buf is None or buf.numel() < nbytes:
         buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
         _workspaces[key] = buf
+    if stream is not None:
+        buf.record_stream(stream)
     return buf
 
 
@@ -266,7 +271,7 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
         if ws_bytes < 0:
             raise AttnError(ATTN_ERR_CUDA, "attn_fwd_workspace_bytes")
         if ws_bytes > 0:
-            ws = _workspace(q.device, ws_bytes)
+            ws = _workspace(q.device, ws_bytes, stream=s)
             st = attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                              B, Hq, Hkv, N, D, causal, scale, ws.data_ptr(), ws.numel(), s.cuda_stream)
         else:
@@ -413,7 +418,7 @@ def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
         ws_bytes = attn_bwd_workspace_bytes(B, Hq, N)
         if ws_bytes < 0:
             raise AttnError(ATTN_ERR_INVALID_ARG, "attn_bwd_workspace_bytes")
-        ws = _workspace(q.device, max(ws_bytes, 256), "bwd")
+        ws = _workspace(q.device, max(ws_bytes, 256), "bwd", stream=s)
         st = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, N, D, causal, scale,
                       ws.data_ptr(), ws.numel(), s.cuda_stream)
@@ -481,7 +486,7 @@ def forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float, c
         ws_bytes = attn_fwd_workspace_bytes(B, Hq, N, D, causal) if split else 0
         if ws_bytes < 0:
             raise AttnError(ATTN_ERR_CUDA, "attn_fwd_workspace_bytes")
-        ws = _workspace(q.device, ws_bytes) if ws_bytes > 0 else None
+        ws = _workspace(q.device, ws_bytes, stream=s) if ws_bytes > 0 else None
         st = attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N,
                           D, causal, scale, q_descale, k_descale, v_descale, ws.data_ptr() if ws is not None else None,
                           ws.numel() if ws is not None else 0, s.cuda_stream)
@@ -552,7 +557,7 @@ def forward_rope(q, k, v, cos_t, sin_t, causal: bool = False, scale: float | Non
         nbytes = attn_fwd_rope_workspace_bytes(B, Hq, Hkv, N, D)
         if nbytes < 0:
             raise AttnError(ATTN_ERR_CUDA, "attn_fwd_rope_workspace_bytes")
-        ws = _workspace(q.device, max(nbytes, 256), "rope")
+        ws = _workspace(q.device, max(nbytes, 256), "rope", stream=s)
         st = attn_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), cos_t.data_ptr(), sin_t.data_ptr(),
                            out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, D, causal, scale, ws.data_ptr(),
                            ws.numel(), s.cuda_stream)
