@@ -34,3 +34,20 @@ def test_warmup_below_three_is_refused():
     proc = run_bench("--impl", "reference", "--warmup", "2", "--steps", "1")
     assert proc.returncode != 0
     assert "--warmup" in proc.stderr
+
+
+def test_reference_arm_under_two_ranks_prints_on_rank_zero_only():
+    """Launched by torchrun with N > 1, the reference arm runs on rank 0 alone (the oracle on the
+    host cores); the other ranks exit 0 without work or output."""
+    outs = {}
+    for rank in (0, 1):
+        env = dict(os.environ, WORLD_SIZE="2", RANK=str(rank), LOCAL_RANK=str(rank))
+        proc = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                               "--workload", "cfg1", "--steps", "1", "--warmup", "3"],
+                              capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
+        assert proc.returncode == 0, proc.stderr
+        outs[rank] = [l for l in proc.stdout.splitlines() if l.strip()]
+    assert outs[1] == []
+    assert len(outs[0]) == 1
+    line = json.loads(outs[0][0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
