@@ -40,7 +40,7 @@ def _rank_main(rank, world, port, out):
 def test_two_gloo_ranks_agree_on_slowest_time_and_draw_distinct_batches():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:   # no fork of a multi-threaded process
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
