@@ -13,7 +13,9 @@ its own (tests/oracle_pins.py); every other pin is independent of the oracle.
 """
 from __future__ import annotations
 
+import json
 import math
+import os
 
 import numpy as np
 import torch
@@ -228,8 +230,23 @@ def pin_bwd_linear_in_do(impl):
         _close(z, 2.0 * x - 3.0 * y, 1e-12, f"linearity {name}")
 
 
+GOLDEN_BWD = os.path.join(os.path.dirname(__file__), "golden", "tiny_backward_closed_form.json")
+
+
+def pin_bwd_golden(impl):
+    """Hand-derived closed forms stored in tests/golden/tiny_backward_closed_form.json (two keys,
+    D = 1: non-causal at scale 1 and 2, causal, and two query heads sharing one KV head)."""
+    with open(GOLDEN_BWD) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        q, k, v, do = (np.array(c[x], dtype=np.float64) for x in ("q", "k", "v", "do"))
+        dq, dk, dv = impl(q, k, v, do, c["causal"], c["scale"])
+        for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
+            _close(got, np.array(c[name]), 1e-12, f"golden {c['name']} {name}")
+
+
 ALL_BWD_PINS = [
-    pin_bwd_finite_differences, pin_bwd_torch_autograd, pin_bwd_brute_force, pin_bwd_dv_sums,
+    pin_bwd_golden, pin_bwd_finite_differences, pin_bwd_torch_autograd, pin_bwd_brute_force, pin_bwd_dv_sums,
     pin_bwd_dk_sums_zero, pin_bwd_key_shift, pin_bwd_uniform, pin_bwd_identical_v, pin_bwd_single_key,
     pin_bwd_causal_first_query, pin_bwd_gqa_is_repeated_mha, pin_bwd_linear_in_do,
 ]
