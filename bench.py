@@ -127,10 +127,10 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
         self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w", prefix="clocks_", suffix=".csv", delete=False)
+        self.path = self.f.name
         try:
-            self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
@@ -139,6 +139,8 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
+            self.f.close()
+            os.unlink(self.path)
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         time.sleep(0.25)
         self.proc.terminate()

@@ -51,3 +51,38 @@ def test_reference_arm_under_two_ranks_prints_on_rank_zero_only():
     assert len(outs[0]) == 1
     line = json.loads(outs[0][0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
+
+
+def test_clock_sampler_parses_nvidia_smi_rows(tmp_path, monkeypatch):
+    """The clock record of the timed region, from a stand-in nvidia-smi on PATH that prints
+    four samples (one idle) in the query's CSV form and then waits to be stopped."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    fake = tmp_path / "nvidia-smi"
+    rows = ["0, 1965, 1965, 120.5, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+            "0, 1900, 1965, 560.0, 100, 0x4, Not Active, Not Active, Not Active, Active",
+            "0, 1880, 1965, 571.5, 100, 0x4, Not Active, Not Active, Not Active, Active",
+            "0, 1920, 1965, 540.0, 99, 0x0, Not Active, Not Active, Not Active, Not Active"]
+    fake.write_text("#!/bin/sh\n" + "".join(f"echo '{r}'\n" for r in rows) + "exec sleep 30\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", f"{tmp_path}{os.pathsep}{os.environ['PATH']}")
+    sampler = bench.ClockSampler(0)
+    path = sampler.path
+    rec = sampler.stop()
+    assert rec["samples"] == 3                      # the idle row is left out
+    assert rec["sm_mhz"] == 1900.0 and rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["sw_power_cap"] and rec["power_w_max"] == 571.5
+    assert not os.path.exists(path)
+
+
+def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    monkeypatch.setenv("PATH", str(tmp_path))
+    sampler = bench.ClockSampler(0)
+    path = sampler.path
+    rec = sampler.stop()
+    assert rec["samples"] == 0 and rec["reasons"] == ["nvidia-smi unavailable"]
+    assert not os.path.exists(path)
