@@ -5,10 +5,11 @@
                     [--pass fwd|bwd]
 
 One step = one attention forward pass over the workload's batch (one kernel
-launch).  Default workload: B=4, Hq=Hkv=16, N=2048, D=128, non-causal, bf16
-inputs drawn i.i.d. N(0,1) from a seeded CPU generator.  Its inputs (100 MB)
-fit in the 126 MB L2, so a 512 MB buffer is written between timed steps to
-flush L2; each step's kernel is timed with CUDA events on its launching stream.
+launch).  Default workload: the largest configuration, GQA B=8, Hq=32, Hkv=8,
+N=8192, D=128, causal, bf16 inputs drawn i.i.d. N(0,1) from a seeded CPU
+generator (768 MiB of inputs, 520 MiB of outputs).  A 512 MB buffer is written
+between timed steps to flush the 126 MB L2 (smaller workloads' inputs would fit
+in it); each step's kernel is timed with CUDA events on its launching stream.
 
 FLOPs counted: 4*B*Hq*N^2*D, halved for causal.  `value` is the whole-job
 throughput (all ranks' FLOPs / the slowest rank's time).  With N>1 GPUs
@@ -49,7 +50,7 @@ sys.path.insert(0, ROOT)
 DATASHEET_BF16_TFLOPS = 2250.0   # B200 dense BF16 (no sparsity)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-DEFAULT_WORKLOAD = "cfg2"
+DEFAULT_WORKLOAD = "cfg4"
 METRIC = "attention fwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
 METRIC_FP8 = "attention fwd E4M3 (FP8) TFLOP/s (1 B200) and % of dense FP8 tensor peak"
 FP8_OVER_BF16 = 2.0  # nominal dense E4M3 / bf16 tensor rate (4.5 / 2.25 PFLOP/s)
@@ -200,6 +201,13 @@ def profile_traffic(workload_name: str, which: str = "fwd"):
     return d.get("dram_bytes_per_launch")
 
 
+def bench_config(w, pass_: str, world: int) -> dict:
+    """The `config` object of the JSON line; both arms print the same one."""
+    return {**w.describe(), "pass": PASS_NAMES[pass_],
+            "l2": "flushed between timed steps (512 MB write)",
+            "parallelism": f"replicas{world}: each rank its own batch, no collective on the data path"}
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 
 def cpu_threads():
@@ -223,7 +231,7 @@ def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = Fa
 
     Returns (TFLOP/s, FLOPs done, seconds, heads done, sample description)."""
     from oracle import head_backward, head_forward, rope_rotate
-    from tiled_attention_forward_03_b200.synth import make_dout, make_qkv, make_qkv_e4m3
+    from attn_inputs import make_dout, make_qkv, make_qkv_e4m3
 
     q, k, v = make_qkv(1, w.Hq, w.Hkv, w.N, w.D, w.seed)  # one batch row holds all heads
     do = make_dout(1, w.Hq, w.N, w.D, w.seed + 500) if backward else None
@@ -264,7 +272,7 @@ def run_ours(args, w):
     dist = init_dist(world, "nccl")
 
     import tiled_attention_forward_03_b200 as attn
-    from tiled_attention_forward_03_b200.synth import make_dout, make_qkv, make_qkv_e4m3
+    from attn_inputs import make_dout, make_qkv, make_qkv_e4m3
 
     fp8 = args.pass_ == "fp8"
     if fp8:
@@ -435,9 +443,7 @@ def run_ours(args, w):
         "vs_baseline": None,
         "dtype": "e4m3" if fp8 else "bf16",
         "data": "synthetic",
-        "config": {**w.describe(), "pass": PASS_NAMES[args.pass_],
-                   "l2": "flushed between timed steps (512 MB write)",
-                   "parallelism": f"replicas{world}: each rank its own batch, no collective on the data path"},
+        "config": bench_config(w, args.pass_, world),
         "pct_of_dense_bf16_peak" if not fp8 else "pct_of_dense_fp8_peak":
             round(100.0 * value / world / (DATASHEET_BF16_TFLOPS * (FP8_OVER_BF16 if fp8 else 1.0)), 2),
         "pct_of_measured_bf16_peak" if not fp8 else "pct_of_measured_fp8_peak": round(100.0 * value / world / peak_burst, 2),
@@ -504,7 +510,7 @@ def run_reference(args, w):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {**w.describe(), "pass": PASS_NAMES[args.pass_]},
+        "config": bench_config(w, args.pass_, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -513,7 +519,7 @@ def run_reference(args, w):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)  # cfg2 forward: ~0.4 s of timed region (clock samples)
+    ap.add_argument("--steps", type=int, default=200)  # cfg4 forward: ~0.7 s of timed region (clock samples)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     help="cfg1..cfg4, a sweep point name (e.g. sweep_D128_N8192_causal), or 'all'")
@@ -527,7 +533,7 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
-    from tiled_attention_forward_03_b200.synth import WORKLOADS, get_workload
+    from attn_inputs import WORKLOADS, get_workload
 
     names = list(WORKLOADS) if args.workload == "all" else [args.workload]
     for i, name in enumerate(names):

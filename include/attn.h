@@ -130,8 +130,11 @@ long long attn_fwd_workspace_bytes(int B, int Hq, int N, int D, int causal);
  *   - Problems whose split needs more than the array (attn_fwd_workspace_bytes() larger
  *     than attn_fwd_noalloc_scratch_bytes(); not reachable at D <= 128 on a 148-SM B200)
  *     are rejected with ATTN_ERR_UNSUPPORTED and a message in attn_last_cuda_error().
- *   - The first call on a device looks up the array's device address and clears the
- *     array (a synchronous cudaMemset); make that first call before any stream capture.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any
+ *     stream capture.  A failed look-up returns ATTN_ERR_CUDA and is retried by the next
+ *     call.  Nothing is cleared: the array starts at zero when the library loads, and the
+ *     kernel tags its counter words with a per-launch epoch and zeroes them after use.
  *   - Every call shares the one array and leaves its contents behind; no later call
  *     needs them cleared.  Calls whose kernels overlap on the GPU (different streams
  *     without ordering) race on the array and must be avoided.

@@ -11,7 +11,6 @@ from .attn_ref import (  # noqa: F401
     attention_rows,
     head_backward,
     head_forward,
-    head_probs,
     head_scores,
     kv_head,
     rope_angles,

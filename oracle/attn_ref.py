@@ -69,14 +69,6 @@ def head_scores(qh: np.ndarray, kh: np.ndarray, causal: bool, scale: float) -> n
     return S
 
 
-def head_probs(qh, kh, causal: bool, scale: float) -> np.ndarray:
-    """Row-softmax of the head's score matrix (each row sums to 1)."""
-    S = head_scores(_as_f64(qh), _as_f64(kh), causal, scale)
-    m = S.max(axis=1, keepdims=True)
-    E = np.exp(S - m)
-    return E / E.sum(axis=1, keepdims=True)
-
-
 def head_forward(qh, kh, vh, causal: bool, scale: float):
     """One head: returns (O [N, D], LSE [N]) in fp64."""
     qh, kh, vh = _as_f64(qh), _as_f64(kh), _as_f64(vh)

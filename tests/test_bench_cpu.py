@@ -86,3 +86,23 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
     rec = sampler.stop()
     assert rec["samples"] == 0 and rec["reasons"] == ["nvidia-smi unavailable"]
     assert not os.path.exists(path)
+
+
+def test_reference_arm_loads_none_of_the_libraries_own_code():
+    """The reference arm is the fp64 oracle alone: it must not map the CUDA library (nor import
+    the package that loads it), and it prints the same `config` object as the CUDA arm."""
+    code = ("import sys; sys.argv=['bench.py']; import bench; "
+            "bench.main(['--impl','reference','--workload','cfg1','--steps','1','--warmup','3']); "
+            "maps=open('/proc/self/maps').read(); "
+            "print('MAPPED' if 'libattn_fwd' in maps else 'CLEAN'); "
+            "print('PKG' if 'tiled_attention_forward_03_b200' in sys.modules else 'NOPKG')")
+    proc = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert proc.returncode == 0, proc.stderr
+    out = proc.stdout.splitlines()
+    assert out[-2:] == ["CLEAN", "NOPKG"]
+    line = json.loads(out[0])
+    sys.path.insert(0, ROOT)
+    import bench
+    from attn_inputs import get_workload
+
+    assert line["config"] == bench.bench_config(get_workload("cfg1"), "fwd", 1)

@@ -54,7 +54,7 @@ def test_single_rank_needs_no_process_group():
 
 
 def test_whole_job_value_counts_every_rank():
-    from tiled_attention_forward_03_b200.synth import get_workload
+    from attn_inputs import get_workload
     w = get_workload("cfg2")
     # value = world * flops * steps / slowest time: two ranks at the same speed double it
     one = 1 * w.flops * 10 / 1.0

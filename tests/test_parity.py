@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from oracle import attention_forward, attention_rows, head_forward
-from tiled_attention_forward_03_b200.synth import (
+from attn_inputs import (
     CFG1, CFG2, CFG3, CFG4, make_qkv, make_workload_inputs, sample_rows, sweep_points, wide_points)
 
 pytestmark = pytest.mark.gpu
@@ -66,8 +66,19 @@ def check_sampled(attn, w, q, k, v, count=256, full_heads=((0, 0),)):
     for (b, h) in full_heads:
         oh, lh = head_forward(q[b, h], k[b, h // g], v[b, h // g], w.causal, w.softmax_scale)
         assert_close(o[b, h], lse[b, h], oh, lh, f"{w.name} head {(b, h)}")
-    # properties at any size: finite everywhere, LSE >= the row's largest allowed score
+    # properties at any size: finite everywhere; on the sampled rows, the row's largest allowed
+    # score m_i <= LSE_i <= m_i + ln(number of allowed keys) (bounds of a log-sum-exp)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    check_lse_bounds(lse, q, k, rows, w.causal, w.softmax_scale, g)
+
+
+def check_lse_bounds(lse, q, k, rows, causal, scale, g):
+    for (b, h, i) in rows:
+        qi = q[b, h, i].double()
+        kk = k[b, h // g].double()
+        n = (i + 1) if causal else kk.shape[0]
+        m = float((scale * (kk[:n] @ qi)).max())
+        assert m - TOL_LSE <= lse[b, h, i] <= m + math.log(n) + TOL_LSE, (b, h, i, m, lse[b, h, i])
 
 
 # ------------------------------------------------------------------ the five workloads
@@ -101,10 +112,11 @@ def test_sweep_point(attn, w):
         check_sampled(attn, w, q, k, v, count=128, full_heads=())
 
 
-@pytest.mark.parametrize("w", [w for w in wide_points() if w.N == 8192 or not w.causal], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", wide_points(), ids=lambda w: w.name)
 def test_wide_point_sampled(attn, w):
-    """Head dims 192 and 256 at the benchmark sizes: sampled rows (every tile edge of one head
-    and seeded draws), each computed by the oracle on its own."""
+    """Head dims 192 and 256 at every benchmark size (N = 2048 and 8192, causal and not):
+    sampled rows (every tile edge of one head and seeded draws), each computed by the oracle on
+    its own."""
     q, k, v = make_workload_inputs(w)
     check_sampled(attn, w, q, k, v, count=96, full_heads=())
 

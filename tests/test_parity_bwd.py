@@ -24,7 +24,7 @@ import pytest
 import torch
 
 from oracle import attention_backward, head_backward
-from tiled_attention_forward_03_b200.synth import CFG2, CFG3, CFG4, make_dout, make_qkv
+from attn_inputs import CFG2, CFG3, CFG4, make_dout, make_qkv
 
 pytestmark = pytest.mark.gpu
 

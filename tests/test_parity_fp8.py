@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from oracle import attention_forward, attention_rows
-from tiled_attention_forward_03_b200.synth import CFG2, make_qkv_e4m3
+from attn_inputs import CFG2, make_qkv_e4m3
 
 pytestmark = pytest.mark.gpu
 
@@ -93,3 +93,21 @@ def test_fp8_cfg2_sampled(attn):
     o_ref, lse_ref = attention_rows(q, k, v, rows, w.causal, w.softmax_scale)
     idx = tuple(np.array(x) for x in zip(*rows))
     assert_close(o[idx], lse[idx], o_ref, lse_ref, "fp8 cfg2 sampled rows")
+
+
+@pytest.mark.parametrize("name", ["cfg3", "sweep_D128_N8192_noncausal", "sweep_D64_N4096_noncausal",
+                                  "sweep_D64_N4096_causal"])
+def test_fp8_benchmark_workloads_sampled(attn, name):
+    """Every workload the E4M3 pass is benchmarked on, at full size: seeded sampled rows (every
+    128-row tile edge of one head plus uniform draws), each computed by the oracle on its own
+    from the dequantized inputs."""
+    from attn_inputs import get_workload, sample_rows
+
+    w = get_workload(name)
+    q8, k8, v8, ds = make_qkv_e4m3(w.B, w.Hq, w.Hkv, w.N, w.D, w.seed)
+    o, lse = run(attn, q8, k8, v8, ds, w.causal, w.softmax_scale)
+    rows = sample_rows(w.B, w.Hq, w.N, 96, seed=w.seed + 11)
+    q, k, v = (x.float() * ds for x in (q8, k8, v8))
+    o_ref, lse_ref = attention_rows(q, k, v, rows, w.causal, w.softmax_scale)
+    idx = tuple(np.array(x) for x in zip(*rows))
+    assert_close(o[idx], lse[idx], o_ref, lse_ref, f"fp8 {w.name} sampled rows")

@@ -16,7 +16,7 @@ import pytest
 import torch
 
 from oracle import attention_forward, attention_forward_rope, attention_rows, rope_rotate
-from tiled_attention_forward_03_b200.synth import CFG2, make_qkv
+from attn_inputs import CFG2, make_qkv
 
 pytestmark = pytest.mark.gpu
 

@@ -63,7 +63,7 @@ def test_device_exp2_poly_error_bound(attn):
 @pytest.mark.gpu
 def test_bounded_wait_reports_timeout_and_context_survives(attn):
     import torch
-    from tiled_attention_forward_03_b200.synth import make_qkv
+    from attn_inputs import make_qkv
     s = torch.cuda.current_stream().cuda_stream
     assert attn.attn_device_status(s) == (attn.ATTN_OK, 0)
     assert attn.attn_selftest_wait_timeout(20000, s) == attn.ATTN_OK      # 20 ms limit

@@ -18,7 +18,7 @@ import pytest
 import torch
 
 from oracle import attention_forward
-from tiled_attention_forward_03_b200.synth import make_qkv
+from attn_inputs import make_qkv
 
 pytestmark = pytest.mark.gpu
 

@@ -6,7 +6,7 @@ import math
 import pytest
 import torch
 
-from tiled_attention_forward_03_b200 import synth
+import attn_inputs as synth
 
 
 def test_the_four_configurations():

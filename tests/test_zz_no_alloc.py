@@ -2,10 +2,12 @@
 
 Such callers (code whose device memory belongs to another allocator, or that must not
 risk the synchronisation an allocation can cause) cannot hand attn_fwd_ws a workspace.
-attn_fwd_noalloc runs the same kernel with its workspace in a static device array of the
-library.  These tests call it through the C ABI and compare it with the existing entry
-points, twice in a row (the array keeps the previous call's contents).  The file is
-named to be collected last.
+attn_fwd_noalloc runs the same kernel with the same schedule, its workspace a static
+device array of the library.  These tests call it through the C ABI and require it to
+equal attn_fwd_ws (given a workspace of its own of the size the schedule needs) bit for
+bit, twice in a row (the array keeps the previous call's contents), with the first call of
+the process on a side stream; one shape is also compared with the fp64 oracle.  The file
+is named to be collected last.
 """
 import math
 
@@ -13,13 +15,10 @@ import numpy as np
 import pytest
 import torch
 
-from tiled_attention_forward_03_b200.synth import make_qkv
+from attn_inputs import make_qkv
+from oracle import attention_forward
 
 pytestmark = pytest.mark.gpu
-
-TOL_O_MAX = 2e-2
-TOL_O_MEAN = 2e-3
-TOL_LSE = 1e-3
 
 
 @pytest.fixture(scope="module")
@@ -30,41 +29,75 @@ def attn():
     return mod
 
 
-def _noalloc(attn, q, k, v, causal, scale):
+def _outputs(q):
     B, Hq, N, D = q.shape
     o = torch.full_like(q, float("nan"))
     lse = torch.full((B, Hq, N), float("nan"), dtype=torch.float32, device=q.device)
+    return o, lse
+
+
+def _noalloc(attn, q, k, v, causal, scale, stream):
+    B, Hq, N, D = q.shape
+    o, lse = _outputs(q)
     st = attn.attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                               B, Hq, k.shape[1], N, D, causal, scale, torch.cuda.current_stream().cuda_stream)
+                               B, Hq, k.shape[1], N, D, causal, scale, stream.cuda_stream)
     assert st == attn.ATTN_OK, attn.attn_status_string(st) + " " + attn.attn_last_cuda_error()
     return o, lse
 
 
-def _close(o, lse, o_ref, lse_ref):
-    d = (o.float() - o_ref.float()).abs()
-    dl = (lse - lse_ref).abs()
-    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
-    assert d.max().item() <= TOL_O_MAX and d.mean().item() <= TOL_O_MEAN and dl.max().item() <= TOL_LSE
+def _with_workspace(attn, q, k, v, causal, scale, stream):
+    """attn_fwd_ws with a workspace of exactly the size the split schedule needs (or none)."""
+    B, Hq, N, D = q.shape
+    need = attn.attn_fwd_workspace_bytes(B, Hq, N, D, causal)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    o, lse = _outputs(q)
+    st = attn.attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq,
+                          k.shape[1], N, D, causal, scale, ws.data_ptr() if need > 0 else None, need,
+                          stream.cuda_stream)
+    assert st == attn.ATTN_OK, attn.attn_status_string(st)
+    return o, lse
 
 
-@pytest.mark.parametrize("shape", [
+SHAPES = [
     (4, 16, 16, 2048, 128, False),   # last wave split: the static array holds the partial rows
     (1, 4, 2, 1100, 64, False),      # split, GQA, empty second tile in the last pair
     (2, 8, 2, 1000, 128, True),      # causal: no split, no scratch use
     (1, 4, 2, 700, 256, False),      # wide head dim: the one-tile kernel, no scratch use
-])
-def test_noalloc_matches_existing_entry_points_twice(attn, shape):
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B{}_Hq{}_Hkv{}_N{}_D{}_{}".format(*s[:5], "c" if s[5] else "nc"))
+def test_noalloc_equals_workspace_entry_point_bitwise_twice(attn, shape):
     B, Hq, Hkv, N, D, causal = shape
     need = attn.attn_fwd_workspace_bytes(B, Hq, N, D, causal)
     assert 0 <= need <= attn.attn_fwd_noalloc_scratch_bytes()
     q, k, v = (x.cuda() for x in make_qkv(B, Hq, Hkv, N, D, seed=6000 + N))
     scale = 1.0 / math.sqrt(D)
-    o_ref, lse_ref = attn.forward(q, k, v, causal=causal, scale=scale)           # attn_fwd_ws / attn_fwd
-    for _ in range(2):                                                            # two calls in a row
-        o, lse = _noalloc(attn, q, k, v, causal, scale)
-        torch.cuda.synchronize()
-        assert attn.device_status() == (attn.ATTN_OK, 0)
-        _close(o, lse, o_ref, lse_ref)
+    side = torch.cuda.Stream()          # a non-blocking stream: the first call must not need the legacy one
+    with torch.cuda.stream(side):
+        for _ in range(2):              # two calls in a row share the array
+            o, lse = _noalloc(attn, q, k, v, causal, scale, side)
+            o_ref, lse_ref = _with_workspace(attn, q, k, v, causal, scale, side)
+            side.synchronize()
+            assert attn.device_status(side) == (attn.ATTN_OK, 0)
+            assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+            assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+
+
+def test_noalloc_split_shape_against_the_oracle(attn):
+    """The split last wave through the static array, against the fp64 definition."""
+    B, Hq, Hkv, N, D = 1, 4, 2, 1100, 64
+    assert attn.attn_fwd_workspace_bytes(B, Hq, N, D, False) > 0
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, seed=6100)
+    scale = 1.0 / math.sqrt(D)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        o, lse = _noalloc(attn, q.cuda(), k.cuda(), v.cuda(), False, scale, side)
+        side.synchronize()
+    o_ref, lse_ref = attention_forward(q, k, v, False, scale)
+    d = np.abs(o.float().cpu().numpy() - o_ref)
+    dl = np.abs(lse.cpu().numpy() - lse_ref)
+    assert d.max() <= 2e-2 and d.mean() <= 2e-3 and dl.max() <= 1e-3, (d.max(), d.mean(), dl.max())
 
 
 def test_noalloc_rejects_bad_arguments_before_touching_the_gpu(attn):

@@ -407,26 +407,35 @@ namespace {
 constexpr size_t kNoallocScratchBytes = sizeof(g_attn_noalloc_scratch);
 
 struct NoallocScratch {
-  std::once_flag once;
+  std::mutex mu;
   void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
 };
 NoallocScratch g_noalloc[kMaxDevices];
 
 // Device address of the scratch array on `dev` (the current device).  In host code the
-// array's name is only a stand-in for it, so the address is looked up once per device,
-// and the array is cleared then (nothing in it must start at zero afterwards: the
-// kernel tags its counters with a per-launch epoch).
+// array's name is only a stand-in for it, so the address is looked up once per device with
+// that device current.  A failed look-up is not remembered: the next call tries again.
+// The array is not cleared: device storage starts at zero when the module loads, and the
+// kernel tags its counter words with a per-launch epoch and zeroes them after use, so the
+// contents a previous call leaves behind are never taken for the current call's.
 void* noalloc_scratch(int dev) {
-  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (dev < 0 || dev >= kMaxDevices) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "attn_fwd_noalloc: device ordinal %d is beyond the library's limit of %d devices", dev,
+                  kMaxDevices);
+    return nullptr;
+  }
   NoallocScratch& ns = g_noalloc[dev];
-  std::call_once(ns.once, [&ns] {
+  std::lock_guard<std::mutex> lock(ns.mu);
+  if (ns.ptr == nullptr) {
     void* ptr = nullptr;
-    ns.err = cudaGetSymbolAddress(&ptr, g_attn_noalloc_scratch);
-    if (ns.err == cudaSuccess) ns.err = cudaMemset(ptr, 0, kNoallocScratchBytes);
-    if (ns.err == cudaSuccess) ns.ptr = ptr;
-  });
-  if (ns.ptr == nullptr) record_cuda_error("no-alloc scratch set-up", ns.err);
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_attn_noalloc_scratch);
+    if (e != cudaSuccess) {
+      record_cuda_error("no-alloc scratch address look-up", e);
+      return nullptr;
+    }
+    ns.ptr = ptr;
+  }
   return ns.ptr;
 }
 
