@@ -363,10 +363,14 @@ def run_ours(args, w):
                                    lse_host=lh, stream=stream, rope_tables=tables, fp8_descales=descales)
         h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-        e2e_path = ("forward_from_host: pinned host q,k,v -> device, "
-                    + ("attn_fwd_rope (device-resident cos/sin tables)" if tables else
-                       ("attn_fwd_fp8 (E4M3 inputs)" if fp8 else "attn_fwd_ws"))
-                    + ", o,lse -> pinned host; in 4 pieces (batch rows), copies overlapping the kernels")
+        if tables or fp8:
+            e2e_path = ("forward_from_host: pinned host q,k,v -> device, "
+                        + ("attn_fwd_rope (device-resident cos/sin tables)" if tables else "attn_fwd_fp8 (E4M3 inputs)")
+                        + ", o,lse -> pinned host; in 4 pieces (batch rows), torch copies overlapping the kernels")
+        else:
+            e2e_path = ("attn_fwd_from_host (C ABI, called by forward_from_host): pinned host q,k,v -> device "
+                        "buffers, attn_fwd_ws per piece, o,lse -> pinned host; 4 pieces (batch rows), the "
+                        "library's copy streams overlapping the kernels; returns after the last download")
     for _ in range(2):
         e2e_call()
     barrier(dist, device)

@@ -1,7 +1,8 @@
 /*
  * attn.h -- C ABI of the B200 (sm_100a) attention library: the forward pass in bf16
- * (attn_fwd, attn_fwd_ws, attn_fwd_noalloc) and E4M3 (attn_fwd_fp8), its gradients
- * (attn_bwd), and rotary position embedding of Q and K (attn_rope_qk, attn_fwd_rope).
+ * (attn_fwd, attn_fwd_ws, attn_fwd_noalloc; attn_fwd_from_host on host buffers) and E4M3
+ * (attn_fwd_fp8), its gradients (attn_bwd), and rotary position embedding of Q and K
+ * (attn_rope_tables, attn_rope_qk, attn_fwd_rope).
  *
  * The operation is the tiled attention forward pass named by "HipKittens:
  * fast and furious AMD kernels" (section "Performance results": an attention
@@ -147,6 +148,54 @@ int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float
 size_t attn_fwd_noalloc_scratch_bytes(void);
 
 /*
+ * attn_fwd_from_host -- the attention forward of attn_fwd_ws on HOST buffers, end to end:
+ * upload q, k, v, compute, download o and lse; returns once o_host and lse_host hold the
+ * results.  (The pages have no counterpart: this is the library's end-to-end entry point for
+ * data that lives in host memory.)
+ *
+ * Arguments:
+ *   q_host, k_host, v_host   bf16 [B, Hq, N, D] / [B, Hkv, N, D] in HOST memory, contiguous. read
+ *   o_host, lse_host         bf16 [B, Hq, N, D] and fp32 [B, Hq, N] in HOST memory.       written
+ *                            Page-locked (pinned) host memory is needed for the copies to
+ *                            overlap the kernels; pageable memory works, without overlap.
+ *   q_dev, k_dev, v_dev, o_dev, lse_dev   DEVICE buffers of the same sizes (16-byte aligned;
+ *                            lse_dev 4-byte), owned by the caller; the call copies into and out
+ *                            of them and leaves the inputs and results there.
+ *   workspace, workspace_bytes   optional split-tail workspace (256-byte aligned, or NULL with
+ *                            0 bytes); a piece whose split needs more makes no split.
+ *                            attn_fwd_from_host_workspace_bytes() gives the size every piece
+ *                            can use.
+ *   B, Hq, Hkv, N, D, causal, scale   as attn_fwd.
+ *   pieces                   >= 1: the problem is cut into up to `pieces` (at most 64)
+ *                            independent parts -- ranges of batch rows, or for B == 1 ranges
+ *                            of whole KV-head groups -- so that each part's upload and
+ *                            download overlap the neighbouring parts' kernels.
+ *   stream                   the kernels run on `stream`; the copies on two non-blocking
+ *                            streams the library creates once per device.  The uploads start
+ *                            after the work enqueued on `stream` before the call.
+ * The library allocates no device memory (streams and events only).  The call is synchronous:
+ * it returns after the last download (or, on an error, after everything it enqueued).
+ * Errors: as attn_fwd_ws; ATTN_ERR_INVALID_ARG also for a null host or device buffer or
+ * pieces < 1; ATTN_ERR_CUDA if a copy, event or stream call fails (text in
+ * attn_last_cuda_error()).  Results equal those of attn_fwd_ws on each piece.
+ * Calls from several host threads share the copy streams (their copies then take turns) and
+ * are otherwise independent, given distinct buffers and workspaces.
+ */
+int attn_fwd_from_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                       float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                       float* lse_dev, void* workspace, size_t workspace_bytes,
+                       int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+                       int pieces, void* stream);
+
+/*
+ * attn_fwd_from_host_workspace_bytes -- the largest split-tail workspace any piece of an
+ * attn_fwd_from_host call with these sizes uses on the current device (0 if none splits);
+ * -1 on invalid sizes or a CUDA error.
+ */
+long long attn_fwd_from_host_workspace_bytes(int B, int Hq, int Hkv, int N, int D, int causal,
+                                             int pieces);
+
+/*
  * attn_bwd -- enqueue the attention backward pass (gradients of the forward) on `stream`.
  *
  * The pages name an attention backward kernel beside the forward ("HipKittens: fast and
@@ -218,6 +267,21 @@ long long attn_bwd_workspace_bytes(int B, int Hq, int N);
  */
 int attn_rope_qk(const void* q, const void* k, const float* cos_t, const float* sin_t,
                  void* q_out, void* k_out, int B, int Hq, int Hkv, int N, int D, void* stream);
+
+/*
+ * attn_rope_tables -- fill the usual RoPE angle tables on the device:
+ *     cos_t[p][d] = cos(theta),  sin_t[p][d] = sin(theta),  theta = p * base^(-2d/D)
+ * for positions p < N and d < D/2 (the frequencies of the rotary embedding the pages' rotary
+ * kernel applies, "HipKittens: fast and furious AMD kernels", section "Performance results";
+ * the pages print no schedule, so this is the common one with a caller-chosen base).
+ *   cos_t, sin_t  DEVICE fp32 [N, D/2], contiguous, 16-byte aligned, caller-owned.  written
+ *   N >= 0, D >= 2 even, base finite and > 0 (10000 is the usual value).
+ *   stream        cudaStream_t (void*); asynchronous.
+ * Numerics: theta, its cosine and sine in fp64, each rounded to fp32 (nearest).
+ * Errors: ATTN_ERR_INVALID_ARG (sizes, base, null pointers with N > 0), ATTN_ERR_MISALIGNED,
+ * ATTN_ERR_UNSUPPORTED for N * D/2 > 2^40, ATTN_ERR_CUDA on a launch failure.
+ */
+int attn_rope_tables(float* cos_t, float* sin_t, int N, int D, double base, void* stream);
 
 /*
  * attn_fwd_rope -- attention forward of RoPE(Q), RoPE(K) and V in one call: attn_rope_qk into

@@ -263,3 +263,40 @@ def test_work_unit_count_limit():
     B, Hq = 1 << 20, 1 << 10                      # B*Hq = 2^30
     assert call(B=B, Hq=Hq, Hkv=Hq, N=2048) == UNSUPPORTED   # 2^30 heads x 8 units
     assert call(B=B, Hq=Hq, Hkv=Hq, N=512) == UNSUPPORTED    # exactly 2^31 units
+
+
+def call_host(**kw):
+    a = dict(qh=P, kh=P, vh=P, oh=P, lh=P, qd=P, kd=P, vd=P, od=P, ld=P, ws=None, wsb=0, B=2, Hq=4, Hkv=2, N=128,
+             D=128, causal=0, scale=0.125, pieces=4)
+    a.update(kw)
+    return attn.attn_fwd_from_host(a["qh"], a["kh"], a["vh"], a["oh"], a["lh"], a["qd"], a["kd"], a["vd"], a["od"],
+                                   a["ld"], a["ws"], a["wsb"], a["B"], a["Hq"], a["Hkv"], a["N"], a["D"], a["causal"],
+                                   a["scale"], a["pieces"], None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(qh=None), INVALID), (dict(oh=None), INVALID), (dict(lh=None), INVALID), (dict(qd=None), INVALID),
+    (dict(ld=None), INVALID), (dict(pieces=0), INVALID), (dict(pieces=-3), INVALID), (dict(Hq=3), INVALID),
+    (dict(scale=math.nan), INVALID), (dict(ws=None, wsb=256), INVALID), (dict(D=80), UNSUPPORTED),
+    (dict(qd=P + 8), MISALIGNED), (dict(od=P + 2), MISALIGNED), (dict(ld=P + 2), MISALIGNED),
+    (dict(ws=P + 128, wsb=4096), MISALIGNED), (dict(B=0), OK), (dict(N=0, qh=None, qd=None), OK),
+])
+def test_host_buffer_entry_point_rejects_before_any_cuda_call(kw, expected):
+    assert call_host(**kw) == expected
+
+
+def test_host_buffer_workspace_query_rejects_bad_sizes():
+    assert attn.attn_fwd_from_host_workspace_bytes(1, 3, 2, 128, 128, 0, 4) == -1
+    assert attn.attn_fwd_from_host_workspace_bytes(1, 2, 2, 128, 80, 0, 4) == -1
+    assert attn.attn_fwd_from_host_workspace_bytes(1, 2, 2, 128, 128, 0, 0) == -1
+    assert attn.attn_fwd_from_host_workspace_bytes(0, 2, 2, 128, 128, 0, 4) == 0
+
+
+@pytest.mark.parametrize("args,expected", [
+    ((P, P, -1, 64, 10000.0), INVALID), ((P, P, 16, 7, 10000.0), INVALID), ((P, P, 16, 0, 10000.0), INVALID),
+    ((P, P, 16, 64, 0.0), INVALID), ((P, P, 16, 64, -2.0), INVALID), ((P, P, 16, 64, math.nan), INVALID),
+    ((P, P, 16, 64, math.inf), INVALID), ((None, P, 16, 64, 10000.0), INVALID), ((P + 4, P, 16, 64, 10000.0), MISALIGNED),
+    ((P, P + 8, 16, 64, 10000.0), MISALIGNED), ((None, None, 0, 64, 10000.0), OK),
+])
+def test_rope_tables_entry_point_rejects_before_any_cuda_call(args, expected):
+    assert attn.attn_rope_tables(*args, None) == expected

@@ -5,14 +5,11 @@
   contiguous block of every tensor; the pieces must cover the problem exactly once; and for
   B == 1 a piece must hold whole GQA groups (its query heads are exactly those of its KV heads),
   so that each piece is an attention problem of its own.
-- rope_tables() builds the cos / sin tables the rotary kernel reads; they must hold the angles
-  of the oracle's rotation.
 """
 import numpy as np
 import pytest
 
 import tiled_attention_forward_03_b200 as attn
-from oracle import rope_angles
 
 
 def _covered(sl, n):
@@ -58,14 +55,3 @@ def test_single_batch_row_is_cut_by_kv_head_groups():
     assert [(_covered(kv, 8), _covered(q, 32)) for _, q, kv in pieces] == [
         ([0, 1], list(range(0, 8))), ([2, 3], list(range(8, 16))),
         ([4, 5], list(range(16, 24))), ([6, 7], list(range(24, 32)))]
-
-
-@pytest.mark.parametrize("N,D,base", [(1, 2, 10000.0), (7, 8, 100.0), (300, 64, 10000.0), (4096, 128, 500000.0)])
-def test_rope_tables_hold_the_oracle_angles(N, D, base):
-    cos_t, sin_t = attn.rope_tables(N, D, base)
-    assert tuple(cos_t.shape) == (N, D // 2) and tuple(sin_t.shape) == (N, D // 2)
-    assert str(cos_t.dtype) == "torch.float32" and cos_t.is_contiguous() and sin_t.is_contiguous()
-    th = rope_angles(N, D, base)
-    # fp32 rounding of values in [-1, 1], plus the fp64 cos / sin of angles up to ~4096 rad
-    assert np.abs(cos_t.numpy().astype(np.float64) - np.cos(th)).max() <= 1e-7
-    assert np.abs(sin_t.numpy().astype(np.float64) - np.sin(th)).max() <= 1e-7

@@ -349,3 +349,61 @@ def test_split_workspace_too_small_is_rejected(attn):
     assert attn.attn_fwd_ws(*args, ws.data_ptr(), need, s) == attn.ATTN_OK
     torch.cuda.synchronize()
     assert torch.isfinite(o.float()).all()
+
+
+def test_default_calls_on_two_streams_at_once(attn):
+    """forward() with its defaults (split last wave, cached workspace) on two streams whose
+    kernels overlap: each stream gets its own workspace, so both results match the oracle.
+    cfg2-sized non-causal problems (their last wave is split), different inputs per stream."""
+    w = CFG2
+    assert attn.attn_fwd_workspace_bytes(w.B, w.Hq, w.N, w.D, False) > 0
+    inputs = [make_qkv(w.B, w.Hq, w.Hkv, w.N, w.D, seed=w.seed + 40 + i) for i in range(2)]
+    dev_in = [tuple(x.cuda() for x in qkv) for qkv in inputs]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    outs = []
+    for _ in range(3):      # several rounds, so the two streams' launches interleave
+        outs = []
+        for (qd, kd, vd), s in zip(dev_in, streams):
+            with torch.cuda.stream(s):
+                outs.append(attn.forward(qd, kd, vd, causal=False, scale=w.softmax_scale, stream=s))
+    torch.cuda.synchronize()
+    assert attn.device_status() == (attn.ATTN_OK, 0)
+    for (q, k, v), (o, lse) in zip(inputs, outs):
+        o_ref, l_ref = attention_forward(q, k, v, False, w.softmax_scale)
+        assert_close(o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
+                     o_ref, l_ref, "two streams")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,causal,pieces", [
+    (3, 4, 2, 700, 128, False, 4), (1, 8, 2, 640, 64, True, 4), (2, 2, 2, 1, 128, False, 1),
+    (1, 16, 4, 1100, 128, False, 3), (4, 16, 16, 2048, 128, False, 4), (2, 4, 1, 513, 96, True, 64),
+])
+def test_host_buffer_entry_point(attn, B, Hq, Hkv, N, D, causal, pieces):
+    """attn_fwd_from_host through the C ABI: pinned host inputs, caller-owned device buffers,
+    results in pinned host outputs; against the oracle, and the device buffers hold the same
+    results."""
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, seed=4200 + N + pieces)
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.full((B, Hq, N, D), float("nan"), dtype=torch.bfloat16).pin_memory()
+    lh = torch.full((B, Hq, N), float("nan"), dtype=torch.float32).pin_memory()
+    qd, kd, vd = (torch.empty(x.shape, dtype=x.dtype, device="cuda") for x in (q, k, v))
+    od = torch.empty((B, Hq, N, D), dtype=torch.bfloat16, device="cuda")
+    ld = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    need = attn.attn_fwd_from_host_workspace_bytes(B, Hq, Hkv, N, D, causal, pieces)
+    assert need >= 0
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+    scale = D ** -0.5
+    s = torch.cuda.Stream()
+    st = attn.attn_fwd_from_host(qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), oh.data_ptr(), lh.data_ptr(),
+                                 qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), ld.data_ptr(),
+                                 ws.data_ptr() if need > 0 else None, need, B, Hq, Hkv, N, D, causal, scale, pieces,
+                                 s.cuda_stream)
+    assert st == attn.ATTN_OK, attn.attn_status_string(st) + " " + attn.attn_last_cuda_error()
+    # the call is synchronous: the host outputs are complete on return
+    o_ref, l_ref = attention_forward(q, k, v, causal, scale)
+    assert_close(oh.float().numpy().astype(np.float64), lh.numpy().astype(np.float64), o_ref, l_ref,
+                 f"attn_fwd_from_host {pieces} pieces")
+    torch.cuda.synchronize()
+    assert torch.equal(od.cpu(), oh) and torch.equal(ld.cpu(), lh)
+    assert attn.device_status() == (attn.ATTN_OK, 0)

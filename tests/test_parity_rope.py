@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import attention_forward, attention_forward_rope, attention_rows, rope_rotate
+from oracle import attention_forward, attention_forward_rope, attention_rows, rope_angles, rope_rotate
 from attn_inputs import CFG2, make_qkv
 
 pytestmark = pytest.mark.gpu
@@ -42,6 +42,20 @@ def test_rope_rotation(attn, B, Hq, Hkv, N, D, base):
         ref = rope_rotate(x, base)
         g = got.float().cpu().numpy().astype(np.float64)
         assert np.all(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6), float(np.max(np.abs(g - ref)))
+
+
+@pytest.mark.parametrize("N,D,base", [(1, 2, 10000.0), (7, 8, 100.0), (300, 64, 10000.0), (4096, 128, 500000.0),
+                                      (16384, 128, 10000.0)])
+def test_rope_tables_hold_the_oracle_angles(attn, N, D, base):
+    """attn_rope_tables fills cos / sin of the oracle's angles p * base^(-2d/D): fp32 rounding
+    of values in [-1, 1] (<= 2^-25) plus the fp64 evaluation of angles up to ~16384 rad."""
+    cos_t, sin_t = attn.rope_tables(N, D, base)
+    torch.cuda.synchronize()
+    assert tuple(cos_t.shape) == (N, D // 2) and tuple(sin_t.shape) == (N, D // 2)
+    assert cos_t.dtype == torch.float32 and cos_t.is_cuda and cos_t.is_contiguous() and sin_t.is_contiguous()
+    th = rope_angles(N, D, base)
+    assert np.abs(cos_t.cpu().numpy().astype(np.float64) - np.cos(th)).max() <= 1e-7
+    assert np.abs(sin_t.cpu().numpy().astype(np.float64) - np.sin(th)).max() <= 1e-7
 
 
 def test_rope_in_place(attn):

@@ -21,7 +21,8 @@ from . import build as _build
 __all__ = [
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED",
     "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "AttnError", "lib", "lib_path", "attn_fwd", "attn_fwd_ws",
-    "attn_fwd_workspace_bytes", "attn_fwd_noalloc", "attn_fwd_noalloc_scratch_bytes",
+    "attn_fwd_workspace_bytes", "attn_fwd_noalloc", "attn_fwd_noalloc_scratch_bytes", "attn_fwd_from_host",
+    "attn_fwd_from_host_workspace_bytes", "attn_rope_tables",
     "attn_status_string", "attn_last_cuda_error", "attn_device_status", "attn_num_units",
     "attn_version", "attn_selftest_exp2_poly", "attn_selftest_wait_timeout", "forward",
     "forward_from_host", "device_status", "attn_bwd", "attn_bwd_workspace_bytes", "backward",
@@ -80,6 +81,13 @@ def _load() -> ctypes.CDLL:
     L.attn_fwd_workspace_bytes.restype = ctypes.c_longlong
     L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.attn_fwd_noalloc.restype = i
+    L.attn_fwd_from_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i, i, i, i, i, i,
+                                     f, i, vp]
+    L.attn_fwd_from_host.restype = i
+    L.attn_fwd_from_host_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+    L.attn_fwd_from_host_workspace_bytes.restype = ctypes.c_longlong
+    L.attn_rope_tables.argtypes = [vp, vp, i, i, ctypes.c_double, vp]
+    L.attn_rope_tables.restype = i
     L.attn_fwd_noalloc_scratch_bytes.argtypes = []
     L.attn_fwd_noalloc_scratch_bytes.restype = ctypes.c_size_t
     L.attn_status_string.argtypes = [i]
@@ -122,6 +130,24 @@ def attn_fwd_noalloc(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, scale, stream) -
     """Direct call of the entry point that allocates nothing (its workspace is a static
     device array in the library); for callers that may not allocate device memory."""
     return lib.attn_fwd_noalloc(q, k, v, o, lse, B, Hq, Hkv, N, D, int(bool(causal)), float(scale), stream)
+
+
+def attn_fwd_from_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, workspace,
+                       workspace_bytes, B, Hq, Hkv, N, D, causal, scale, pieces, stream) -> int:
+    """Direct call of the host-buffer entry point (host and device pointers, sizes and stream as
+    integers); returns once the host outputs hold the results."""
+    return lib.attn_fwd_from_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev,
+                                  workspace, workspace_bytes, B, Hq, Hkv, N, D, int(bool(causal)), float(scale),
+                                  pieces, stream)
+
+
+def attn_fwd_from_host_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int, causal: bool, pieces: int) -> int:
+    return lib.attn_fwd_from_host_workspace_bytes(B, Hq, Hkv, N, D, int(bool(causal)), pieces)
+
+
+def attn_rope_tables(cos_t, sin_t, N, D, base, stream) -> int:
+    """Direct call of the RoPE table entry point (device pointers and stream as integers)."""
+    return lib.attn_rope_tables(cos_t, sin_t, N, D, float(base), stream)
 
 
 def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, causal, scale, workspace, workspace_bytes,
@@ -220,21 +246,22 @@ def _check(t, name, dtype, shape):
 _workspaces: dict = {}
 
 
-def _workspace(device, nbytes: int, purpose: str = "fwd", stream=None):
-    """A cached device buffer of at least nbytes, per device and purpose ("fwd": the
-    split-tail schedule, "bwd": the backward pass's per-row delta and LSE, "rope": the
-    rotated q and k).  The buffer is marked as used on ``stream``, so that when a larger one
-    replaces it, torch's allocator does not hand its memory to another stream's allocation
-    before the kernels enqueued on ``stream`` have finished with it."""
+def _workspace(device, nbytes: int, purpose: str, stream):
+    """A cached device buffer of at least nbytes, per device, purpose ("fwd": the split-tail
+    schedule, "bwd": the backward pass's per-row delta and LSE, "rope": the rotated q and k)
+    and stream.  Calls on one stream run in order, so they may share a buffer; calls on
+    different streams get different buffers and may overlap on the GPU.  The buffer is marked
+    as used on ``stream``, so that when a larger one replaces it, torch's allocator does not
+    hand its memory to another stream's allocation before the kernels enqueued on ``stream``
+    have finished with it."""
     import torch
 
-    key = (device.type, device.index, purpose)
+    key = (device.type, device.index, purpose, stream.cuda_stream)
     buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
         buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
         _workspaces[key] = buf
-    if stream is not None:
-        buf.record_stream(stream)
+    buf.record_stream(stream)
     return buf
 
 
@@ -244,9 +271,8 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
 
     Runs on ``stream`` (a torch.cuda.Stream) or torch's current stream.  With ``split``
     (default) a non-causal problem whose last wave would leave the GPU half idle splits
-    that wave's KV ranges across SMs (attn_fwd_ws, workspace cached per device);
-    ``split=False`` calls attn_fwd.  Calls that share the cached workspace are ordered
-    on one stream; pass distinct streams only with split=False.
+    that wave's KV ranges across SMs (attn_fwd_ws, with a workspace cached per device and
+    stream, so calls on different streams may run at once); ``split=False`` calls attn_fwd.
     """
     import torch
 
@@ -271,7 +297,7 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
         if ws_bytes < 0:
             raise AttnError(ATTN_ERR_CUDA, "attn_fwd_workspace_bytes")
         if ws_bytes > 0:
-            ws = _workspace(q.device, ws_bytes, stream=s)
+            ws = _workspace(q.device, ws_bytes, "fwd", s)
             st = attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                              B, Hq, Hkv, N, D, causal, scale, ws.data_ptr(), ws.numel(), s.cuda_stream)
         else:
@@ -348,18 +374,23 @@ def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None,
 
     Returns host tensors (o, lse).  The problem is cut into up to ``pieces`` independent parts
     (batch rows, or KV-head groups when B == 1); each part's upload, kernel and download are
-    enqueued so that the copies of neighbouring parts overlap the kernels (copies on two side
-    streams, kernels on ``stream``).  The call returns after the last download.  With
-    ``rope_tables`` = (cos_t, sin_t) (device tables from rope_tables()), the attention is that
-    of RoPE(q), RoPE(k) and v (forward_rope).  With ``fp8_descales`` = (q_descale, k_descale,
-    v_descale), q, k, v are float8_e4m3fn and the call is forward_fp8.
+    enqueued so that the copies of neighbouring parts overlap the kernels.  The bf16 forward
+    is the library's own host-buffer call, attn_fwd_from_host (device buffers and the split
+    workspace come from torch, on ``stream``).  With ``rope_tables`` = (cos_t, sin_t) (device
+    tables from rope_tables()), the attention is that of RoPE(q), RoPE(k) and v (forward_rope),
+    and with ``fp8_descales`` = (q_descale, k_descale, v_descale), q, k, v are float8_e4m3fn and
+    the call is forward_fp8: those two are pipelined here, with torch copies on two side streams.
     """
     import torch
 
     dev = torch.device(device if device is not None else "cuda")
+    if dev.index is None:
+        dev = torch.device(dev.type, torch.cuda.current_device())
     s = stream if stream is not None else torch.cuda.current_stream(dev)
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
     with torch.cuda.stream(s):
         qd, kd, vd = (torch.empty(x.shape, dtype=x.dtype, device=dev) for x in (q, k, v))
         od = torch.empty((B, Hq, N, D), dtype=torch.bfloat16, device=dev)
@@ -368,6 +399,27 @@ def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None,
         out_host = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
     if lse_host is None:
         lse_host = torch.empty(ld.shape, dtype=ld.dtype, pin_memory=True)
+    if rope_tables is None and fp8_descales is None:
+        for name, t, shape in (("q", q, (B, Hq, N, D)), ("k", k, (B, Hkv, N, D)), ("v", v, (B, Hkv, N, D)),
+                               ("out_host", out_host, (B, Hq, N, D))):
+            if t.is_cuda or t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous bf16 host tensor of shape {shape}")
+        if lse_host.is_cuda or lse_host.dtype != torch.float32 or tuple(lse_host.shape) != (B, Hq, N) \
+                or not lse_host.is_contiguous():
+            raise ValueError(f"lse_host must be a contiguous fp32 host tensor of shape {(B, Hq, N)}")
+        with torch.cuda.device(dev):
+            ws_bytes = attn_fwd_from_host_workspace_bytes(B, Hq, Hkv, N, D, causal, pieces)
+            if ws_bytes < 0:
+                raise AttnError(ATTN_ERR_INVALID_ARG, "attn_fwd_from_host_workspace_bytes")
+            ws = _workspace(dev, ws_bytes, "fwd", s) if ws_bytes > 0 else None
+            st = attn_fwd_from_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out_host.data_ptr(),
+                                    lse_host.data_ptr(), qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                                    ld.data_ptr(), ws.data_ptr() if ws is not None else None,
+                                    ws.numel() if ws is not None else 0, B, Hq, Hkv, N, D, causal, scale, pieces,
+                                    s.cuda_stream)
+        if st != ATTN_OK:
+            raise AttnError(st, "attn_fwd_from_host")
+        return out_host, lse_host
     qi = lambda pc: (pc[0], pc[1])
     ki = lambda pc: (pc[0], pc[2])
 
@@ -375,10 +427,8 @@ def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None,
         a, b, c, o, lse = qd[qi(pc)], kd[ki(pc)], vd[ki(pc)], od[qi(pc)], ld[qi(pc)]
         if rope_tables is not None:
             forward_rope(a, b, c, rope_tables[0], rope_tables[1], causal=causal, scale=scale, out=o, lse=lse, stream=s)
-        elif fp8_descales is not None:
-            forward_fp8(a, b, c, *fp8_descales, causal=causal, scale=scale, out=o, lse=lse, stream=s)
         else:
-            forward(a, b, c, causal=causal, scale=scale, out=o, lse=lse, stream=s)
+            forward_fp8(a, b, c, *fp8_descales, causal=causal, scale=scale, out=o, lse=lse, stream=s)
 
     _pipelined(dev, s, _pieces(B, Hq, Hkv, pieces), [(q, qd, qi), (k, kd, ki), (v, vd, ki)],
                [(out_host, od, qi), (lse_host, ld, qi)], compute)
@@ -391,7 +441,7 @@ def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
 
     ``o`` and ``lse`` are the forward's outputs for the same q, k, v, causal and scale;
     ``dout`` is the bf16 gradient of the loss with respect to o.  The workspace (per-row
-    delta and LSE) is cached per device; calls sharing it are ordered on one stream.
+    delta and LSE) is cached per device and stream.
     """
     import torch
 
@@ -418,7 +468,7 @@ def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
         ws_bytes = attn_bwd_workspace_bytes(B, Hq, N)
         if ws_bytes < 0:
             raise AttnError(ATTN_ERR_INVALID_ARG, "attn_bwd_workspace_bytes")
-        ws = _workspace(q.device, max(ws_bytes, 256), "bwd", stream=s)
+        ws = _workspace(q.device, max(ws_bytes, 256), "bwd", s)
         st = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, N, D, causal, scale,
                       ws.data_ptr(), ws.numel(), s.cuda_stream)
@@ -486,7 +536,7 @@ def forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float, c
         ws_bytes = attn_fwd_workspace_bytes(B, Hq, N, D, causal) if split else 0
         if ws_bytes < 0:
             raise AttnError(ATTN_ERR_CUDA, "attn_fwd_workspace_bytes")
-        ws = _workspace(q.device, ws_bytes, stream=s) if ws_bytes > 0 else None
+        ws = _workspace(q.device, ws_bytes, "fwd", s) if ws_bytes > 0 else None
         st = attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N,
                           D, causal, scale, q_descale, k_descale, v_descale, ws.data_ptr() if ws is not None else None,
                           ws.numel() if ws is not None else 0, s.cuda_stream)
@@ -495,17 +545,21 @@ def forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float, c
     return out, lse
 
 
-def rope_tables(N: int, D: int, base: float = 10000.0, device=None):
-    """cos and sin tables [N, D/2] (fp32, computed in fp64) of the angles p * base^(-2d/D)."""
+def rope_tables(N: int, D: int, base: float = 10000.0, device=None, stream=None):
+    """cos and sin tables [N, D/2] (fp32) of the angles p * base^(-2d/D), filled on the device by
+    attn_rope_tables (fp64 arithmetic rounded to fp32).  ``device`` defaults to the current CUDA
+    device; the tables are written on ``stream`` (or torch's current stream)."""
     import torch
 
-    p = torch.arange(N, dtype=torch.float64)[:, None]
-    d = torch.arange(D // 2, dtype=torch.float64)[None, :]
-    theta = p * torch.pow(torch.tensor(float(base), dtype=torch.float64), -2.0 * d / D)
-    cos_t, sin_t = torch.cos(theta).to(torch.float32), torch.sin(theta).to(torch.float32)
-    if device is not None:
-        cos_t, sin_t = cos_t.to(device), sin_t.to(device)
-    return cos_t.contiguous(), sin_t.contiguous()
+    dev = torch.device(device if device is not None else "cuda")
+    with torch.cuda.device(dev):
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        cos_t = torch.empty((N, D // 2), dtype=torch.float32, device=dev)
+        sin_t = torch.empty((N, D // 2), dtype=torch.float32, device=dev)
+        st = attn_rope_tables(cos_t.data_ptr(), sin_t.data_ptr(), N, D, base, s.cuda_stream)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_rope_tables")
+    return cos_t, sin_t
 
 
 def rope(q, k, cos_t, sin_t, q_out=None, k_out=None, stream=None):
@@ -535,8 +589,7 @@ def rope(q, k, cos_t, sin_t, q_out=None, k_out=None, stream=None):
 def forward_rope(q, k, v, cos_t, sin_t, causal: bool = False, scale: float | None = None, out=None, lse=None,
                  stream=None):
     """Attention forward of RoPE(q), RoPE(k), v in one call (attn_fwd_rope); returns (o, lse).
-    The workspace (rotated q and k, split tail) is cached per device; calls sharing it are
-    ordered on one stream."""
+    The workspace (rotated q and k, split tail) is cached per device and stream."""
     import torch
 
     B, Hq, N, D = q.shape
@@ -557,7 +610,7 @@ def forward_rope(q, k, v, cos_t, sin_t, causal: bool = False, scale: float | Non
         nbytes = attn_fwd_rope_workspace_bytes(B, Hq, Hkv, N, D)
         if nbytes < 0:
             raise AttnError(ATTN_ERR_CUDA, "attn_fwd_rope_workspace_bytes")
-        ws = _workspace(q.device, max(nbytes, 256), "rope", stream=s)
+        ws = _workspace(q.device, max(nbytes, 256), "rope", s)
         st = attn_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), cos_t.data_ptr(), sin_t.data_ptr(),
                            out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, D, causal, scale, ws.data_ptr(),
                            ws.numel(), s.cuda_stream)

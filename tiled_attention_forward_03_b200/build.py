@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libattn_fwd.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = ["attn_api.cu"]
-HEADERS = ["attn_fwd_kernel.cuh", "attn_fwd_wide_kernel.cuh", "attn_bwd_kernel.cuh", "attn_rope_kernel.cuh", "sm100_ptx.cuh"]
+HEADERS = ["attn_fwd_kernel.cuh", "attn_fwd_colsplit_kernel.cuh", "attn_fwd_wide_kernel.cuh", "attn_bwd_kernel.cuh", "attn_rope_kernel.cuh", "sm100_ptx.cuh"]
 EXPECTED_REGS = 168
 
 NVCC_FLAGS = [
@@ -76,18 +76,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + log)
     # register count of each forward-kernel instance (bf16 D = 32/64/96/128, E4M3 D = 64/128;
     # the self-test kernels are exempt)
+    # and the column-split kernel D = 32/64/96/128; both use the same warpgroup register split)
     regs, spills, current = [], [], None
+    split_kernel = lambda name: "attn_fwd_sm100" in name or "attn_fwd_colsplit_sm100" in name
     for line in log.splitlines():
         m = re.search(r"Compiling entry function '(\w+)'", line)
         if m:
             current = m.group(1)
         m = re.search(r"Used (\d+) registers", line)
-        if m and current and "attn_fwd_sm100" in current:
+        if m and current and split_kernel(current):
             regs.append(int(m.group(1)))
         m = re.search(r"(\d+) bytes spill stores", line)
-        if m and current and "attn_fwd_sm100" in current:
+        if m and current and split_kernel(current):
             spills.append(int(m.group(1)))
-    if len(regs) != 6 or any(r != EXPECTED_REGS for r in regs):
+    if len(regs) != 10 or any(r != EXPECTED_REGS for r in regs):
         os.remove(tmp)
         raise RuntimeError(f"unexpected kernel register counts {regs} (want {EXPECTED_REGS}):\n{log}")
     if verbose:
@@ -101,7 +103,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
 # The files that define each measured path's kernels and their launch: a traffic record taken
 # with ncu stays valid while these files are unchanged.
 DIGEST_FILES = {
-    "fwd": ["attn_fwd_kernel.cuh", "sm100_ptx.cuh", "attn_api.cu"],
+    "fwd": ["attn_fwd_colsplit_kernel.cuh", "attn_fwd_kernel.cuh", "sm100_ptx.cuh", "attn_api.cu"],
     "wide": ["attn_fwd_wide_kernel.cuh", "attn_fwd_kernel.cuh", "sm100_ptx.cuh", "attn_api.cu"],
     "bwd": ["attn_bwd_kernel.cuh", "attn_fwd_kernel.cuh", "sm100_ptx.cuh", "attn_api.cu"],
     "all": SOURCES + HEADERS,

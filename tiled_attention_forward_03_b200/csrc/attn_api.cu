@@ -19,6 +19,7 @@
 #include "attn_bwd_kernel.cuh"
 #include "attn_rope_kernel.cuh"
 #include "attn_fwd_wide_kernel.cuh"
+#include "attn_fwd_colsplit_kernel.cuh"
 
 #define ATTN_VERSION_STRING "b200-attn 0.1 (sm_100a, tcgen05/TMA/TMEM)"
 
@@ -80,6 +81,10 @@ bool device_setup(int dev, int* num_sms) {
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64>), attn::SmemPlan<64>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<96>), attn::SmemPlan<96>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<128>), attn::SmemPlan<128>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<32>), attn::CsPlan<32>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<64>), attn::CsPlan<64>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<96>), attn::CsPlan<96>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<128>), attn::CsPlan<128>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, true>), attn::SmemPlan<64, true>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<128, true>), attn::SmemPlan<128, true>::kAlloc);
     // the wide-head kernel has no register split: dynamic shared memory opt-in only
@@ -129,6 +134,29 @@ int encode_map(CUtensorMap* map, const void* base, long long heads, int N, int D
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     record_driver_error("cuTensorMapEncodeTiled", (int)r);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+// The output O [heads, N, D] (bf16) as a TMA store target: boxes of 32 columns (64 bytes) x 128 rows x
+// 1 head with 64-byte swizzle, matching the column-split kernel's staging buffers; rows past N are not
+// written.
+int encode_map_o(CUtensorMap* map, void* base, long long heads, int N, int D) {
+  auto enc = tensor_map_encoder();
+  if (!enc) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled entry point unavailable");
+    return ATTN_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * (cuuint64_t)D * 2};
+  cuuint32_t box[3] = {32, (cuuint32_t)attn::kBlockM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    record_driver_error("cuTensorMapEncodeTiled (output)", (int)r);
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
@@ -348,6 +376,55 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   const Schedule plan0 = plan_schedule(p.num_units, p.num_steps, p.num_blocks, num_sms, p.causal, D, true);
   const bool split = workspace != nullptr && plan0.parts > 1;
   if (split && workspace_bytes < plan0.ws_bytes()) return ATTN_ERR_INVALID_ARG;
+  if (!e4m3 && !split) {
+    // bf16 without a split last wave: the column-split kernel (one Q tile per unit)
+    CUtensorMap mo;
+    if ((st = encode_map_o(&mo, o, (long long)B * Hq, N, D)) != ATTN_OK) return st;
+    attn::CsParams cp;
+    cp.lse = lse;
+    cp.Hq = Hq;
+    cp.Hkv = Hkv;
+    cp.N = N;
+    cp.group = Hq / Hkv;
+    cp.num_tiles = p.num_blocks;
+    const long long units = (long long)B * Hq * p.num_blocks;
+    if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    cp.num_units = (int)units;
+    cp.causal = p.causal;
+    cp.num_steps = p.causal ? (int)((long long)B * Hq * ((p.num_blocks + 1) / 2)) : cp.num_units;
+    cp.div_tiles = attn::make_fast_div((uint32_t)p.num_blocks);
+    cp.div_steps = attn::make_fast_div((uint32_t)((p.num_blocks + 1) / 2));
+    cp.div_hq = p.div_hq;
+    cp.div_group = p.div_group;
+    cp.c = p.c;
+    cp.idesc_s = p.idesc_s;
+    cp.idesc_pv = p.idesc_pv;
+    const long long cgrid = cp.num_steps < num_sms ? cp.num_steps : num_sms;
+    switch (D) {
+      case 32:
+        attn::attn_fwd_colsplit_sm100<32><<<(unsigned)cgrid, attn::kCsThreads, attn::CsPlan<32>::kAlloc, s>>>(
+            mq, mk, mv, mo, cp);
+        break;
+      case 64:
+        attn::attn_fwd_colsplit_sm100<64><<<(unsigned)cgrid, attn::kCsThreads, attn::CsPlan<64>::kAlloc, s>>>(
+            mq, mk, mv, mo, cp);
+        break;
+      case 96:
+        attn::attn_fwd_colsplit_sm100<96><<<(unsigned)cgrid, attn::kCsThreads, attn::CsPlan<96>::kAlloc, s>>>(
+            mq, mk, mv, mo, cp);
+        break;
+      default:
+        attn::attn_fwd_colsplit_sm100<128><<<(unsigned)cgrid, attn::kCsThreads, attn::CsPlan<128>::kAlloc, s>>>(
+            mq, mk, mv, mo, cp);
+        break;
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      record_cuda_error("kernel launch", e);
+      return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+  }
   const Schedule sc = split ? plan0 : plan_schedule(p.num_units, p.num_steps, p.num_blocks, num_sms, p.causal, D, false);
   p.whole_per_cta = sc.whole_per_cta;
   p.tail_units = sc.tail_units;
@@ -760,6 +837,224 @@ int attn_fwd_rope(const void* q, const void* k, const void* v, const float* cos_
   if ((st = launch_rope(q, k, cos_t, sin_t, ws, ws + q_part, B, Hq, Hkv, N, D, s)) != ATTN_OK) return st;
   return launch_forward(ws, ws + q_part, v, o, lse, B, Hq, Hkv, N, D, causal, scale, split_ws,
                         split_ws ? rest : 0, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// RoPE angle tables, and the forward pass on host buffers.
+
+namespace {
+
+// Independent pieces of a [B, H, ...] problem for the host-buffer call: ranges of batch rows,
+// or, for a single batch row with several KV heads, ranges of whole KV-head groups (a KV head
+// and the query heads that read it).  Each piece is a contiguous block of every tensor.
+struct Piece {
+  long long q_off, kv_off, lse_off;  // element offsets of the piece's first q / k,v / lse entry
+  int B, Hq, Hkv;                    // the piece's own problem sizes
+};
+
+int make_pieces(int B, int Hq, int Hkv, int N, int D, int want, Piece* out) {
+  const int g = Hq / Hkv;
+  int n = 0;
+  if (B >= 2 || Hkv == 1) {
+    const int k = want < B ? want : B;
+    for (int i = 0; i < k; ++i) {
+      const long long b0 = (long long)B * i / k, b1 = (long long)B * (i + 1) / k;
+      if (b1 <= b0) continue;
+      out[n++] = Piece{b0 * Hq * N * D, b0 * Hkv * N * D, b0 * Hq * N, (int)(b1 - b0), Hq, Hkv};
+    }
+  } else {
+    const int k = want < Hkv ? want : Hkv;
+    for (int i = 0; i < k; ++i) {
+      const long long h0 = (long long)Hkv * i / k, h1 = (long long)Hkv * (i + 1) / k;
+      if (h1 <= h0) continue;
+      out[n++] = Piece{h0 * g * N * D, h0 * N * D, h0 * g * N, 1, (int)((h1 - h0) * g), (int)(h1 - h0)};
+    }
+  }
+  return n;
+}
+
+constexpr int kMaxPieces = 64;
+
+struct CopyStreams {
+  std::mutex mu;
+  cudaStream_t in = nullptr, out = nullptr;
+};
+CopyStreams g_copy_streams[kMaxDevices];
+
+// The two copy streams of the host-buffer call on `dev` (the current device), created once
+// (non-blocking, so they never wait for the legacy default stream).  A failure is retried by
+// the next call.
+bool copy_streams(int dev, cudaStream_t* in, cudaStream_t* out) {
+  if (dev < 0 || dev >= kMaxDevices) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "device ordinal %d beyond the library's limit", dev);
+    return false;
+  }
+  CopyStreams& cs = g_copy_streams[dev];
+  std::lock_guard<std::mutex> lock(cs.mu);
+  if (cs.in == nullptr) {
+    cudaStream_t a = nullptr, b = nullptr;
+    cudaError_t e = cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking);
+    if (e != cudaSuccess) {
+      if (a) cudaStreamDestroy(a);
+      record_cuda_error("copy stream creation", e);
+      return false;
+    }
+    cs.in = a;
+    cs.out = b;
+  }
+  *in = cs.in;
+  *out = cs.out;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_rope_tables(float* cos_t, float* sin_t, int N, int D, double base, void* stream) {
+  if (N < 0 || D < 2 || (D % 2) != 0 || !std::isfinite(base) || !(base > 0.0)) return ATTN_ERR_INVALID_ARG;
+  if ((long long)N * (D / 2) > (1LL << 40)) return ATTN_ERR_UNSUPPORTED;
+  if (N == 0) return ATTN_OK;
+  if (!cos_t || !sin_t) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(cos_t, 16) || !aligned(sin_t, 16)) return ATTN_ERR_MISALIGNED;
+  const long long items = (long long)N * (D / 2);
+  attn::attn_rope_tables_kernel<<<(unsigned)((items + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      cos_t, sin_t, N, D, base);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    record_cuda_error("rope tables kernel launch", e);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+long long attn_fwd_from_host_workspace_bytes(int B, int Hq, int Hkv, int N, int D, int causal, int pieces) {
+  if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || pieces < 1 || !supported_head_dim(D)) return -1;
+  if (B == 0 || N == 0) return 0;
+  Piece pc[kMaxPieces];
+  const int n = make_pieces(B, Hq, Hkv, N, D, pieces < kMaxPieces ? pieces : kMaxPieces, pc);
+  long long need = 0;
+  for (int i = 0; i < n; ++i) {
+    const long long b = attn_fwd_workspace_bytes(pc[i].B, pc[i].Hq, N, D, causal);
+    if (b < 0) return -1;
+    if (b > need) need = b;
+  }
+  return need;
+}
+
+int attn_fwd_from_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, float* lse_host,
+                       void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_dev, void* workspace,
+                       size_t workspace_bytes, int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+                       int pieces, void* stream) {
+  // ---- host-side validation (no CUDA call before this block passes)
+  if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale) || pieces < 1)
+    return ATTN_ERR_INVALID_ARG;
+  if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > 0x7fffffffLL || attn_num_units(B, Hq, N) > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return ATTN_OK;
+  if (!q_host || !k_host || !v_host || !o_host || !lse_host || !q_dev || !k_dev || !v_dev || !o_dev || !lse_dev)
+    return ATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr && workspace_bytes != 0) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q_dev, 16) || !aligned(k_dev, 16) || !aligned(v_dev, 16) || !aligned(o_dev, 16) ||
+      !aligned(lse_dev, 4) || (workspace != nullptr && !aligned(workspace, 256)))
+    return ATTN_ERR_MISALIGNED;
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    record_cuda_error("cudaGetDevice", e);
+    return ATTN_ERR_CUDA;
+  }
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  if (!copy_streams(dev, &s_in, &s_out)) return ATTN_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  Piece pc[kMaxPieces];
+  const int n = make_pieces(B, Hq, Hkv, N, D, pieces < kMaxPieces ? pieces : kMaxPieces, pc);
+  // events: start, then per piece "inputs landed" and "outputs ready", then done
+  cudaEvent_t ev[2 * kMaxPieces + 2];
+  int made = 0;
+  for (; made < 2 * n + 2; ++made) {
+    e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming);
+    if (e != cudaSuccess) break;
+  }
+  auto release = [&]() {
+    for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+  };
+  if (e != cudaSuccess) {
+    release();
+    record_cuda_error("cudaEventCreate", e);
+    return ATTN_ERR_CUDA;
+  }
+  cudaEvent_t ev_start = ev[0], ev_done = ev[1];
+  const size_t eb = 2;  // bf16
+  const char* qh = static_cast<const char*>(q_host);
+  const char* kh = static_cast<const char*>(k_host);
+  const char* vh = static_cast<const char*>(v_host);
+  char* oh = static_cast<char*>(o_host);
+  char* lh = reinterpret_cast<char*>(lse_host);
+  char* qd = static_cast<char*>(q_dev);
+  char* kd = static_cast<char*>(k_dev);
+  char* vd = static_cast<char*>(v_dev);
+  char* od = static_cast<char*>(o_dev);
+  char* ld = reinterpret_cast<char*>(lse_dev);
+
+  int st = ATTN_OK;
+  const char* what = nullptr;
+  // The uploads wait for the caller's earlier work on `stream`, which may still use the
+  // device buffers.
+  if ((e = cudaEventRecord(ev_start, s)) != cudaSuccess) what = "cudaEventRecord";
+  if (!what && (e = cudaStreamWaitEvent(s_in, ev_start, 0)) != cudaSuccess) what = "cudaStreamWaitEvent";
+  for (int i = 0; i < n && !what && st == ATTN_OK; ++i) {
+    const Piece& p = pc[i];
+    const size_t q_bytes = (size_t)p.B * p.Hq * N * D * eb, kv_bytes = (size_t)p.B * p.Hkv * N * D * eb;
+    const size_t l_bytes = (size_t)p.B * p.Hq * N * sizeof(float);
+    const size_t qo = (size_t)p.q_off * eb, ko = (size_t)p.kv_off * eb, lo = (size_t)p.lse_off * sizeof(float);
+    cudaEvent_t ev_in = ev[2 + 2 * i], ev_c = ev[3 + 2 * i];
+    if ((e = cudaMemcpyAsync(qd + qo, qh + qo, q_bytes, cudaMemcpyHostToDevice, s_in)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(kd + ko, kh + ko, kv_bytes, cudaMemcpyHostToDevice, s_in)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(vd + ko, vh + ko, kv_bytes, cudaMemcpyHostToDevice, s_in)) != cudaSuccess) {
+      what = "host-to-device copy";
+      break;
+    }
+    if ((e = cudaEventRecord(ev_in, s_in)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ev_in, 0)) != cudaSuccess) {
+      what = "event record/wait";
+      break;
+    }
+    const long long need = attn_fwd_workspace_bytes(p.B, p.Hq, N, D, causal);
+    void* ws = (workspace != nullptr && need > 0 && (size_t)need <= workspace_bytes) ? workspace : nullptr;
+    st = launch_forward(qd + qo, kd + ko, vd + ko, od + qo, reinterpret_cast<float*>(ld + lo), p.B, p.Hq, p.Hkv, N,
+                        D, causal, scale, ws, ws ? workspace_bytes : 0, stream);
+    if (st != ATTN_OK) break;
+    if ((e = cudaEventRecord(ev_c, s)) != cudaSuccess || (e = cudaStreamWaitEvent(s_out, ev_c, 0)) != cudaSuccess) {
+      what = "event record/wait";
+      break;
+    }
+    if ((e = cudaMemcpyAsync(oh + qo, od + qo, q_bytes, cudaMemcpyDeviceToHost, s_out)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(lh + lo, ld + lo, l_bytes, cudaMemcpyDeviceToHost, s_out)) != cudaSuccess) {
+      what = "device-to-host copy";
+      break;
+    }
+  }
+  if (!what && st == ATTN_OK) {
+    if ((e = cudaEventRecord(ev_done, s_out)) != cudaSuccess || (e = cudaEventSynchronize(ev_done)) != cudaSuccess)
+      what = "waiting for the downloads";
+  } else {
+    // leave nothing of this call in flight: its copies and kernels read and write the
+    // caller's buffers
+    cudaStreamSynchronize(s_in);
+    cudaStreamSynchronize(s);
+    cudaStreamSynchronize(s_out);
+  }
+  release();
+  if (what) {
+    record_cuda_error(what, e);
+    return ATTN_ERR_CUDA;
+  }
+  return st;
 }
 
 }  // extern "C"

@@ -87,3 +87,23 @@ __global__ void __launch_bounds__(256) attn_rope_qk(const __nv_bfloat16* q, cons
 }
 
 }  // namespace attn
+
+namespace attn {
+
+// The usual angle schedule for the tables above: theta_pd = p * base^(-2d/D) for p < N and
+// d < D/2, evaluated in fp64 and stored as fp32 cos / sin.  One thread per (p, d).
+__global__ void __launch_bounds__(256) attn_rope_tables_kernel(float* __restrict__ cos_t, float* __restrict__ sin_t,
+                                                               int N, int D, double base) {
+  const int half = D / 2;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)N * half) return;
+  const int p = (int)(i / half);
+  const int d = (int)(i - (long long)p * half);
+  const double theta = (double)p * pow(base, -2.0 * (double)d / (double)D);
+  double s, c;
+  sincos(theta, &s, &c);
+  cos_t[i] = (float)c;
+  sin_t[i] = (float)s;
+}
+
+}  // namespace attn
