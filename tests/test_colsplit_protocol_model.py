@@ -1,9 +1,10 @@
 """A model of the column-split forward kernel's schedule and synchronisation, run on the CPU.
 
 The kernel (one 128-row Q tile per work unit, two score buffers, the score columns of each block
-split between two softmax warpgroups) coordinates five agents through mbarriers: the TMA producer,
-the MMA issuer, the tensor pipe (which runs MMAs and their commits in issue order), and the two
-softmax warpgroups.  Here each agent's program is restated step for step as a Python generator,
+split between two softmax warpgroups) coordinates six agents through mbarriers: the TMA producer,
+the MMA issuer, the tensor pipe (which runs MMAs and their commits in issue order), the two
+softmax warpgroups, and the store warp (which writes each unit's O, staged in the unit's Q
+buffer, with TMA stores and then gives the buffer back to the producer).  Here each agent's program is restated step for step as a Python generator,
 the mbarrier waits are evaluated with the hardware's parity rule (a wait on parity P passes when
 the barrier's current phase has the other parity), and a scheduler runs the agents in many
 different interleavings.  Each run checks that
@@ -13,7 +14,9 @@ different interleavings.  Each run checks that
   * every read finds the data it expects: the score buffer holds S of the right block, the P
     halves of the right block are present when P V is issued, a ring stage holds the K or V tile
     the MMA expects, the Q buffer holds the unit's Q, O is overwritten only after the previous
-    unit's epilogue has read it, and the O rescale waits for the last P V of the block before;
+    unit's epilogue has read it, the O rescale waits for the last P V of the block before, O is
+    staged in a Q buffer only after every S of that unit has read it, and the producer reloads a
+    Q buffer only after the stores of the O staged in it have read it;
   * the units of all CTAs cover every (head, query tile) exactly once, each with its KV blocks.
 """
 import random
@@ -90,6 +93,7 @@ def run_cta(P, units, S_stages, rng, rescale_every_block=True):
     for i in range(2):
         for name in (f"q_full{i}", f"q_empty{i}", f"s_full{i}", f"p_full{i}0", f"p_full{i}1"):
             bars[name] = Barrier(name, 1)
+        bars[f"o_staged{i}"] = Barrier(f"o_staged{i}", 2)
     for i in range(S_stages):
         bars[f"kv_full{i}"] = Barrier(f"kv_full{i}", 1)
         bars[f"kv_empty{i}"] = Barrier(f"kv_empty{i}", 1)
@@ -101,6 +105,8 @@ def run_cta(P, units, S_stages, rng, rescale_every_block=True):
         "stage_busy": [0] * S_stages,        # issued MMAs that read the stage and have not completed
         "q_buf": [None, None],
         "q_busy": [0, 0],
+        "q_staged": [None, None],            # unit whose O is staged in each Q buffer (until stored)
+        "q_store_reading": [False, False],
         "s_buf": [None, None],               # which block's S each score buffer holds
         "p_buf": [[None, None], [None, None]],
         "o_unit": None,                      # (unit, "acc" | "done") accumulated in O
@@ -141,6 +147,8 @@ def run_cta(P, units, S_stages, rng, rescale_every_block=True):
                 q_par ^= 1 << qb
                 q_uses[qb] += 1
                 assert state["q_busy"][qb] == 0, "Q buffer reloaded while an S MMA still reads it"
+                assert state["q_staged"][qb] is None and not state["q_store_reading"][qb], \
+                    "Q buffer reloaded while its staged O is still being stored"
                 tma_q.append(("q", qb, u))
             yield from load_kv("K", u, w, j)
 
@@ -187,8 +195,6 @@ def run_cta(P, units, S_stages, rng, rescale_every_block=True):
             tensor_q.append(("S", gs, gs & 1, st, qb))
             tensor_q.append(("commit", f"s_full{gs & 1}"))
             tensor_q.append(("commit", f"kv_empty{st}"))
-            if j == w[2] - 1:
-                tensor_q.append(("commit", f"q_empty{qb}"))
 
         gs = 0
         for _ in range(2):
@@ -243,6 +249,29 @@ def run_cta(P, units, S_stages, rng, rescale_every_block=True):
             assert state["o_unit"] == (u, "done"), "epilogue before the unit's last P V completed"
             state["o_read_by"].add(h)
             bars["o_free"].arrive()
+            qb = u & 1
+            assert state["q_busy"][qb] == 0 and state["q_buf"][qb] == u, "O staged over a Q still read by S"
+            assert state["q_staged"][qb] in (None, u) and not state["q_store_reading"][qb]
+            state["q_staged"][qb] = u
+            bars[f"o_staged{qb}"].arrive()
+            u += 1
+
+    # ------------------------------------------------------------ store warp
+    def store():
+        st_par = 0
+        u = 0
+        for w in units:
+            if w is None:
+                continue
+            qb = u & 1
+            yield from W(f"o_staged{qb}", (st_par >> qb) & 1, u >> 1)
+            st_par ^= 1 << qb
+            assert state["q_staged"][qb] == u
+            state["q_store_reading"][qb] = True
+            yield ("store_read",)          # the TMA engine reads the staged rows (any time later)
+            state["q_store_reading"][qb] = False
+            state["q_staged"][qb] = None
+            bars[f"q_empty{qb}"].arrive()
             u += 1
 
     # ------------------------------------------------------------ tensor pipe and TMA engine
@@ -280,7 +309,7 @@ def run_cta(P, units, S_stages, rng, rescale_every_block=True):
             state["smem_stage"][op[1]] = op[2]
             bars[f"kv_full{op[1]}"].arrive()
 
-    agents = {"producer": producer(), "mma": mma(), "sm0": softmax(0), "sm1": softmax(1)}
+    agents = {"producer": producer(), "mma": mma(), "sm0": softmax(0), "sm1": softmax(1), "store": store()}
     pending = {a: None for a in agents}   # the event an agent is blocked on (None: runnable)
     done = set()
     for _ in range(10 ** 6):
@@ -297,6 +326,8 @@ def run_cta(P, units, S_stages, rng, rescale_every_block=True):
                 return True
             if ev[0] == "wait":
                 return bars[ev[1]].phase > ev[2]
+            if ev[0] == "store_read":
+                return True
             other = "sm1" if a == "sm0" else "sm0"
             return pending[other] == ev
 

@@ -117,3 +117,45 @@ def test_forward_rope_cfg2_sampled(attn):
         o_ref, l_ref = attention_rows(qr, kr, v[b:b + 1, h:h + 1], rows, w.causal, w.softmax_scale)
         idx = [r[2] for r in rows]
         assert_fwd_close(o[b, h, idx], lse[b, h, idx], o_ref, l_ref, f"cfg2 rope head {(b, h)}")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,causal", [
+    (1, 1, 1, 2048, 128, False),    # the split last wave: both KV ranges rotate their own copy of Q
+    (1, 4, 4, 1500, 96, False),
+    (2, 4, 2, 700, 64, True),
+    (1, 8, 2, 1025, 32, True),
+])
+def test_fused_rope_matches_rotate_then_forward(attn, B, Hq, Hkv, N, D, causal):
+    """For D <= 128 the forward kernel rotates each Q tile in shared memory (K goes through the
+    rotary kernel): the result must agree with rotating both tensors first and running the plain
+    forward, and with the oracle."""
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, 4300 + N + D)
+    scale = D ** -0.5
+    if not causal and B * Hq * N == 2048:
+        assert attn.attn_fwd_workspace_bytes(B, Hq, N, D, False) > 0
+    o, lse = check_forward_rope(attn, q, k, v, causal, scale)
+    cos_t, sin_t = attn.rope_tables(N, D)
+    qr, kr = attn.rope(q.cuda(), k.cuda(), cos_t, sin_t)
+    o2, l2 = attn.forward(qr, kr, v.cuda(), causal=causal, scale=scale, split=False)
+    torch.cuda.synchronize()
+    o2 = o2.float().cpu().numpy().astype(np.float64)
+    l2 = l2.cpu().numpy().astype(np.float64)
+    # the same rotated operands, two schedules: fp32 summation order only
+    assert np.abs(o - o2).max() <= 2e-2 and np.abs(lse - l2).max() <= 1e-4
+    o_ref, lse_ref = attention_forward(rot_bf16(q), rot_bf16(k), v, causal, scale)
+    assert_fwd_close(o, lse, o_ref, lse_ref, f"fused rope B{B} Hq{Hq} Hkv{Hkv} N{N} D{D} c{causal}")
+
+
+def test_fused_rope_long_sequence_sampled(attn):
+    """N = 8192 (angles up to ~8200 rad), causal GQA: sampled rows of two heads."""
+    B, Hq, Hkv, N, D = 1, 4, 2, 8192, 128
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, 4400)
+    o, lse = check_forward_rope(attn, q, k, v, True, D ** -0.5)
+    rng = np.random.default_rng(19)
+    for h in (0, Hq - 1):
+        qr = rot_bf16(q[:, h:h + 1])
+        kr = rot_bf16(k[:, h // 2:h // 2 + 1])
+        rows = [(0, 0, int(i)) for i in sorted(set(rng.integers(0, N, 48)) | {0, 1, 4095, N - 1})]
+        o_ref, l_ref = attention_rows(qr, kr, v[:, h // 2:h // 2 + 1], rows, True, D ** -0.5)
+        idx = [r[2] for r in rows]
+        assert_fwd_close(o[0, h, idx], lse[0, h, idx], o_ref, l_ref, f"long rope head {h}")

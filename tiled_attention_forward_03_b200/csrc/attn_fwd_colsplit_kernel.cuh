@@ -21,7 +21,8 @@
 //   warps 4-7   softmax warpgroup 1 (score columns 64-127)
 //   warp  8     TMA producer: Q per unit (two buffers), K and V through a ring, in MMA order
 //   warp  9     MMA issuer
-//   warps 10-11 idle (they complete the third warpgroup, which gives up registers)
+//   warp  10    output store: TMA tensor stores of each unit's staged O
+//   warp  11    idle (completes the third warpgroup, which gives up registers)
 //
 // Tensor memory (512 columns):  S_0 [0,128)  S_1 [128,256)  O_0 [256,256+D)  O_1 [384,384+D).
 // P_h(j) (bf16 pairs) overwrites the first 32 columns of warpgroup h's own 64 score columns.
@@ -31,8 +32,9 @@
 // where P(g)V(g) is two MMAs of K = 64 (O_0 += P_0 V[0:64], O_1 += P_1 V[64:128]) and S(g+2)
 // reuses S(g)'s buffer after both have been issued (tcgen05 MMAs of a CTA run in issue order).
 // S of a unit's first blocks is computed while the previous unit finishes: Q has two buffers.
-// The epilogue of a unit stages O through shared memory (64-byte swizzle, 32 columns at a time)
-// and writes it with TMA tensor stores.
+// The epilogue of a unit stages O in that unit's Q buffer, free once its last S has completed
+// (64-byte swizzle, 32-column chunks); the store warp writes it out with TMA tensor stores and
+// hands the buffer back to the producer once the stores have read it.
 //
 // A work unit is one 128-row query tile of one head.  Persistent grid, static stride: causal
 // steps pair a head's heaviest and lightest tiles (tile T-1-s and tile s: T+1 blocks per step);
@@ -55,6 +57,7 @@ enum : unsigned {
   kSiteCsMma = 32,
   kSiteCsSoftmax = 33,
   kSiteCsEpilogue = 34,
+  kSiteCsStore = 35,
 };
 
 template <int D>
@@ -66,13 +69,14 @@ struct CsPlan {
   static constexpr int kStages = kChunks == 2 ? 4 : 8;    // K/V ring depth (tiles)
   static constexpr int kOChunks = D / 32;                 // 32-column output chunks (64-byte rows)
   static constexpr int kStageBytes = kBlockM * 64;        // one staged output chunk: 8 KB
-  static constexpr int kQOff = 0;                         // two Q buffers
+  static_assert(kOChunks * kStageBytes <= kTileBytes, "staged O must fit in a Q buffer");
+  static constexpr int kQOff = 0;                         // two Q buffers (O staging after their last use)
   static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kOOff = kKVOff + kStages * kTileBytes;  // output staging, one buffer per warpgroup
-  static constexpr int kXOff = kOOff + 2 * kStageBytes;   // (m, l) exchange [unit parity][warpgroup][row]
+  static constexpr int kXOff = kKVOff + kStages * kTileBytes;  // (m, l) exchange [unit parity][warpgroup][row]
   static constexpr int kBarOff = kXOff + 2 * 2 * kBlockM * 8;
-  // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2 buffers][2 halves] pv_done o_full o_free drain
-  static constexpr int kNumBars = 4 + 2 * kStages + 2 + 4 + 4;
+  // q_full[2] q_empty[2] o_staged[2] kv_full[S] kv_empty[S] s_full[2] p_full[2 buffers][2 halves]
+  // pv_done o_full o_free drain
+  static constexpr int kNumBars = 6 + 2 * kStages + 2 + 4 + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;             // slack for 1024-byte alignment
@@ -175,12 +179,12 @@ __global__ void __launch_bounds__(kCsThreads, 1)
 
   uint8_t* sQ = smem + Plan::kQOff;
   uint8_t* sKV = smem + Plan::kKVOff;
-  uint8_t* sO = smem + Plan::kOOff;
   float2* xml = reinterpret_cast<float2*>(smem + Plan::kXOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kBarOff);
   uint64_t* q_full = bars;                 // [2]
-  uint64_t* q_empty = bars + 2;            // [2]
-  uint64_t* kv_full = bars + 4;            // [S]
+  uint64_t* q_empty = bars + 2;            // [2]: released by the store warp
+  uint64_t* o_staged = bars + 4;           // [2]: the unit's O is staged in Q buffer [qb]
+  uint64_t* kv_full = bars + 6;            // [S]
   uint64_t* kv_empty = kv_full + S;        // [S]
   uint64_t* s_full = kv_empty + S;         // [2]
   uint64_t* p_full = s_full + 2;           // [2 buffers][2 halves]
@@ -198,6 +202,7 @@ __global__ void __launch_bounds__(kCsThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+      mbar_init(&o_staged[i], 2 * kBlockM);
       mbar_init(&s_full[i], 1);
     }
     for (int i = 0; i < 4; ++i) mbar_init(&p_full[i], kBlockM);
@@ -341,7 +346,6 @@ __global__ void __launch_bounds__(kCsThreads, 1)
         __syncwarp();
         commit(&s_full[gs & 1u]);
         commit(&kv_empty[st]);
-        if (c.j == c.w.n - 1) commit(&q_empty[qb]);
         ++gs;
         return true;
       };
@@ -404,8 +408,6 @@ __global__ void __launch_bounds__(kCsThreads, 1)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t t_o0 = tmem_base + lane_off + 256;  // O_0; O_1 at +128
     const uint32_t t_oh = t_o0 + 128 * h;
-    uint8_t* stage = sO + h * Plan::kStageBytes;
-    const uint32_t stage_row = smem_u32(stage) + r * 64;
     const float c = p.c;
     uint32_t g = 0, o_par = 0;
     bool ok = true;
@@ -537,6 +539,9 @@ __global__ void __launch_bounds__(kCsThreads, 1)
         tc_fence_before();
         mbar_arrive(o_free);
       }
+      // O is staged in this unit's Q buffer: its last S has completed (o_full follows every MMA
+      // of the unit), and the producer reloads it only after the store warp has released it.
+      const uint32_t stage_row = smem_u32(sQ + (u & 1) * Plan::kTileBytes) + r * 64;
 #pragma unroll
       for (int ch = h; ch < Plan::kOChunks; ch += 2) {
         uint32_t x0[32], x1[32];
@@ -555,26 +560,50 @@ __global__ void __launch_bounds__(kCsThreads, 1)
         for (int i = 0; i < 16; ++i)
           packed[i] = pack_bf16x2(fmaf(__uint_as_float(x1[2 * i]), w1, __uint_as_float(x0[2 * i]) * w0),
                                   fmaf(__uint_as_float(x1[2 * i + 1]), w1, __uint_as_float(x0[2 * i + 1]) * w0));
-        // the staging buffer is free once this warpgroup's previous TMA store has read it
-        if (r == 0) bulk_wait_group_read0();
-        named_bar_sync(5 + h, kBlockM);
-        // row r: 64 bytes, four 16-byte pieces, 64-byte swizzle (piece q of row r at q ^ ((r >> 1) & 3))
+        // chunk ch: 128 rows of 64 bytes, four 16-byte pieces per row, 64-byte swizzle (piece q of
+        // row r at position q ^ ((r >> 1) & 3))
+        const uint32_t row_addr = stage_row + ch * Plan::kStageBytes;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          st_shared_v4(stage_row + ((q ^ ((r >> 1) & 3)) << 4), packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+          st_shared_v4(row_addr + ((q ^ ((r >> 1) & 3)) << 4), packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
                        packed[4 * q + 3]);
-        fence_proxy_async_smem();
-        named_bar_sync(5 + h, kBlockM);
-        if (r == 0) {
-          tma_store_3d(&tmap_o, stage, ch * 32, w.row0, w.head_q);
-          bulk_commit_group();
-        }
       }
+      // make the staged rows visible to the TMA (async proxy), then hand them to the store warp
+      fence_proxy_async_smem();
+      mbar_arrive(&o_staged[u & 1]);
       if (h == 0 && row < p.N) p.lse[(size_t)w.head_q * p.N + row] = (mt + log2f(lt)) * 0.69314718055994530942f;
       ++u;
     }
-    // every TMA store of this warpgroup has completed before the CTA exits
-    if (r == 0) bulk_wait_group0();
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ output store warp
+    // Per unit: wait until both softmax warpgroups have staged O in the unit's Q buffer, store
+    // it with TMA tensor stores (rows past N are not written), wait until the stores have read
+    // the buffer and give it back to the producer.
+    regs_decrease<kRegsControl>();
+    if (lane == 0) {
+      uint32_t st_par = 0u;  // bit qb: parity of the next wait on o_staged[qb]
+      int u = 0;
+      for (int it = 0;; ++it) {
+        CsUnit w;
+        const int got = cs_item(p, it, w);
+        if (got == 0) break;
+        if (got == 2) continue;
+        const int qb = u & 1;
+        if (!wait_phase(&o_staged[qb], (st_par >> qb) & 1u, abort_flag, kSiteCsStore)) break;
+        st_par ^= 1u << qb;
+        const uint8_t* stage = sQ + qb * Plan::kTileBytes;
+#pragma unroll
+        for (int ch = 0; ch < Plan::kOChunks; ++ch)
+          tma_store_3d(&tmap_o, stage + ch * Plan::kStageBytes, ch * 32, w.row0, w.head_q);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        mbar_arrive(&q_empty[qb]);
+        ++u;
+      }
+      // every TMA store has completed before the CTA exits
+      bulk_wait_group0();
+    }
+    __syncwarp();
   } else {
     regs_decrease<kRegsControl>();
   }
