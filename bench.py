@@ -385,7 +385,7 @@ def run_ours(args, w):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
     barrier(dist, device)
 
-    rope_ms = unfused_ms = None
+    rope_ms = None
     if args.pass_ == "rope":
         # the rotary kernel alone (attn_rope_qk), L2 flushed between launches
         qo, ko = torch.empty_like(qd), torch.empty_like(kd)
@@ -400,20 +400,6 @@ def run_ours(args, w):
             re_[i].record(stream)
         torch.cuda.synchronize(device)
         rope_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(rs, re_))
-        # the unfused composition for comparison: rotate Q and K, then the plain forward
-        us_ = [torch.cuda.Event(enable_timing=True) for _ in range(20)]
-        ue_ = [torch.cuda.Event(enable_timing=True) for _ in range(20)]
-        for i in range(23):
-            flush.zero_()
-            if i >= 3:
-                us_[i - 3].record(stream)
-            attn.rope(qd, kd, cos_t, sin_t, q_out=qo, k_out=ko, stream=stream)
-            attn.forward(qo, ko, vd, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
-            if i >= 3:
-                ue_[i - 3].record(stream)
-        torch.cuda.synchronize(device)
-        unfused_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(us_, ue_))
-
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -435,9 +421,7 @@ def run_ours(args, w):
         kv_side = w.B * w.Hkv * w.N * w.D * 2
         algo_bytes = 4 * q_side + 4 * kv_side + 4 * w.B * w.Hq * w.N
     elif args.pass_ == "rope":
-        kernel = (f"attn_fwd_rope call: attn_rope_qk on K + attn_fwd_sm100<{w.D}> rotating each Q tile in shared "
-                  f"memory, timed together" if w.D <= 128 else
-                  f"attn_fwd_rope call: attn_rope_qk on Q and K + attn_fwd_wide_sm100<{w.D}>, timed together")
+        kernel = f"attn_fwd_rope call: attn_rope_qk on Q and K + the forward kernel, timed together"
         algo_bytes = w.algorithmic_bytes
     elif fp8:
         kernel = f"attn_fwd_sm100<{w.D}, E4M3>"
@@ -446,7 +430,10 @@ def run_ours(args, w):
         peak_burst = peak_burst * FP8_OVER_BF16
         peak_kind = f"{peak_kind} bf16 matmul x {FP8_OVER_BF16:g} (nominal E4M3/bf16 ratio)"
     else:
-        kernel = f"attn_fwd_sm100<{w.D}>"
+        # the kernel the library picks for this shape (bf16, no split last wave)
+        colsplit = w.causal and w.D == 128 and w.N <= 2048
+        kernel = f"attn_fwd_colsplit_sm100<{w.D}>" if colsplit else (
+            f"attn_fwd_sm100<{w.D}>" if w.D <= 128 else f"attn_fwd_wide_sm100<{w.D}>")
         algo_bytes = w.algorithmic_bytes
 
     line = {
@@ -488,10 +475,6 @@ def run_ours(args, w):
                                "frac": round(gbs / hbm, 4), "us_per_launch": round(rope_ms * 1e3, 2),
                                "algorithmic_bytes": rope_bytes, "kernel": "attn_rope_qk",
                                "peak_kind": "measured HBM copy bandwidth"}
-        line["rope_unfused"] = {"value": round(flops_step / (unfused_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                                "ms_per_step": round(unfused_ms, 5),
-                                "what": "attn_rope_qk on Q and K, then the plain forward on the rotated tensors "
-                                        "(the composition the fused call replaces), L2 flushed between steps"}
     if world == 1 and not args.no_cpu_baseline:
         tf, _, el, done, sample = time_oracle(w, CPU_SAMPLE_SECONDS, backward=backward, rope=args.pass_ == "rope")
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",

@@ -284,20 +284,15 @@ int attn_rope_qk(const void* q, const void* k, const float* cos_t, const float* 
 int attn_rope_tables(float* cos_t, float* sin_t, int N, int D, double base, void* stream);
 
 /*
- * attn_fwd_rope -- attention forward of RoPE(Q), RoPE(K) and V in one call (both parts enqueued
- * on `stream`).  For D <= 128 the rotation of Q is fused into the forward kernel: each 128-row Q
- * tile is rotated in shared memory after its TMA load, with the arithmetic of attn_rope_qk (fp32
- * from the bf16 values and fp32 tables, rounded to bf16), and only K goes through the rotary
- * kernel, into the workspace.  For D = 192 and 256 both go through the rotary kernel first.
- * Arguments as attn_fwd plus the tables of attn_rope_qk and
+ * attn_fwd_rope -- attention forward of RoPE(Q), RoPE(K) and V in one call: attn_rope_qk into
+ * the caller's workspace, then the forward kernel on the rotated tensors (both enqueued on
+ * `stream`).  Arguments as attn_fwd plus the tables of attn_rope_qk and
  *   workspace        device pointer, 256-byte aligned, at least
- *                    attn_fwd_rope_workspace_bytes() bytes (fewer, but at least room for the two
- *                    rotated tensors, also works: the forward then makes no split); after the call
- *                    it holds RoPE(K) at offset round_up(B*Hq*N*D*2, 256), and for D > 128 also
- *                    RoPE(Q) at offset 0.
+ *                    attn_fwd_rope_workspace_bytes() bytes (fewer, but at least the two rotated
+ *                    tensors, also works: the forward then makes no split); after the call it
+ *                    holds RoPE(Q) at offset 0 and RoPE(K) at offset round_up(B*Hq*N*D*2, 256).
  * Errors as attn_fwd and attn_rope_qk (ATTN_ERR_INVALID_ARG for a null or too small
- * workspace).  The result is that of attn_fwd on the outputs of attn_rope_qk, up to the fp32
- * summation order of the kernel the forward runs on.
+ * workspace).  The result equals attn_fwd_ws on the outputs of attn_rope_qk.
  */
 int attn_fwd_rope(const void* q, const void* k, const void* v, const float* cos_t, const float* sin_t,
                   void* o, float* lse, int B, int Hq, int Hkv, int N, int D, int causal, float scale,

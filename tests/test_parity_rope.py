@@ -120,15 +120,15 @@ def test_forward_rope_cfg2_sampled(attn):
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,N,D,causal", [
-    (1, 1, 1, 2048, 128, False),    # the split last wave: both KV ranges rotate their own copy of Q
+    (1, 1, 1, 2048, 128, False),    # the split last wave
     (1, 4, 4, 1500, 96, False),
     (2, 4, 2, 700, 64, True),
     (1, 8, 2, 1025, 32, True),
 ])
-def test_fused_rope_matches_rotate_then_forward(attn, B, Hq, Hkv, N, D, causal):
-    """For D <= 128 the forward kernel rotates each Q tile in shared memory (K goes through the
-    rotary kernel): the result must agree with rotating both tensors first and running the plain
-    forward, and with the oracle."""
+def test_forward_rope_matches_rotate_then_forward(attn, B, Hq, Hkv, N, D, causal):
+    """attn_fwd_rope (the rotary kernel into the workspace, then the forward, the split last wave
+    included) against rotating both tensors with attn_rope_qk and running the plain forward
+    without a split, and against the oracle."""
     q, k, v = make_qkv(B, Hq, Hkv, N, D, 4300 + N + D)
     scale = D ** -0.5
     if not causal and B * Hq * N == 2048:
@@ -146,7 +146,7 @@ def test_fused_rope_matches_rotate_then_forward(attn, B, Hq, Hkv, N, D, causal):
     assert_fwd_close(o, lse, o_ref, lse_ref, f"fused rope B{B} Hq{Hq} Hkv{Hkv} N{N} D{D} c{causal}")
 
 
-def test_fused_rope_long_sequence_sampled(attn):
+def test_forward_rope_long_sequence_sampled(attn):
     """N = 8192 (angles up to ~8200 rad), causal GQA: sampled rows of two heads."""
     B, Hq, Hkv, N, D = 1, 4, 2, 8192, 128
     q, k, v = make_qkv(B, Hq, Hkv, N, D, 4400)

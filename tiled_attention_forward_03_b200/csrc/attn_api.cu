@@ -212,11 +212,17 @@ unsigned next_epoch() {
 
 // e4m3: q, k, v hold E4M3 bytes whose values are multiplied by qk_descale (in the scores) and
 // o_scale (in the output); otherwise bf16 and both factors 1.
-// rope_cos / rope_sin: RoPE tables [N][D/2] when the two-tile kernel rotates Q itself (bf16, D <= 128).
 int launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                    int N, int D, int causal, float scale, void* workspace, size_t workspace_bytes,
-                   void* stream, bool e4m3 = false, float qk_descale = 1.f, float o_scale = 1.f,
-                   const float* rope_cos = nullptr, const float* rope_sin = nullptr);
+                   void* stream, bool e4m3 = false, float qk_descale = 1.f, float o_scale = 1.f);
+
+// bf16 forward without a split last wave: which kernel runs.  Measured on B200 by interleaved
+// A/B runs of the two kernels on the same inputs: the column-split kernel (one Q tile per unit,
+// two score buffers) is 5-8 % faster for causal D = 128 at N <= 2048, where the two-tile
+// kernel's unit boundaries and lone diagonal blocks weigh most; everywhere else the two-tile
+// kernel is as fast or faster (N >= 4096: 6-13 %; D = 64: 2-9 %), because each K/V tile it loads
+// feeds 256 query rows instead of 128.
+bool use_column_split(int N, int D, int causal) { return causal && D == 128 && N <= 2048; }
 
 }  // namespace
 
@@ -285,8 +291,7 @@ namespace {
 
 int launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                    int N, int D, int causal, float scale, void* workspace, size_t workspace_bytes,
-                   void* stream, bool e4m3, float qk_descale, float o_scale, const float* rope_cos,
-                   const float* rope_sin) {
+                   void* stream, bool e4m3, float qk_descale, float o_scale) {
 
   // ---- host-side validation (no CUDA call before this block passes)
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
@@ -379,8 +384,8 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   const Schedule plan0 = plan_schedule(p.num_units, p.num_steps, p.num_blocks, num_sms, p.causal, D, true);
   const bool split = workspace != nullptr && plan0.parts > 1;
   if (split && workspace_bytes < plan0.ws_bytes()) return ATTN_ERR_INVALID_ARG;
-  if (!e4m3 && !split && rope_cos == nullptr) {
-    // bf16 without a split last wave: the column-split kernel (one Q tile per unit)
+  if (!e4m3 && !split && use_column_split(N, D, causal)) {
+    // the column-split kernel (one Q tile per unit)
     CUtensorMap mo;
     if ((st = encode_map_o(&mo, o, (long long)B * Hq, N, D)) != ATTN_OK) return st;
     attn::CsParams cp;
@@ -436,8 +441,6 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   p.ws_ml = split ? reinterpret_cast<float*>(static_cast<char*>(workspace) + sc.cnt_bytes) : nullptr;
   p.ws_o = split ? reinterpret_cast<float*>(static_cast<char*>(workspace) + sc.cnt_bytes + sc.ml_bytes) : nullptr;
   p.epoch = split ? next_epoch() : 0u;
-  p.rope_cos = e4m3 ? nullptr : rope_cos;
-  p.rope_sin = e4m3 ? nullptr : rope_sin;
   const long long grid = sc.grid;
   if (e4m3) {
     if (D == 64)
@@ -839,13 +842,6 @@ int attn_fwd_rope(const void* q, const void* k, const void* v, const float* cos_
   if (need < 0) return ATTN_ERR_CUDA;
   const size_t rest = workspace_bytes - q_part - k_part;
   void* split_ws = (need > 0 && (size_t)need <= rest) ? ws + q_part + k_part : nullptr;
-  if (narrow_head_dim(D)) {
-    // D <= 128: the forward kernel rotates each Q tile in shared memory after loading it, so
-    // only K goes through the rotary kernel (into the workspace, at its K offset).
-    if ((st = launch_rope(k, k, cos_t, sin_t, ws + q_part, ws + q_part, B, 0, Hkv, N, D, s)) != ATTN_OK) return st;
-    return launch_forward(q, ws + q_part, v, o, lse, B, Hq, Hkv, N, D, causal, scale, split_ws, split_ws ? rest : 0,
-                          stream, false, 1.f, 1.f, cos_t, sin_t);
-  }
   if ((st = launch_rope(q, k, cos_t, sin_t, ws, ws + q_part, B, Hq, Hkv, N, D, s)) != ATTN_OK) return st;
   return launch_forward(ws, ws + q_part, v, o, lse, B, Hq, Hkv, N, D, causal, scale, split_ws,
                         split_ws ? rest : 0, stream);

@@ -1,6 +1,8 @@
 // attn_fwd_colsplit_kernel.cuh -- bf16 attention forward for head dims 32..128 on B200 (sm_100a),
 // one Q tile per work unit, two score buffers, and the score columns split between two softmax
-// warpgroups.
+// warpgroups.  The library runs it for causal D = 128 at N <= 2048, where it measured 5-8 %
+// faster than the two-tile kernel (attn_fwd_kernel.cuh); at longer N the two-tile kernel wins,
+// because there each K/V tile it loads serves 256 query rows instead of 128.
 //
 // Method: the tiled attention forward with an online softmax ("Making AMD GPUs go brrr",
 // section "Real kernel example": score matmul, exp2, row sums, probability-times-V matmul;

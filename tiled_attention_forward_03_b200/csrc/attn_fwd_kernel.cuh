@@ -73,7 +73,6 @@ enum : unsigned {
   kSiteDrain = 9,
   kSiteSelfTest = 10,
   kSiteSplitMerge = 11,
-  kSiteSoftmaxQ = 24,  // the softmax warpgroup waiting for its Q tile to rotate (fused RoPE)
 };
 
 __device__ unsigned int g_attn_fault_site = 0;
@@ -94,8 +93,7 @@ struct SmemPlan {
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] o_free[2] drain
-  // q_ready[2] (Q tile rotated in place, when RoPE is fused)
-  static constexpr int kNumBars = 4 + 2 * kStages + 8 + 1 + 2;
+  static constexpr int kNumBars = 4 + 2 * kStages + 8 + 1;
   // tmem base (u32), abort flag (u32), per-tile "last range" flags (2 x u32)
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
@@ -155,10 +153,6 @@ struct FwdParams {
   float o_scale;     // multiplies the normalised output (the V descale for E4M3 inputs, else 1)
   uint32_t idesc_s;  // S = Q K^T instruction descriptor (negates A when scale < 0)
   uint32_t idesc_pv; // O += P V instruction descriptor
-  // RoPE of Q fused into the kernel (bf16 only): tables [N][D/2] of cos and sin of the rotation
-  // angle of position p and frequency d, or null (Q is used as loaded).
-  const float* rope_cos;
-  const float* rope_sin;
 };
 
 struct Unit {
@@ -340,12 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_full = s_full + 4;
   uint64_t* o_free = s_full + 6;
   uint64_t* drain = s_full + 8;
-  uint64_t* q_ready = s_full + 9;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Plan::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Plan::kMiscOff + 4);
-  // With RoPE fused, the MMA warp waits for the softmax warpgroup to have rotated the Q tile.
-  const bool rope = !kF8 && p.rope_cos != nullptr;
-  uint64_t* q_mma = rope ? q_ready : q_full;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -353,7 +343,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
-      mbar_init(&q_ready[i], kBlockM);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], kBlockM);
@@ -507,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n0 = w.n0, n1 = w.valid1 ? w.n1 : 0;
 
         // First block's scores for both tiles.
-        if (!(ok = wait_all(&q_mma[0], q_par[0], kSiteMmaQ))) break;
+        if (!(ok = wait_all(&q_full[0], q_par[0], kSiteMmaQ))) break;
         q_par[0] ^= 1u;
         const uint32_t k0_stage = ring.stage;
         if (!(ok = wait_all(&kv_full[k0_stage], ring.phase, kSiteMmaKV))) break;
@@ -517,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         commit(&s_full[0]);
         if (n0 == jb + 1) commit(&q_empty[0]);
         if (n1 > 0) {
-          if (!(ok = wait_all(&q_mma[1], q_par[1], kSiteMmaQ))) break;
+          if (!(ok = wait_all(&q_full[1], q_par[1], kSiteMmaQ))) break;
           q_par[1] ^= 1u;
           tc_fence_after();
           issue_s(1, k0_stage);
@@ -576,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_s = tmem_base + lane_off + t * 128;
     const uint32_t t_o = tmem_base + lane_off + 256 + t * 128;
     const float c = p.c;
-    uint32_t s_par = 0u, o_par = 0u, qf_par = 0u;
+    uint32_t s_par = 0u, o_par = 0u;
     bool ok = true;
 
     for (int it = 0; ok; ++it) {
@@ -589,51 +578,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = w.q0 + t * kBlockM + r;
       const int key_lim = p.causal ? min(row, p.N - 1) : (p.N - 1);
       float m = -INFINITY, l = 0.f;
-
-      if constexpr (!kF8) {
-        if (rope) {
-          // RoPE of this thread's Q row in shared memory (rotate-half pairing: element d with
-          // d + D/2, d < D/2, angle of position `row`), in fp32 from the bf16 values and the
-          // fp32 tables, rounded to bf16: the arithmetic of the standalone rotary kernel.
-          if (!(ok = wait_phase(&q_full[t], qf_par, abort_flag, kSiteSoftmaxQ))) break;
-          qf_par ^= 1u;
-          if (row < p.N) {
-            uint8_t* qrow = sQ + t * Plan::kTileBytes + r * 128;
-            const float* cs_row = p.rope_cos + (size_t)row * (D / 2);
-            const float* sn_row = p.rope_sin + (size_t)row * (D / 2);
-            // 16-byte pieces of 8 elements: piece P (elements 8P..8P+7) pairs with P + D/16; in
-            // the 128-byte swizzle, piece P sits in chunk P/8 at position (P%8) ^ (r%8).
-#pragma unroll
-            for (int P = 0; P < D / 16; ++P) {
-              const int P2 = P + D / 16;
-              uint4* pa = reinterpret_cast<uint4*>(qrow + (P / 8) * Plan::kChunkBytes + (((P & 7) ^ (r & 7)) << 4));
-              uint4* pb = reinterpret_cast<uint4*>(qrow + (P2 / 8) * Plan::kChunkBytes + (((P2 & 7) ^ (r & 7)) << 4));
-              const uint4 ua = *pa, ub = *pb;
-              const float4 c0 = __ldg(reinterpret_cast<const float4*>(cs_row + 8 * P));
-              const float4 c1 = __ldg(reinterpret_cast<const float4*>(cs_row + 8 * P + 4));
-              const float4 s0 = __ldg(reinterpret_cast<const float4*>(sn_row + 8 * P));
-              const float4 s1 = __ldg(reinterpret_cast<const float4*>(sn_row + 8 * P + 4));
-              const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-              const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-              const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&ua);
-              const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&ub);
-              uint32_t oa[4], ob[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 a = __bfloat1622float2(ha[e]);
-                const float2 b = __bfloat1622float2(hb[e]);
-                oa[e] = pack_bf16x2(fmaf(a.x, cs[2 * e], -b.x * sn[2 * e]), fmaf(a.y, cs[2 * e + 1], -b.y * sn[2 * e + 1]));
-                ob[e] = pack_bf16x2(fmaf(b.x, cs[2 * e], a.x * sn[2 * e]), fmaf(b.y, cs[2 * e + 1], a.y * sn[2 * e + 1]));
-              }
-              *pa = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-              *pb = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-            }
-          }
-          // the tensor core (async proxy) reads the rotated tile next
-          fence_proxy_async_smem();
-          mbar_arrive(&q_ready[t]);
-        }
-      }
 
       for (int j = w.jb; j < n; ++j) {
         if (!(ok = wait_phase(&s_full[t], s_par, abort_flag, kSiteSoftmaxS))) break;
