@@ -131,6 +131,9 @@ EDGE = [
     (1, 2, 2, 256, 128, False), (1, 2, 2, 257, 128, True), (2, 4, 2, 383, 64, True),
     (1, 4, 1, 1000, 128, True), (1, 4, 1, 1000, 128, False), (1, 8, 1, 640, 64, True),
     (3, 8, 4, 300, 128, False), (1, 16, 2, 513, 128, True),
+    # causal GQA past N = 2048 at D = 128 (two-tile kernel, units of two query heads of one KV head):
+    # ragged tail, odd tile count (the middle step holds one unit), groups 2 and 4
+    (1, 4, 2, 2100, 128, True), (2, 8, 2, 2304, 128, True),
 ]
 
 

@@ -158,3 +158,58 @@ def test_causal_steps_pair_heavy_with_light(N):
     if N % 512 == 0:  # no ragged tail: every step is a full pair of pairs
         assert len(set(totals.values())) == 1
     assert all(len(v) in (1, 2) for v in work.values())
+
+
+def walk_head_pairs(B, Hq, Hkv, N, sms):
+    """Causal GQA with an even group: a unit is query tile `tile` of heads 2hp and 2hp + 1 (one KV
+    head), both tiles seeing KV blocks 0..tile; steps pair a head pair's heaviest and lightest tiles."""
+    assert (Hq // Hkv) % 2 == 0
+    T = -(-N // BLOCK)
+    steps = B * (Hq // 2) * ((T + 1) // 2)
+    grid = min(steps, sms)
+    sph = (T + 1) // 2
+    g = Hq // Hkv
+    items = []
+    for cta in range(grid):
+        it = 0
+        while True:
+            step = cta + (it >> 1) * grid
+            if step >= steps:
+                break
+            slot, s = divmod(step, sph)
+            part = it & 1
+            tile = T - 1 - s if part == 0 else s
+            if not (part == 1 and tile == T - 1 - s):
+                b, hp = divmod(slot, Hq // 2)
+                h0 = b * Hq + 2 * hp
+                items.append(dict(cta=cta, step=step, heads=(h0, h0 + 1), kv=b * Hkv + (2 * hp) // g,
+                                  rows=tile * BLOCK, n=min(T, tile + 1)))
+            it += 1
+    return T, items
+
+
+@pytest.mark.parametrize("sms", [1, 7, 148])
+@pytest.mark.parametrize("B,Hq,Hkv,N", [(1, 2, 1, 1), (1, 4, 2, 300), (2, 8, 2, 1000), (8, 32, 8, 8192),
+                                        (1, 4, 1, 4097), (3, 6, 3, 256)])
+def test_head_pair_units_cover_every_tile_once(B, Hq, Hkv, N, sms):
+    T, items = walk_head_pairs(B, Hq, Hkv, N, sms)
+    seen = {}
+    for w in items:
+        h0, h1 = w["heads"]
+        assert h1 == h0 + 1 and h0 // Hq == h1 // Hq           # same batch row
+        g = Hq // Hkv
+        assert (h0 % Hq) // g == (h1 % Hq) // g                # same KV head
+        assert w["kv"] == (h0 // Hq) * Hkv + (h0 % Hq) // g
+        assert 0 <= w["rows"] < N and w["n"] == w["rows"] // BLOCK + 1
+        for h in (h0, h1):
+            seen[(h, w["rows"] // BLOCK)] = seen.get((h, w["rows"] // BLOCK), 0) + 1
+    assert seen == {(h, t): 1 for h in range(B * Hq) for t in range(T)}
+
+
+def test_head_pair_steps_balance_work():
+    T, items = walk_head_pairs(2, 8, 2, 8192, 148)
+    work = {}
+    for w in items:
+        work.setdefault(w["step"], []).append(w["n"])
+    full = [sum(v) for v in work.values() if len(v) == 2]
+    assert set(full) == {T + 1}

@@ -365,6 +365,15 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   p.causal = causal ? 1 : 0;
   p.units_per_step = p.causal ? 2 : 1;
   p.num_steps = p.causal ? (long long)B * Hq * ((p.num_pairs + 1) / 2) : p.num_units;
+  // Causal GQA with an even group: units pair two query heads of one KV head at the same query
+  // tile (both tiles then see the same KV blocks; no lone diagonal block for tile 1).
+  p.head_pairs = (p.causal && (Hq / Hkv) % 2 == 0) ? 1 : 0;
+  p.div_hq2 = attn::make_fast_div((uint32_t)(Hq / 2 > 0 ? Hq / 2 : 1));
+  if (p.head_pairs) {
+    p.num_pairs = p.num_blocks;                                         // units per head pair
+    p.num_units = (long long)B * (Hq / 2) * p.num_blocks;
+    p.num_steps = (long long)B * (Hq / 2) * ((p.num_blocks + 1) / 2);
+  }
   p.div_pairs = attn::make_fast_div((uint32_t)p.num_pairs);
   p.div_steps = attn::make_fast_div((uint32_t)((p.num_pairs + 1) / 2));
   p.div_hq = attn::make_fast_div((uint32_t)Hq);
@@ -442,25 +451,28 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   p.ws_o = split ? reinterpret_cast<float*>(static_cast<char*>(workspace) + sc.cnt_bytes + sc.ml_bytes) : nullptr;
   p.epoch = split ? next_epoch() : 0u;
   const long long grid = sc.grid;
+  // O as a TMA store target for the two-tile kernel: bf16, boxes of 64 columns x 128 rows
+  CUtensorMap mo;
+  if ((st = encode_map(&mo, o, (long long)B * Hq, N, D, 2)) != ATTN_OK) return st;
   if (e4m3) {
     if (D == 64)
       attn::attn_fwd_sm100<64, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64, true>::kAlloc, s>>>(
-          mq, mk, mv, p);
+          mq, mk, mv, mo, p);
     else
       attn::attn_fwd_sm100<128, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128, true>::kAlloc, s>>>(
-          mq, mk, mv, p);
+          mq, mk, mv, mo, p);
   } else switch (D) {
     case 32:
-      attn::attn_fwd_sm100<32><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32>::kAlloc, s>>>(mq, mk, mv, p);
+      attn::attn_fwd_sm100<32><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32>::kAlloc, s>>>(mq, mk, mv, mo, p);
       break;
     case 64:
-      attn::attn_fwd_sm100<64><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(mq, mk, mv, p);
+      attn::attn_fwd_sm100<64><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(mq, mk, mv, mo, p);
       break;
     case 96:
-      attn::attn_fwd_sm100<96><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<96>::kAlloc, s>>>(mq, mk, mv, p);
+      attn::attn_fwd_sm100<96><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<96>::kAlloc, s>>>(mq, mk, mv, mo, p);
       break;
     default:
-      attn::attn_fwd_sm100<128><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128>::kAlloc, s>>>(mq, mk, mv, p);
+      attn::attn_fwd_sm100<128><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128>::kAlloc, s>>>(mq, mk, mv, mo, p);
       break;
   }
   e = cudaGetLastError();

@@ -12,7 +12,8 @@
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp  8    TMA producer: Q tiles once per unit, K_j / V_j through a smem ring
 //   warp  9    MMA issuer (one elected lane): S_t = Q_t K_j^T and O_t += P_t V_j on tcgen05
-//   warps 10-11 idle (they complete the third warpgroup, which gives up registers)
+//   warp  10   output store (bf16 D = 128): TMA tensor stores of each tile's O, staged in shared memory
+//   warp  11   idle (completes the third warpgroup, which gives up registers)
 //
 // A work unit is 256 query rows (two 128-row tiles) of one query head; a persistent
 // grid walks the units with a static stride.  Units of one head are adjacent (and
@@ -73,6 +74,8 @@ enum : unsigned {
   kSiteDrain = 9,
   kSiteSelfTest = 10,
   kSiteSplitMerge = 11,
+  kSiteStore = 25,      // the store warp waiting for a staged O tile
+  kSiteStageFree = 26,  // a softmax warpgroup waiting for the staging buffer
 };
 
 __device__ unsigned int g_attn_fault_site = 0;
@@ -91,13 +94,22 @@ struct SmemPlan {
   static constexpr int kStages = (kChunks == 2) ? 4 : 8;    // K/V ring depth
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  // bf16 D = 128: one tile's O (bf16) staged for the TMA store: 64-column chunks of 128-byte rows,
+  // 128-byte swizzle, the two tiles using it in turn (measured 1-3 % faster than 16-byte stores
+  // from the softmax warps at D = 128, and 6-10 % slower at D = 64, where the softmax warps bound
+  // the kernel; other instances store O directly)
+  static constexpr bool kStagedStore = !kF8 && D == 128;
+  static constexpr int kOChunks = (D + 63) / 64;
+  static constexpr int kOStageOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kOStageOff + (kStagedStore ? kOChunks * kChunkBytes : 0);
   // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] o_free[2] drain
-  static constexpr int kNumBars = 4 + 2 * kStages + 8 + 1;
+  // o_staged stage_free
+  static constexpr int kNumBars = 4 + 2 * kStages + 8 + 1 + 2;
   // tmem base (u32), abort flag (u32), per-tile "last range" flags (2 x u32)
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;              // slack for 1024-byte alignment
+  static_assert(kAlloc <= 232448, "forward shared memory plan exceeds 227 KB");
 };
 
 // Division by a divisor fixed for the launch, as a multiply-high by a precomputed reciprocal
@@ -149,6 +161,11 @@ struct FwdParams {
   FastDiv div_steps;  // (num_pairs + 1) / 2: causal scheduling steps per head
   FastDiv div_hq;     // Hq
   FastDiv div_group;  // group
+  // Causal with an even GQA group: a unit is one 128-row query tile of two query heads that
+  // share a KV head (tile 0 head h, tile 1 head h + 1, the same rows), so both tiles see the same
+  // KV blocks.  num_pairs is then the query-tile count and the "head" of a step is a head pair.
+  int head_pairs;
+  FastDiv div_hq2;    // Hq / 2
   float c;           // |scale| * log2(e) (times the Q and K descales for E4M3 inputs)
   float o_scale;     // multiplies the normalised output (the V descale for E4M3 inputs, else 1)
   uint32_t idesc_s;  // S = Q K^T instruction descriptor (negates A when scale < 0)
@@ -157,7 +174,9 @@ struct FwdParams {
 
 struct Unit {
   int q0;          // first query row of tile 0
-  int head_q;      // b * Hq + hq
+  int head_q;      // b * Hq + hq (tile 0)
+  int row1;        // first query row of tile 1
+  int head_q1;     // query head of tile 1
   int head_kv;     // b * Hkv + hq / group
   int jb;          // first KV block of this work item (0 unless the unit is split)
   int n0, n1;      // end (exclusive) of the KV blocks visited by tile 0 / tile 1
@@ -176,6 +195,8 @@ __device__ __forceinline__ Unit make_unit(const FwdParams& p, uint32_t head, int
   w.head_q = (int)head;
   w.head_kv = (int)(b * (uint32_t)p.Hkv + fast_div(hq, p.div_group));
   w.valid1 = (w.q0 + kBlockM) < p.N;
+  w.row1 = w.q0 + kBlockM;
+  w.head_q1 = (int)head;
   if (p.causal) {
     w.n0 = min(p.num_blocks, 2 * pair + 1);
     w.n1 = min(p.num_blocks, 2 * pair + 2);
@@ -198,6 +219,25 @@ __device__ __forceinline__ Unit make_unit(const FwdParams& p, uint32_t head, int
 // one head (and the heads of one GQA group are consecutive), so K/V tiles are shared
 // through L2 by the CTAs running at the same time.  Returns false if the step has no
 // such unit (the middle pair of a head with an odd pair count).
+// Head-pair unit (causal, even GQA group): query tile `tile` of heads 2hp and 2hp + 1 of batch b.
+__device__ __forceinline__ Unit make_unit_hp(const FwdParams& p, uint32_t slot, int tile) {
+  Unit w;
+  const uint32_t b = fast_div(slot, p.div_hq2);
+  const uint32_t hq0 = 2u * (slot - b * p.div_hq2.d);
+  w.q0 = tile * kBlockM;
+  w.row1 = w.q0;
+  w.head_q = (int)(b * (uint32_t)p.Hq + hq0);
+  w.head_q1 = w.head_q + 1;
+  w.head_kv = (int)(b * (uint32_t)p.Hkv + fast_div(hq0, p.div_group));
+  w.valid1 = true;
+  w.n0 = w.n1 = w.nmax = min(p.num_blocks, tile + 1);
+  w.jb = 0;
+  w.parts = 1;
+  w.part = 0;
+  w.tail = 0;
+  return w;
+}
+
 __device__ __forceinline__ bool unit_at(const FwdParams& p, uint32_t step, int part, Unit& w) {
   if (!p.causal) {
     const uint32_t head = fast_div(step, p.div_pairs);
@@ -208,7 +248,7 @@ __device__ __forceinline__ bool unit_at(const FwdParams& p, uint32_t step, int p
   const int s = (int)(step - head * p.div_steps.d);
   const int pair = part == 0 ? p.num_pairs - 1 - s : s;
   if (part == 1 && pair == p.num_pairs - 1 - s) return false;
-  w = make_unit(p, head, pair);
+  w = p.head_pairs ? make_unit_hp(p, head, pair) : make_unit(p, head, pair);
   return true;
 }
 
@@ -310,7 +350,8 @@ struct Ring {
 template <int D, bool kF8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                   const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
+                   const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
+                   const FwdParams p) {
   using Plan = SmemPlan<D, kF8>;
   // 32-byte K steps of the tensor-core instructions: 16 bf16 or 32 E4M3 elements each
   constexpr int kSSteps = D * Plan::kElemBytes / 32;
@@ -334,6 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_full = s_full + 4;
   uint64_t* o_free = s_full + 6;
   uint64_t* drain = s_full + 8;
+  uint64_t* o_staged = s_full + 9;   // a tile's O is in the staging buffer (128 arrivals)
+  uint64_t* stage_free = s_full + 10;  // the store warp's TMA stores have read it
+  uint8_t* sOst = smem + Plan::kOStageOff;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Plan::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Plan::kMiscOff + 4);
 
@@ -354,6 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(o_staged, kBlockM);
+    mbar_init(stage_free, 1);
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -365,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
+    tma_prefetch_desc(&tmap_o);
   }
   tc_fence_before();
   __syncthreads();
@@ -415,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (got == 0) break;
         if (got == 2) continue;
         ok = load_q(0, w.q0, w.head_q) && load_kv(&tmap_k, w.jb * kBlockN, w.head_kv) &&
-             (!w.valid1 || load_q(1, w.q0 + kBlockM, w.head_q)) && load_kv(&tmap_v, w.jb * kBlockN, w.head_kv);
+             (!w.valid1 || load_q(1, w.row1, w.head_q1)) && load_kv(&tmap_v, w.jb * kBlockN, w.head_kv);
         for (int j = w.jb + 1; j < w.nmax && ok; ++j)
           ok = load_kv(&tmap_k, j * kBlockN, w.head_kv) && load_kv(&tmap_v, j * kBlockN, w.head_kv);
       }
@@ -566,6 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_o = tmem_base + lane_off + 256 + t * 128;
     const float c = p.c;
     uint32_t s_par = 0u, o_par = 0u;
+    uint32_t stage_uses = 0u;  // tiles staged before this unit (both tiles, in the store warp's order)
     bool ok = true;
 
     for (int it = 0; ok; ++it) {
@@ -573,9 +621,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int got_item = item_at(p, it, w);
       if (got_item == 0) break;
       if (got_item == 2) continue;
+      // staging order: per unit without a split, tile 0 then (if it has rows) tile 1
+      const uint32_t my_use = stage_uses + (uint32_t)t;
+      if (w.parts == 1) stage_uses += w.valid1 ? 2u : 1u;
       if (t == 1 && !w.valid1) continue;
       const int n = t ? w.n1 : w.n0;
-      const int row = w.q0 + t * kBlockM + r;
+      const int row = (t ? w.row1 : w.q0) + r;
+      const int head_o = t ? w.head_q1 : w.head_q;   // query head of this tile's rows
       const int key_lim = p.causal ? min(row, p.N - 1) : (p.N - 1);
       float m = -INFINITY, l = 0.f;
 
@@ -722,8 +774,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       o_par ^= 1u;
       tc_fence_after();
       const bool row_ok = row < p.N;
-      __nv_bfloat16* orow = p.o + ((size_t)w.head_q * p.N + (row_ok ? row : 0)) * D;
-      if (w.parts == 1) {
+      __nv_bfloat16* orow = p.o + ((size_t)head_o * p.N + (row_ok ? row : 0)) * D;
+      if (w.parts == 1 && Plan::kStagedStore) {
+        // O / l -> bf16 pairs in registers; O's tensor memory is then free for the next unit.
+        const float inv_l = 1.f / l;
+        uint32_t packed[D / 2];
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t ov[32];
+          tmem_ld32(t_o + ch * 32, ov);
+          tmem_ld_wait();
+          reg_fence32(ov);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            packed[16 * ch + i] =
+                pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+        }
+        tc_fence_before();
+        mbar_arrive(&o_free[t]);
+        // Stage the row (64-column chunks, 128-byte swizzle: piece q of row r at q ^ (r % 8)) once
+        // the previous tile's stores have read the buffer, then hand it to the store warp.
+        if (my_use > 0 && !(ok = wait_phase(stage_free, (my_use - 1u) & 1u, abort_flag, kSiteStageFree))) break;
+        const uint32_t srow = smem_u32(sOst) + r * 128;
+#pragma unroll
+        for (int q = 0; q < D / 8; ++q)
+          st_shared_v4(srow + (q >> 3) * Plan::kChunkBytes + (((q & 7) ^ (r & 7)) << 4), packed[4 * q],
+                       packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+        fence_proxy_async_smem();
+        mbar_arrive(o_staged);
+        if (row_ok) p.lse[(size_t)head_o * p.N + row] = (m + log2f(l)) * 0.69314718055994530942f;
+      } else if (w.parts == 1) {
         const float inv_l = (kF8 ? p.o_scale : 1.f) / l;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
@@ -744,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&o_free[t]);
-        if (row_ok) p.lse[(size_t)w.head_q * p.N + row] = (m + log2f(l)) * 0.69314718055994530942f;
+        if (row_ok) p.lse[(size_t)head_o * p.N + row] = (m + log2f(l)) * 0.69314718055994530942f;
       } else {
         // One of the two KV ranges of a split unit.  The ranges first agree on their
         // finishing order; the first publishes its unnormalised O rows and (m, l) and
@@ -845,13 +925,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                   dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
               }
             }
-            if (row_ok) p.lse[(size_t)w.head_q * p.N + row] = (mt + log2f(lt)) * 0.69314718055994530942f;
+            if (row_ok) p.lse[(size_t)head_o * p.N + row] = (mt + log2f(lt)) * 0.69314718055994530942f;
           }
           tc_fence_before();
           mbar_arrive(&o_free[t]);
         }
       }
     }
+  } else if (warp == 10 && Plan::kStagedStore) {
+    // ------------------------------------------------------------ output store warp
+    // Tiles in the order the softmax warpgroups stage them (per unit without a split: tile 0,
+    // then tile 1 if it has rows): wait until staged, store with TMA (rows past N are not
+    // written), wait until the stores have read the buffer and release it.
+    regs_decrease<kRegsControl>();
+    if (lane == 0) {
+      uint32_t st_par = 0u;
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        Unit w;
+        const int got = item_at(p, it, w);
+        if (got == 0) break;
+        if (got == 2 || w.parts > 1) continue;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (t == 1 && !w.valid1) continue;
+          if (!(ok = wait_phase(o_staged, st_par, abort_flag, kSiteStore))) break;
+          st_par ^= 1u;
+#pragma unroll
+          for (int ch = 0; ch < Plan::kOChunks; ++ch)
+            tma_store_3d(&tmap_o, sOst + ch * Plan::kChunkBytes, ch * 64, t ? w.row1 : w.q0, t ? w.head_q1 : w.head_q);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(stage_free);
+        }
+      }
+      // every TMA store has completed before the CTA exits
+      bulk_wait_group0();
+    }
+    __syncwarp();
   } else {
     regs_decrease<kRegsControl>();
   }
