@@ -181,6 +181,14 @@ def test_backward_cfg4_sampled_kv_head(attn):
     check_heads(attn, CFG4, [(3, 6)])
 
 
+@pytest.mark.parametrize("name,heads", [("sweep_D128_N8192_noncausal", [(1, 15)]),
+                                        ("sweep_D64_N4096_causal", [(0, 0), (3, 9)])])
+def test_backward_sweep_benchmark_shapes_sampled_heads(attn, name, heads):
+    """The other workloads the backward is benchmarked on, at full size: whole KV heads."""
+    from attn_inputs import get_workload
+    check_heads(attn, get_workload(name), heads)
+
+
 @pytest.mark.parametrize("B,Hq,Hkv", [(3, 4, 2), (1, 8, 2)])
 def test_backward_host_path_in_pieces_equals_device_call(attn, B, Hq, Hkv):
     """backward_from_host pipelines batch rows (or whole KV-head groups when B == 1); the
