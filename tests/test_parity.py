@@ -13,7 +13,7 @@ import torch
 
 from oracle import attention_forward, attention_rows, head_forward
 from attn_inputs import (
-    CFG1, CFG2, CFG3, CFG4, make_qkv, make_workload_inputs, sample_rows, sweep_points, wide_points)
+    CFG1, CFG2, CFG3, CFG4, Workload, make_qkv, make_workload_inputs, sample_rows, sweep_points, wide_points)
 
 pytestmark = pytest.mark.gpu
 
@@ -56,9 +56,10 @@ def check_full(attn, q, k, v, causal, scale, what=""):
     return o, lse
 
 
-def check_sampled(attn, w, q, k, v, count=256, full_heads=((0, 0),)):
+def check_sampled(attn, w, q, k, v, count=256, full_heads=((0, 0),), rows=None):
     o, lse = gpu_forward(attn, q, k, v, w.causal, w.softmax_scale)
-    rows = sample_rows(w.B, w.Hq, w.N, count, seed=w.seed + 7)
+    if rows is None:
+        rows = sample_rows(w.B, w.Hq, w.N, count, seed=w.seed + 7)
     o_ref, lse_ref = attention_rows(q, k, v, rows, w.causal, w.softmax_scale)
     idx = tuple(np.array(x) for x in zip(*rows))
     assert_close(o[idx], lse[idx], o_ref, lse_ref, w.name + " sampled rows")
@@ -142,6 +143,37 @@ def test_edge_shapes(attn, shape):
     B, Hq, Hkv, N, D, causal = shape
     q, k, v = make_qkv(B, Hq, Hkv, N, D, seed=3000 + N + D + Hq)
     check_full(attn, q, k, v, causal, 1.0 / math.sqrt(D), str(shape))
+
+
+LONG = [
+    # (B, Hq, Hkv, N, D, causal): sequences past the benchmark sizes, up to 128K keys per head
+    (1, 2, 1, 131072, 128, True), (1, 2, 1, 131072, 128, False), (1, 2, 2, 65536, 64, True),
+    (1, 3, 3, 100000, 128, False),
+]
+
+
+@pytest.mark.parametrize("shape", LONG, ids=lambda s: "B{}_Hq{}_Hkv{}_N{}_D{}_{}".format(*s[:5], "c" if s[5] else "nc"))
+def test_long_sequences_sampled(attn, shape):
+    """Long sequences (1024 KV blocks per head at N = 128K): seeded rows against the oracle row
+    by row, and the LSE bounds on those rows."""
+    B, Hq, Hkv, N, D, causal = shape
+    w = Workload(f"long_B{B}_Hq{Hq}_Hkv{Hkv}_N{N}_D{D}_{'c' if causal else 'nc'}", B, Hq, Hkv, N, D, causal,
+                 4000 + N % 997 + D)
+    q, k, v = make_workload_inputs(w)
+    # rows on both sides of the edges of twelve query tiles (the first two, the last two and
+    # eight seeded ones) of the last head, the first and last rows, and 48 seeded draws
+    g = np.random.default_rng(w.seed)
+    T = -(-N // 128)
+    tiles = {0, 1, T - 2, T - 1} | set(int(x) for x in g.choice(T, 8, replace=False))
+    rows = {(0, 0, 0), (B - 1, Hq - 1, N - 1)}
+    for t in tiles:
+        for i in (t * 128 - 1, t * 128, t * 128 + 127):
+            if 0 <= i < N:
+                rows.add((B - 1, Hq - 1, i))
+    for x in g.integers(0, B * Hq * N, 48):
+        b, rem = divmod(int(x), Hq * N)
+        rows.add((b, rem // N, rem % N))
+    check_sampled(attn, w, q, k, v, full_heads=(), rows=sorted(rows))
 
 
 HEAD_DIMS = [
