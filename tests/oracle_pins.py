@@ -8,12 +8,14 @@ oracle and checks that each planted mistake fails at least one pin.
 """
 from __future__ import annotations
 
+import functools
 import json
 import math
 import os
 
 import numpy as np
 import torch
+from threadpoolctl import threadpool_limits
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "tiny_closed_form.json")
 TIGHT = 1e-12
@@ -249,9 +251,26 @@ def pin_large_scores(impl):
     _close(L[0, 0, 0], 900.0 + math.log1p(w), 1e-12, "large-score LSE")
 
 
-ALL_PINS = [
+def _single_threaded(pin):
+    """Runs a pin with one BLAS thread and one torch thread.  The pins compare fp64 results at
+    1e-10 and tighter; with several threads a library call was seen, rarely, to differ from its
+    own single-threaded result by ~6e-10 (torch.logsumexp beside the oracle's LSE), which says
+    nothing about the oracle."""
+    @functools.wraps(pin)
+    def run(impl):
+        threads = torch.get_num_threads()
+        torch.set_num_threads(1)
+        try:
+            with threadpool_limits(1):
+                return pin(impl)
+        finally:
+            torch.set_num_threads(threads)
+    return run
+
+
+ALL_PINS = [_single_threaded(p) for p in (
     pin_golden, pin_brute_force, pin_torch_sdpa, pin_row_sums, pin_identical_v_rows,
     pin_causal_first_query, pin_permutation, pin_single_key, pin_uniform_scores,
     pin_causal_prefix, pin_gqa_is_repeated_mha, pin_key_shift, pin_linear_in_v,
     pin_large_scores,
-]
+)]
