@@ -21,6 +21,7 @@ import numpy as np
 import torch
 
 from oracle import attention_forward
+from oracle_pins import _single_threaded
 
 
 def _rand(shape, seed, scale=1.0):
@@ -245,8 +246,9 @@ def pin_bwd_golden(impl):
             _close(got, np.array(c[name]), 1e-12, f"golden {c['name']} {name}")
 
 
-ALL_BWD_PINS = [
+# one BLAS thread and one torch thread, as for the forward pins (their tolerances are as tight)
+ALL_BWD_PINS = [_single_threaded(p) for p in (
     pin_bwd_golden, pin_bwd_finite_differences, pin_bwd_torch_autograd, pin_bwd_brute_force, pin_bwd_dv_sums,
     pin_bwd_dk_sums_zero, pin_bwd_key_shift, pin_bwd_uniform, pin_bwd_identical_v, pin_bwd_single_key,
     pin_bwd_causal_first_query, pin_bwd_gqa_is_repeated_mha, pin_bwd_linear_in_do,
-]
+)]
