@@ -366,10 +366,10 @@ def run_ours(args, w):
         if tables or fp8:
             e2e_path = ("forward_from_host: pinned host q,k,v -> device, "
                         + ("attn_fwd_rope (device-resident cos/sin tables)" if tables else "attn_fwd_fp8 (E4M3 inputs)")
-                        + ", o,lse -> pinned host; in 4 pieces (batch rows), torch copies overlapping the kernels")
+                        + ", o,lse -> pinned host; in 8 pieces (batch rows), torch copies overlapping the kernels")
         else:
             e2e_path = ("attn_fwd_from_host (C ABI, called by forward_from_host): pinned host q,k,v -> device "
-                        "buffers, attn_fwd_ws per piece, o,lse -> pinned host; 4 pieces (batch rows), the "
+                        "buffers, attn_fwd_ws per piece, o,lse -> pinned host; 8 pieces (batch rows), the "
                         "library's copy streams overlapping the kernels; returns after the last download")
     for _ in range(2):
         e2e_call()

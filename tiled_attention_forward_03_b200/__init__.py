@@ -369,7 +369,7 @@ def _pipelined(dev, stream, pieces, inputs, outputs, compute):
 
 def forward_from_host(q, k, v, causal: bool = False, scale: float | None = None, device=None,
                       out_host=None, lse_host=None, stream=None, rope_tables=None, fp8_descales=None,
-                      pieces: int = 4):
+                      pieces: int = 8):
     """End-to-end call on host (ideally pinned) tensors: copy in, attention, copy out.
 
     Returns host tensors (o, lse).  The problem is cut into up to ``pieces`` independent parts
