@@ -4,7 +4,11 @@
 column-split case) coordinates, in each CTA, the TMA producer warp, the MMA-issuing warp, the
 tensor pipe (which runs MMAs and commits in issue order), two softmax warpgroups (one per 128-row
 query tile; P is written over the tile's scores in tensor memory) and, for bf16 D = 128, a store
-warp that writes each tile's O from a shared-memory staging buffer with TMA stores.  Split units
+warp that writes each tile's O from a shared-memory staging buffer with TMA stores.  For
+non-causal bf16 D <= 64 the kernel takes a second form (`sep` below): P has tensor-memory columns
+of its own beside O, and each tile has its own MMA warp, which issues the tile's next S once the
+softmax has read the current one (S-free and P-free barriers; each K/V stage is released by both
+MMA warps, used or not).  Split units
 of a non-causal last wave add a protocol between two CTAs: the KV range that finishes first
 publishes its unnormalised rows and (m, l) in the workspace and raises a ready flag; the other
 waits for the flag and merges.
@@ -100,8 +104,9 @@ def blocks_needed(P, tile):
     return set(range(min(P["num_blocks"], tile[1] + 1))) if P["causal"] else set(range(P["num_blocks"]))
 
 
-def run_grid(P, ctas, S_stages, staged, rng, mutation=None):
-    """All agents of all CTAs in one random interleaving; returns the outputs written."""
+def run_grid(P, ctas, S_stages, staged, rng, mutation=None, sep=False):
+    """All agents of all CTAs in one random interleaving; returns the outputs written.  sep: the
+    D <= 64 form (P in columns of its own, one MMA warp per tile)."""
     outputs = {}                     # (head, tile) -> set of KV blocks folded into the written rows
     ws = {}                          # (tail, t) -> {"count", "ready", "rows"}
     agents, pending, done = {}, {}, set()
@@ -115,14 +120,19 @@ def run_grid(P, ctas, S_stages, staged, rng, mutation=None):
                 bars[f"{name}{t}"] = Barrier(f"{name}{t}", count)
         for s in range(S_stages):
             bars[f"kv_full{s}"] = Barrier(f"kv_full{s}", 1)
-            bars[f"kv_empty{s}"] = Barrier(f"kv_empty{s}", 1)
-        for name, count in (("drain", 1), ("o_staged", BLOCK), ("stage_free", 1)):
+            bars[f"kv_empty{s}"] = Barrier(f"kv_empty{s}", 2 if sep else 1)
+        for name, count in (("drain", 2 if sep else 1), ("o_staged", BLOCK), ("stage_free", 1)):
             bars[name] = Barrier(name, count)
+        for t in range(2):
+            bars[f"s_free{t}"] = Barrier(f"s_free{t}", BLOCK)
+            bars[f"p_free{t}"] = Barrier(f"p_free{t}", 1)
         st = {
             "stage": [None] * S_stages, "stage_busy": [0] * S_stages,
             "q": [None, None], "q_busy": [0, 0],
             "s": [None, None],       # ("S" | "P", item index, block) held in tile t's score columns
             "p_read": [True, True],  # the P in the score columns has been read by its P V
+            "p": [None, None],       # sep: ("P", item index, block) in tile t's own P columns
+            "s_read": [True, True],  # sep: the softmax has read the S in tile t's score columns
             "o": [None, None],       # [item index, blocks accumulated, epilogue read]
             "pv_last": [(-1, -1), (-1, -1)],   # (item, block) of tile t's last completed P V
             "staging": None, "store_reading": False,
@@ -250,8 +260,92 @@ def run_grid(P, ctas, S_stages, staged, rng, mutation=None):
             commit("drain")
             yield from W("drain", 0, 0)
 
+        def mma_sep(t):
+            """The D <= 64 form: one MMA warp per tile; a tile's next S follows the softmax's read of
+            the current one; every ring stage is released by both warps (used or not)."""
+            stage, phase, uses = 0, 0, [0] * S_stages
+            cnt = {"q": 0, "p": 0, "s": 0, "o": 0}
+            issued = False
+
+            def take():
+                nonlocal stage, phase
+                s_ = stage
+                yield from W(f"kv_full{s_}", phase, uses[s_])
+                uses[s_] += 1
+                stage += 1
+                if stage == S_stages:
+                    stage, phase = 0, phase ^ 1
+                return s_
+
+            def issue_s(i, j, s_):
+                nonlocal issued
+                if issued and mutation != "sep_s_without_free":
+                    yield from W(f"s_free{t}", cnt["s"] & 1, cnt["s"])
+                    cnt["s"] += 1
+                issued = True
+                assert st["stage"][s_] == ("K", i, j), f"S({t},{i},{j}) reads {st['stage'][s_]}"
+                assert st["q"][t] == i, "S reads the wrong Q tile"
+                st["stage_busy"][s_] += 1
+                st["q_busy"][t] += 1
+                tensor_q.append(("S", t, i, j, s_))
+                tensor_q.append(("commit", f"s_full{t}"))
+
+            for i, w in seq:
+                jb = w["jb"]
+                n = w["n0"] if t == 0 else w["n1"]
+                j_end = jb
+                if n > jb:
+                    yield from W(f"q_full{t}", cnt["q"] & 1, cnt["q"])
+                    cnt["q"] += 1
+                    ks = yield from take()
+                    yield from issue_s(i, jb, ks)
+                    if n == jb + 1:
+                        tensor_q.append(("commit", f"q_empty{t}"))
+                    tensor_q.append(("commit", f"kv_empty{ks}"))
+                    for j in range(jb, n):
+                        vs, vuse = stage, uses[stage]
+                        stage += 1
+                        if stage == S_stages:
+                            stage, phase = 0, phase ^ 1
+                        if j + 1 < n:
+                            ks = yield from take()
+                            yield from issue_s(i, j + 1, ks)
+                            if j + 2 == n:
+                                tensor_q.append(("commit", f"q_empty{t}"))
+                            tensor_q.append(("commit", f"kv_empty{ks}"))
+                        yield from W(f"p_full{t}", cnt["p"] & 1, cnt["p"])
+                        cnt["p"] += 1
+                        if j == jb:
+                            yield from W(f"o_free{t}", (cnt["o"] - 1) & 1 if cnt["o"] else 1, cnt["o"] - 1)
+                            cnt["o"] += 1
+                        yield from W(f"kv_full{vs}", vuse & 1, vuse)
+                        uses[vs] = vuse + 1
+                        assert st["stage"][vs] == ("V", i, j), f"PV({t},{i},{j}) reads {st['stage'][vs]}"
+                        assert st["p"][t] == ("P", i, j), f"PV({t},{i},{j}) reads P {st['p'][t]}"
+                        st["stage_busy"][vs] += 1
+                        tensor_q.append(("PV", t, i, j, vs, j > jb))
+                        if mutation != "sep_p_free_dropped":
+                            tensor_q.append(("commit", f"p_free{t}"))
+                        if j == n - 1:
+                            tensor_q.append(("commit", f"o_full{t}"))
+                        tensor_q.append(("commit", f"kv_empty{vs}"))
+                    j_end = n
+                for j in range(j_end, w["nmax"]):
+                    for _ in range(2):
+                        if mutation == "sep_skip_without_wait":
+                            s_ = stage
+                            uses[s_] += 1
+                            stage += 1
+                            if stage == S_stages:
+                                stage, phase = 0, phase ^ 1
+                        else:
+                            s_ = yield from take()
+                        bars[f"kv_empty{s_}"].arrive()
+            tensor_q.append(("commit", "drain"))
+            yield from W("drain", 0, 0)
+
         def softmax(t):
-            s_uses, o_uses, stage_uses = 0, 0, 0
+            s_uses, o_uses, stage_uses, p_uses = 0, 0, 0, 0
             for i, w in seq:
                 my_use = stage_uses + t
                 if w["parts"] == 1:
@@ -263,10 +357,20 @@ def run_grid(P, ctas, S_stages, staged, rng, mutation=None):
                     yield from W(f"s_full{t}", s_uses & 1, s_uses)
                     s_uses += 1
                     assert st["s"][t] == ("S", i, j), f"softmax {t} reads {st['s'][t]} for {(i, j)}"
+                    if sep:
+                        st["s_read"][t] = True
+                        bars[f"s_free{t}"].arrive(BLOCK)
+                        if p_uses > 0:
+                            yield from W(f"p_free{t}", (p_uses - 1) & 1, p_uses - 1)
+                        assert st["p_read"][t], "P rewritten before its P V read it"
+                        p_uses += 1
                     if j > w["jb"]:
                         # the lazy O rescale: the P V of every earlier block has completed
                         assert st["pv_last"][t] == (i, j - 1), "O rescaled while a P V still runs"
-                    st["s"][t] = ("P", i, j)
+                    if sep:
+                        st["p"][t] = ("P", i, j)
+                    else:
+                        st["s"][t] = ("P", i, j)
                     st["p_read"][t] = False
                     bars[f"p_full{t}"].arrive(BLOCK)
                 yield from W(f"o_full{t}", o_uses & 1, o_uses)
@@ -330,13 +434,17 @@ def run_grid(P, ctas, S_stages, staged, rng, mutation=None):
             op = tensor_q.pop(0)
             if op[0] == "S":
                 _, t, i, j, s = op
-                assert st["p_read"][t], "S overwrote a P that its P V had not read"
+                if sep:
+                    assert st["s_read"][t], "S overwrote scores the softmax had not read"
+                    st["s_read"][t] = False
+                else:
+                    assert st["p_read"][t], "S overwrote a P that its P V had not read"
                 st["s"][t] = ("S", i, j)
                 st["stage_busy"][s] -= 1
                 st["q_busy"][t] -= 1
             elif op[0] == "PV":
                 _, t, i, j, v, acc = op
-                assert st["s"][t] == ("P", i, j)
+                assert (st["p"] if sep else st["s"])[t] == ("P", i, j)
                 st["p_read"][t] = True
                 if not acc:
                     prev = st["o"][t]
@@ -358,7 +466,11 @@ def run_grid(P, ctas, S_stages, staged, rng, mutation=None):
                 st["stage"][op[1]] = op[2]
                 bars[f"kv_full{op[1]}"].arrive()
 
-        progs = {"producer": producer(), "mma": mma(), "sm0": softmax(0), "sm1": softmax(1)}
+        progs = {"producer": producer(), "sm0": softmax(0), "sm1": softmax(1)}
+        if sep:
+            progs["mma0"], progs["mma1"] = mma_sep(0), mma_sep(1)
+        else:
+            progs["mma"] = mma()
         if staged:
             progs["store"] = store()
         return dict(bars=bars, state=st, tensor_q=tensor_q, tma_q=tma_q, progs=progs,
@@ -448,6 +560,18 @@ def test_protocol_runs_without_deadlock_or_race(case, stages, staged):
         check_outputs(P, ctas, outputs)
 
 
+@pytest.mark.parametrize("stages", [4, 8])
+@pytest.mark.parametrize("case", CASES)
+def test_separate_p_protocol_runs_without_deadlock_or_race(case, stages):
+    """The separate-P form (non-causal D <= 64 runs it with an 8-stage ring; 4 stages as a
+    harder case, and the causal and head-pair items as well)."""
+    B, Hq, Hkv, N, causal, sms = case
+    P, ctas = schedule(B, Hq, Hkv, N, causal, sms)
+    for seed in range(8):
+        outputs = run_grid(P, ctas, stages, False, random.Random(104729 * seed + N), sep=True)
+        check_outputs(P, ctas, outputs)
+
+
 def test_cases_cover_split_tails_head_pairs_and_empty_slots():
     kinds = set()
     for B, Hq, Hkv, N, causal, sms in CASES:
@@ -465,10 +589,12 @@ def test_cases_cover_split_tails_head_pairs_and_empty_slots():
     assert kinds == {"empty", "split", "head_pair", "lone_tile"}
 
 
-@pytest.mark.parametrize("mutation", ["kv_empty_before_s1", "o_free_parity", "q_empty_dropped",
-                                      "kv_empty_next_dropped", "stage_free_dropped", "stage_without_free",
-                                      "flag_before_rows"])
-def test_planted_protocol_mistakes_are_caught(mutation):
+@pytest.mark.parametrize("mutation,sep", [
+    ("kv_empty_before_s1", False), ("o_free_parity", False), ("q_empty_dropped", False),
+    ("kv_empty_next_dropped", False), ("stage_free_dropped", False), ("stage_without_free", False),
+    ("flag_before_rows", False), ("sep_s_without_free", True), ("sep_p_free_dropped", True),
+    ("sep_skip_without_wait", True)])
+def test_planted_protocol_mistakes_are_caught(mutation, sep):
     """Each planted mistake makes some interleaving deadlock or read the wrong data."""
     caught = False
     for case in CASES:
@@ -476,7 +602,7 @@ def test_planted_protocol_mistakes_are_caught(mutation):
         P, ctas = schedule(B, Hq, Hkv, N, causal, sms)
         for seed in range(8):
             try:
-                outputs = run_grid(P, ctas, 4, True, random.Random(seed), mutation=mutation)
+                outputs = run_grid(P, ctas, 4, not sep, random.Random(seed), mutation=mutation, sep=sep)
                 check_outputs(P, ctas, outputs)
             except (AssertionError, Deadlock):
                 caught = True

@@ -85,6 +85,8 @@ bool device_setup(int dev, int* num_sms) {
     setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<64>), attn::CsPlan<64>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<96>), attn::CsPlan<96>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<128>), attn::CsPlan<128>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<32, false, true>), attn::SmemPlan<32>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, false, true>), attn::SmemPlan<64>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, true>), attn::SmemPlan<64, true>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<128, true>), attn::SmemPlan<128, true>::kAlloc);
     // the wide-head kernel has no register split: dynamic shared memory opt-in only
@@ -462,11 +464,21 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
       attn::attn_fwd_sm100<128, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128, true>::kAlloc, s>>>(
           mq, mk, mv, mo, p);
   } else switch (D) {
+    // non-causal D <= 64: P beside O, one MMA warp per tile (2-7 % faster there; causal units
+    // are short, and there it measured 0 to 8 % slower)
     case 32:
-      attn::attn_fwd_sm100<32><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32>::kAlloc, s>>>(mq, mk, mv, mo, p);
+      if (!p.causal)
+        attn::attn_fwd_sm100<32, false, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32>::kAlloc, s>>>(
+            mq, mk, mv, mo, p);
+      else
+        attn::attn_fwd_sm100<32><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32>::kAlloc, s>>>(mq, mk, mv, mo, p);
       break;
     case 64:
-      attn::attn_fwd_sm100<64><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(mq, mk, mv, mo, p);
+      if (!p.causal)
+        attn::attn_fwd_sm100<64, false, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(
+            mq, mk, mv, mo, p);
+      else
+        attn::attn_fwd_sm100<64><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(mq, mk, mv, mo, p);
       break;
     case 96:
       attn::attn_fwd_sm100<96><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<96>::kAlloc, s>>>(mq, mk, mv, mo, p);

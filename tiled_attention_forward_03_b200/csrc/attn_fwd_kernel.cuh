@@ -15,6 +15,10 @@
 //   warp  10   output store (bf16 D = 128): TMA tensor stores of each tile's O, staged in shared memory
 //   warp  11   idle (completes the third warpgroup, which gives up registers)
 //
+// Non-causal bf16 D <= 64 (kSepP): P gets tensor-memory columns of its own beside O, and each
+// tile has its own MMA warp (warp 9: tile 0, warp 11: tile 1), which issues the tile's next S as
+// soon as its softmax has read the current one, so S no longer waits for the P V before it.
+//
 // A work unit is 256 query rows (two 128-row tiles) of one query head; a persistent
 // grid walks the units with a static stride.  Units of one head are adjacent (and
 // the heads of one GQA group are adjacent) so K/V blocks are re-read from L2; in the
@@ -24,6 +28,7 @@
 //   [  0,128) S_0 fp32 scores of tile 0; its first 64 columns are overwritten by P_0 (bf16x2)
 //   [128,256) S_1 / P_1
 //   [256,256+D) O_0 fp32 accumulator;  [384,384+D) O_1
+//   kSepP (D <= 64): P_0 at [320,384) and P_1 at [448,512) instead of over the scores
 //
 // Online softmax in base 2 with c = |scale| * log2(e):  m = running max of s*c,
 // p = 2^(s*c - m), l = sum p.  The max is applied lazily: O and l are rescaled only
@@ -55,8 +60,8 @@ constexpr float kRescaleLog2 = 8.0f;
 // Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial instead of the
 // special-function unit; measured best on B200: 2 at D=128, 1 at D=64 (more polynomial work
 // costs issue slots that the MMA-issuing warp shares with the softmax warps).
-template <int D, bool kF8 = false>
-__host__ __device__ constexpr int poly_pairs_per8() { return D == 128 ? 2 : 1; }
+template <int D, bool kF8 = false, bool kSepP = false>
+__host__ __device__ constexpr int poly_pairs_per8() { return (D == 128 || kSepP) ? 2 : 1; }
 // (D = 32 and 96 take 1 of 8, like D = 64: their tensor work per block is smaller than at
 // D = 128, so the exponentials weigh more and fewer issue slots can go to the polynomial.)
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s for any single wait
@@ -76,6 +81,8 @@ enum : unsigned {
   kSiteSplitMerge = 11,
   kSiteStore = 25,      // the store warp waiting for a staged O tile
   kSiteStageFree = 26,  // a softmax warpgroup waiting for the staging buffer
+  kSitePFree = 27,      // kSepP: a softmax warpgroup waiting for the last P V to have read P
+  kSiteMmaSFree = 28,   // kSepP: an MMA warp waiting for the softmax to have read S
 };
 
 __device__ unsigned int g_attn_fault_site = 0;
@@ -103,8 +110,8 @@ struct SmemPlan {
   static constexpr int kOStageOff = kKVOff + kStages * kTileBytes;
   static constexpr int kBarOff = kOStageOff + (kStagedStore ? kOChunks * kChunkBytes : 0);
   // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] o_free[2] drain
-  // o_staged stage_free
-  static constexpr int kNumBars = 4 + 2 * kStages + 8 + 1 + 2;
+  // o_staged stage_free s_free[2] p_free[2] (the last four used by the separate-P form only)
+  static constexpr int kNumBars = 4 + 2 * kStages + 8 + 1 + 2 + 4;
   // tmem base (u32), abort flag (u32), per-tile "last range" flags (2 x u32)
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
@@ -347,12 +354,13 @@ struct Ring {
   }
 };
 
-template <int D, bool kF8 = false>
+template <int D, bool kF8 = false, bool kSepP = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
                    const FwdParams p) {
   using Plan = SmemPlan<D, kF8>;
+  static_assert(!kSepP || (D <= 64 && !kF8), "P beside O needs D <= 64 (bf16)");
   // 32-byte K steps of the tensor-core instructions: 16 bf16 or 32 E4M3 elements each
   constexpr int kSSteps = D * Plan::kElemBytes / 32;
   constexpr int kPVSteps = kBlockN * Plan::kElemBytes / 32;
@@ -377,6 +385,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = s_full + 8;
   uint64_t* o_staged = s_full + 9;   // a tile's O is in the staging buffer (128 arrivals)
   uint64_t* stage_free = s_full + 10;  // the store warp's TMA stores have read it
+  uint64_t* s_free = s_full + 11;      // kSepP: the softmax has read S_t (128 arrivals)
+  uint64_t* p_free = s_full + 13;      // kSepP: P_t V completed
   uint8_t* sOst = smem + Plan::kOStageOff;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Plan::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Plan::kMiscOff + 4);
@@ -395,9 +405,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < S; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], kSepP ? 2 : 1);   // kSepP: released by both MMA warps
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, kSepP ? 2 : 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_free[i], kBlockM);
+      mbar_init(&p_free[i], 1);
+    }
     mbar_init(o_staged, kBlockM);
     mbar_init(stage_free, 1);
     *abort_flag = 0u;
@@ -471,6 +485,135 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (filled & (1u << s)) drain_phase(&kv_full[s], (fill_par >> s) & 1u, abort_flag);
       for (int t = 0; t < 2; ++t)
         if (q_filled[t]) drain_phase(&q_full[t], q_fill_par[t], abort_flag);
+    }
+    __syncwarp();
+  } else if (kSepP && (warp == 9 || warp == 11)) {
+    // ------------------------------------------------------------ MMA issuers, one per tile (D <= 64)
+    // P has tensor-memory columns of its own, so a tile's next S is issued as soon as its
+    // softmax has read the current one; each warp walks the K/V ring in the producer's order
+    // and releases every stage it passes (a stage is refilled once both tiles released it).
+    regs_decrease<kRegsControl>();
+    {
+      const int t = (warp == 9) ? 0 : 1;
+      Ring ring;
+      // bit 0: Q full parity, 1: P full, 2: S free, 3: O free; bit 4: an S was issued before
+      uint32_t par = 0x8u;
+      const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_base, 0);
+      const uint64_t desc_q = smem_desc_kmajor_sw128(smem_u32(sQ)) + (uint64_t)((t * Plan::kTileBytes) >> 4);
+      const uint64_t desc_k = smem_desc_kmajor_sw128(smem_u32(sKV));
+      const uint64_t desc_v = smem_desc_mnmajor_sw128(smem_u32(sKV), Plan::kChunkBytes);
+      const uint32_t idesc_s = p.idesc_s, idesc_pv = p.idesc_pv;
+      const uint32_t t_sacc = tmem + t * 128;          // S of this tile
+      const uint32_t t_oacc = tmem + 256 + t * 128;    // O of this tile
+      const uint32_t t_pa = t_oacc + 64;               // P of this tile
+
+      auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+      auto wait_all = [&](uint64_t* bar, uint32_t parity, unsigned site) -> bool {
+        const bool mine = wait_phase(bar, parity, abort_flag, site);
+        return __all_sync(0xffffffffu, mine);
+      };
+      auto commit = [&](uint64_t* bar) {
+        if (elect_one()) tc_commit(bar);
+        __syncwarp();
+      };
+      // Next ring stage: waits until it holds its tile; returns the stage.
+      auto take = [&](uint32_t& st) -> bool {
+        st = ring.stage;
+        const bool got = wait_all(&kv_full[st], ring.phase, kSiteMmaKV);
+        ring.advance<S>();
+        return got;
+      };
+      // S = Q_t K^T into this tile's score columns, once the softmax has read the previous S.
+      auto issue_s = [&](uint32_t stage) -> bool {
+        if (par & 0x10u) {
+          if (!wait_all(&s_free[t], (par >> 2) & 1u, kSiteMmaSFree)) return false;
+          par ^= 0x4u;
+        }
+        par |= 0x10u;
+        tc_fence_after();
+        const uint64_t db = adv(desc_k, stage * Plan::kTileBytes);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kSSteps; ++kk) {
+            const uint32_t off = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
+            if constexpr (kF8)
+              mma_ss_f8(t_sacc, adv(desc_q, off), adv(db, off), idesc_s, kk > 0 ? 1u : 0u);
+            else
+              mma_ss(t_sacc, adv(desc_q, off), adv(db, off), idesc_s, kk > 0 ? 1u : 0u);
+          }
+        }
+        __syncwarp();
+        commit(&s_full[t]);
+        return true;
+      };
+
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        Unit w;
+        const int got = item_at(p, it, w);
+        if (got == 0) break;
+        if (got == 2) continue;
+        const int jb = w.jb;
+        const int n = t ? (w.valid1 ? w.n1 : 0) : w.n0;
+        int j_end = jb;
+        if (n > jb) {
+          uint32_t ks;
+          if (!(ok = wait_all(&q_full[t], par & 1u, kSiteMmaQ))) break;
+          par ^= 0x1u;
+          if (!(ok = take(ks))) break;
+          if (!(ok = issue_s(ks))) break;
+          if (n == jb + 1) commit(&q_empty[t]);
+          commit(&kv_empty[ks]);
+          for (int j = jb; j < n; ++j) {
+            const uint32_t vs = ring.stage, vph = ring.phase;
+            ring.advance<S>();
+            if (j + 1 < n) {
+              if (!(ok = take(ks))) break;
+              if (!(ok = issue_s(ks))) break;
+              if (j + 2 == n) commit(&q_empty[t]);
+              commit(&kv_empty[ks]);
+            }
+            if (!(ok = wait_all(&p_full[t], (par >> 1) & 1u, kSiteMmaP))) break;
+            par ^= 0x2u;
+            if (j == jb) {
+              if (!(ok = wait_all(&o_free[t], (par >> 3) & 1u, kSiteMmaOFree))) break;
+              par ^= 0x8u;
+            }
+            if (!(ok = wait_all(&kv_full[vs], vph, kSiteMmaKV))) break;
+            tc_fence_after();
+            const uint64_t dv = adv(desc_v, vs * Plan::kTileBytes);
+            if (elect_one()) {
+#pragma unroll
+              for (int kk = 0; kk < kPVSteps; ++kk) {
+                if constexpr (kF8)
+                  mma_ts_f8(t_oacc, t_pa + kk * 8, adv(dv, kk * kPVStepBytes), idesc_pv, (j > jb || kk > 0) ? 1u : 0u);
+                else
+                  mma_ts(t_oacc, t_pa + kk * 8, adv(dv, kk * kPVStepBytes), idesc_pv, (j > jb || kk > 0) ? 1u : 0u);
+              }
+            }
+            __syncwarp();
+            commit(&p_free[t]);
+            if (j == n - 1) commit(&o_full[t]);
+            commit(&kv_empty[vs]);
+          }
+          if (!ok) break;
+          j_end = n;
+        }
+        // K/V stages of blocks this tile does not visit (a causal unit's last block for tile 0,
+        // every block when tile 1 has no rows): released once they hold their tile.
+        for (int j = j_end; j < w.nmax && ok; ++j) {
+#pragma unroll
+          for (int kv = 0; kv < 2 && ok; ++kv) {
+            uint32_t st;
+            if (!(ok = take(st))) break;
+            if (lane == 0) mbar_arrive(&kv_empty[st]);
+            __syncwarp();
+          }
+        }
+      }
+      // Drain: all MMAs issued by this warp complete before TMEM is released.
+      commit(drain);
+      drain_phase(drain, 0u, abort_flag);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -610,6 +753,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = threadIdx.x & 127;               // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem_base + lane_off + t * 128;
+    // where P goes: over the scores, or (kSepP) its own columns after O_t
+    const uint32_t t_p = kSepP ? tmem_base + lane_off + 256 + t * 128 + 64 : t_s;
+    uint32_t p_uses = 0u;   // kSepP: P tiles written by this warpgroup
     const uint32_t t_o = tmem_base + lane_off + 256 + t * 128;
     const float c = p.c;
     uint32_t s_par = 0u, o_par = 0u;
@@ -647,6 +793,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           reg_fence32(a1);
           reg_fence32(a2);
           reg_fence32(a3);
+          if constexpr (kSepP) {
+            // the scores are in registers: this tile's MMA warp may compute the next S over them
+            tc_fence_before();
+            mbar_arrive(&s_free[t]);
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             s[i] = __uint_as_float(a0[i]);
@@ -696,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int col = half * 64 + i;
               const float2 x = fma2(make_float2(s[col], s[col + 1]), c2, nm2);
               float2 pr;
-              if (((col >> 1) & 7) < poly_pairs_per8<D, kF8>()) {
+              if (((col >> 1) & 7) < poly_pairs_per8<D, kF8, kSepP>()) {
                 pr = exp2_poly2(x);
               } else {
                 pr.x = ex2_approx(x.x);
@@ -718,9 +869,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint32_t pk16[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) pk16[i] = pk[i];
-              tmem_st16(t_s + half * 16, pk16);
+              tmem_st16(t_p + half * 16, pk16);
             } else {
-              tmem_st32(t_s + half * 32, pk);
+              tmem_st32(t_p + half * 32, pk);
             }
           }
           const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
@@ -742,6 +893,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             l *= alpha;
             m = m_new;
           }
+        }
+        if constexpr (kSepP) {
+          // P_t's columns (and O_t, for a rescale) are free once the previous P_t V completed
+          if (p_uses > 0u && !(ok = wait_phase(&p_free[t], (p_uses - 1u) & 1u, abort_flag, kSitePFree))) break;
+          ++p_uses;
+          tc_fence_after();
         }
         l += exp_row(m);
         if (any_rescale) {
