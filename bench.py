@@ -440,7 +440,9 @@ def run_ours(args, w):
     else:
         # the kernel the library picks for this shape (bf16, no split last wave)
         colsplit = w.causal and w.D == 128 and w.N <= 2048
+        sep_p = not w.causal and w.D <= 64          # P beside O, one MMA warp per tile
         kernel = f"attn_fwd_colsplit_sm100<{w.D}>" if colsplit else (
+            f"attn_fwd_sm100<{w.D}, bf16, P beside O>" if sep_p else
             f"attn_fwd_sm100<{w.D}>" if w.D <= 128 else f"attn_fwd_wide_sm100<{w.D}>")
         algo_bytes = w.algorithmic_bytes
 
