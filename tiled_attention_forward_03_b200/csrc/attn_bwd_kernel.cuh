@@ -68,10 +68,12 @@ namespace attn {
 constexpr int kBwdThreads = 320;
 constexpr float kLog2e = 1.4426950408889634f;
 // Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial (exp2_poly2)
-// instead of the special-function unit.  Measured on B200: none is best here (the
-// backward's exponentials are not the limit; the polynomial's FMA work only delays P).
+// instead of the special-function unit.  Measured on B200 (interleaved A/B): at D = 64 the
+// exponentials bound the block and 3 of 8 is best (+7 to +13 % against none; 4 of 8 is
+// slower again), at D = 32 2 of 8 (+7 %); at D = 96 and 128 none (the polynomial's FMA work
+// only delays P there).
 template <int D, bool kKV>
-__host__ __device__ constexpr int bwd_poly_pairs_per8() { return 0; }
+__host__ __device__ constexpr int bwd_poly_pairs_per8() { return D <= 32 ? 2 : (D <= 64 ? 3 : 0); }
 
 enum : unsigned {
   kSiteBwdProducer = 12,
