@@ -58,16 +58,15 @@ constexpr int kBlockM = 128;  // query rows per tile
 constexpr int kBlockN = 128;  // keys per KV block
 constexpr float kRescaleLog2 = 8.0f;
 // Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial instead of the
-// special-function unit; measured best on B200: 2 at D=128, 1 at D=64 (more polynomial work
-// costs issue slots that the MMA-issuing warp shares with the softmax warps); 2 in the
-// separate-P form (both softmax warpgroups busy back to back); 3 for E4M3 at D = 64, whose
-// halved tensor work leaves the exponentials the limit (+4 to +12 % against 1).
+// special-function unit, measured best on B200 (interleaved A/B; more polynomial work costs
+// issue slots that the MMA-issuing warp shares with the softmax warps): bf16 2 at D = 128 and
+// 64, 3 at D = 96 and 32 (+3 to +6 % against 1 there); 2 in the separate-P form (both softmax
+// warpgroups busy back to back; 3 was slower); E4M3 2 at D = 128 and 3 at D = 64, whose halved
+// tensor work leaves the exponentials the limit (+4 to +12 % against 1).
 template <int D, bool kF8 = false, bool kSepP = false>
 __host__ __device__ constexpr int poly_pairs_per8() {
-  return kF8 ? (D == 128 ? 2 : 3) : ((D == 128 || kSepP) ? 2 : 1);
+  return kF8 ? (D == 128 ? 2 : 3) : (kSepP ? 2 : ((D == 128 || D == 64) ? 2 : 3));
 }
-// (D = 32 and 96 take 1 of 8, like D = 64: their tensor work per block is smaller than at
-// D = 128, so the exponentials weigh more and fewer issue slots can go to the polynomial.)
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s for any single wait
 
 // Fault-site codes written to g_attn_fault_site when a bounded wait gives up.
