@@ -135,6 +135,8 @@ EDGE = [
     # causal GQA past N = 2048 at D = 128 (two-tile kernel, units of two query heads of one KV head):
     # ragged tail, odd tile count (the middle step holds one unit), groups 2 and 4
     (1, 4, 2, 2100, 128, True), (2, 8, 2, 2304, 128, True),
+    # non-causal GQA at D = 64 and 32 (the separate-P form): ragged tails, split last waves
+    (2, 8, 2, 1000, 64, False), (2, 4, 1, 777, 32, False), (3, 6, 3, 2049, 64, False),
 ]
 
 
@@ -148,7 +150,7 @@ def test_edge_shapes(attn, shape):
 LONG = [
     # (B, Hq, Hkv, N, D, causal): sequences past the benchmark sizes, up to 128K keys per head
     (1, 2, 1, 131072, 128, True), (1, 2, 1, 131072, 128, False), (1, 2, 2, 65536, 64, True),
-    (1, 3, 3, 100000, 128, False),
+    (1, 3, 3, 100000, 128, False), (1, 4, 1, 131072, 64, False),
 ]
 
 
