@@ -2,7 +2,7 @@
  * attn.h -- C ABI of the B200 (sm_100a) attention library: the forward pass in bf16
  * (attn_fwd, attn_fwd_ws, attn_fwd_noalloc; attn_fwd_from_host on host buffers) and E4M3
  * (attn_fwd_fp8), its gradients (attn_bwd), and rotary position embedding of Q and K
- * (attn_rope_tables, attn_rope_qk, attn_fwd_rope).
+ * (attn_rope_tables, attn_rope_qk, attn_fwd_rope; their backward attn_rope_qk_inverse, attn_bwd_rope).
  *
  * The operation is the tiled attention forward pass named by "HipKittens:
  * fast and furious AMD kernels" (section "Performance results": an attention
@@ -304,6 +304,44 @@ int attn_fwd_rope(const void* q, const void* k, const void* v, const float* cos_
  * workspace of attn_fwd_workspace_bytes().  -1 on invalid sizes or a CUDA error.
  */
 long long attn_fwd_rope_workspace_bytes(int B, int Hq, int Hkv, int N, int D);
+
+/*
+ * attn_rope_qk_inverse -- the inverse of attn_rope_qk: rotates by -theta, i.e. for d < D/2
+ *     x_d       = y_d cos(theta_pd) + y_{d+D/2} sin(theta_pd)
+ *     x_{d+D/2} = y_{d+D/2} cos(theta_pd) - y_d sin(theta_pd).
+ * The rotation is orthogonal, so this is also its transpose: given the gradients of a loss with
+ * respect to RoPE(q) and RoPE(k) it returns the gradients with respect to q and k (the backward
+ * of the rotary step).  Arguments, layouts, tables, in-place use and errors as attn_rope_qk
+ * (dq_rot, dk_rot in; dq, dk out).
+ */
+int attn_rope_qk_inverse(const void* dq_rot, const void* dk_rot, const float* cos_t, const float* sin_t,
+                         void* dq, void* dk, int B, int Hq, int Hkv, int N, int D, void* stream);
+
+/*
+ * attn_bwd_rope -- the backward of attn_fwd_rope: gradients of a loss L with respect to q, k
+ * (before the rotation) and v, given dO = dL/dO for O = attention(RoPE(q), RoPE(k), v), with
+ * the forward's O and LSE (as attn_fwd_rope wrote them).  Three steps on `stream`: attn_rope_qk
+ * into the workspace, attn_bwd on the rotated tensors (writing dL/dRoPE(q), dL/dRoPE(k) into dq,
+ * dk, and dv), then attn_rope_qk_inverse on dq, dk in place.  Arguments as attn_bwd plus the
+ * tables of attn_rope_qk and
+ *   workspace        device pointer, 256-byte aligned, at least attn_bwd_rope_workspace_bytes()
+ *                    bytes; after the call it holds RoPE(q) at offset 0 and RoPE(k) at offset
+ *                    round_up(B*Hq*N*D*2, 256), then the backward's per-row data.
+ * D is 32, 64, 96 or 128 (the backward's head dims).  Every argument is checked before the
+ * first launch; errors as attn_bwd and attn_rope_qk (ATTN_ERR_INVALID_ARG for a null or too
+ * small workspace).
+ */
+int attn_bwd_rope(const void* q, const void* k, const void* v, const float* cos_t, const float* sin_t,
+                  const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                  int B, int Hq, int Hkv, int N, int D, int causal, float scale,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_bwd_rope_workspace_bytes -- workspace attn_bwd_rope needs: the rotated Q and K (each
+ * rounded up to 256 bytes) plus attn_bwd_workspace_bytes().  -1 on invalid sizes (D must be
+ * 32, 64, 96 or 128).
+ */
+long long attn_bwd_rope_workspace_bytes(int B, int Hq, int Hkv, int N, int D);
 
 /*
  * attn_fwd_fp8 -- the attention forward on E4M3 (8-bit float) Q, K and V.

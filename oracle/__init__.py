@@ -6,6 +6,7 @@ library and its Python binding) never does.
 """
 from .attn_ref import (  # noqa: F401
     attention_backward,
+    attention_backward_rope,
     attention_forward,
     attention_forward_rope,
     attention_rows,
@@ -15,4 +16,5 @@ from .attn_ref import (  # noqa: F401
     kv_head,
     rope_angles,
     rope_rotate,
+    rope_rotate_transpose,
 )

@@ -206,3 +206,26 @@ def rope_rotate(x, base: float = 10000.0, angles=None):
 def attention_forward_rope(q, k, v, causal: bool, scale: float, base: float = 10000.0):
     """Attention of RoPE(q), RoPE(k) and v (all fp64); returns (O, LSE) as attention_forward."""
     return attention_forward(rope_rotate(q, base), rope_rotate(k, base), v, causal, scale)
+
+
+# The backward of the rotary step.  Each (x_d, x_{d+D/2}) pair is turned by the 2x2 rotation
+# R(theta) = [[cos, -sin], [sin, cos]], so by the chain rule the gradient with respect to the
+# unrotated pair is R(theta)^T times the gradient with respect to the rotated one:
+#     g_d       =  g'_d cos(theta) + g'_{d+D/2} sin(theta)
+#     g_{d+D/2} = -g'_d sin(theta) + g'_{d+D/2} cos(theta)
+
+def rope_rotate_transpose(g, base: float = 10000.0, angles=None):
+    """R(theta)^T applied to the last dimension of g [..., N, D] (the rotation by -theta)."""
+    g = _as_f64(g)
+    N, D = g.shape[-2], g.shape[-1]
+    th = rope_angles(N, D, base) if angles is None else np.asarray(angles, dtype=np.float64)
+    c, s = np.cos(th), np.sin(th)
+    a, b = g[..., : D // 2], g[..., D // 2:]
+    return np.concatenate([a * c + b * s, b * c - a * s], axis=-1)
+
+
+def attention_backward_rope(q, k, v, do, causal: bool, scale: float, base: float = 10000.0):
+    """Gradients (dQ, dK, dV) of sum(O o dO) for O = attention(RoPE(q), RoPE(k), v): the
+    attention backward at the rotated inputs, then the rotation's transpose on dQ and dK."""
+    dqr, dkr, dv = attention_backward(rope_rotate(q, base), rope_rotate(k, base), v, do, causal, scale)
+    return rope_rotate_transpose(dqr, base), rope_rotate_transpose(dkr, base), dv

@@ -201,6 +201,51 @@ def test_fwd_rope_rejected_before_any_cuda_call(kw, expected):
     assert call_fwd_rope(**kw) == expected
 
 
+def call_rope_inverse(**kw):
+    args = dict(q=P, k=P, c=P, s=P, qo=P, ko=P, B=1, Hq=2, Hkv=1, N=128, D=128)
+    args.update(kw)
+    return attn.attn_rope_qk_inverse(args["q"], args["k"], args["c"], args["s"], args["qo"], args["ko"], args["B"],
+                                     args["Hq"], args["Hkv"], args["N"], args["D"], None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(q=None), INVALID), (dict(ko=None), INVALID), (dict(c=None), INVALID), (dict(Hq=3, Hkv=2), INVALID),
+    (dict(D=80), UNSUPPORTED), (dict(k=P + 8), MISALIGNED), (dict(qo=P + 2), MISALIGNED),
+])
+def test_rope_inverse_rejected_before_any_cuda_call(kw, expected):
+    assert call_rope_inverse(**kw) == expected
+    assert call_rope_inverse(B=0) == OK
+
+
+def call_bwd_rope(**kw):
+    args = dict(q=P, k=P, v=P, c=P, s=P, o=P, lse=P, do=P, dq=P, dk=P, dv=P, B=1, Hq=2, Hkv=1, N=128, D=128,
+                causal=0, scale=0.125, ws=P, nbytes=1 << 24)
+    args.update(kw)
+    return attn.attn_bwd_rope(args["q"], args["k"], args["v"], args["c"], args["s"], args["o"], args["lse"],
+                              args["do"], args["dq"], args["dk"], args["dv"], args["B"], args["Hq"], args["Hkv"],
+                              args["N"], args["D"], args["causal"], args["scale"], args["ws"], args["nbytes"], None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(v=None), INVALID), (dict(o=None), INVALID), (dict(lse=None), INVALID), (dict(do=None), INVALID),
+    (dict(dq=None), INVALID), (dict(dk=None), INVALID), (dict(dv=None), INVALID), (dict(ws=None), INVALID),
+    (dict(nbytes=1024), INVALID), (dict(scale=math.nan), INVALID), (dict(c=None), INVALID),
+    (dict(D=192), UNSUPPORTED), (dict(D=48), UNSUPPORTED), (dict(ws=P + 64), MISALIGNED),
+    (dict(dk=P + 8), MISALIGNED), (dict(lse=P + 2), MISALIGNED), (dict(do=P + 8), MISALIGNED),
+])
+def test_bwd_rope_rejected_before_any_cuda_call(kw, expected):
+    assert call_bwd_rope(**kw) == expected
+
+
+def test_bwd_rope_empty_problem_and_workspace_query():
+    assert call_bwd_rope(B=0) == OK and call_bwd_rope(N=0) == OK
+    need = attn.attn_bwd_rope_workspace_bytes(2, 4, 2, 300, 64)
+    rot = -(-2 * 4 * 300 * 64 * 2 // 256) * 256 + -(-2 * 2 * 300 * 64 * 2 // 256) * 256
+    assert need == rot + attn.attn_bwd_workspace_bytes(2, 4, 300)
+    assert attn.attn_bwd_rope_workspace_bytes(1, 2, 1, 100, 256) == -1
+    assert attn.attn_bwd_rope_workspace_bytes(0, 2, 1, 100, 64) == 0
+
+
 # ---------------------------------------------------------------- E4M3 forward
 
 def call_fp8(**kw):

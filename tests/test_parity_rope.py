@@ -1,5 +1,5 @@
-"""GPU parity: RoPE of Q and K, and the attention forward of the rotated tensors, against the
-fp64 oracle (needs a B200).
+"""GPU parity: RoPE of Q and K, the attention forward of the rotated tensors and the backward
+through both, against the fp64 oracle (needs a B200).
 
 The rotation alone: the kernel works in fp32 on the bf16 inputs and fp32 tables and rounds to
 bf16 (nearest even), so each element is within half a bf16 step of the exact rotation plus
@@ -15,8 +15,9 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import attention_forward, attention_forward_rope, attention_rows, rope_angles, rope_rotate
-from attn_inputs import CFG2, make_qkv
+from oracle import attention_backward, attention_forward, attention_forward_rope, attention_rows, rope_angles
+from oracle import rope_rotate, rope_rotate_transpose
+from attn_inputs import CFG2, make_dout, make_qkv
 
 pytestmark = pytest.mark.gpu
 
@@ -159,3 +160,81 @@ def test_forward_rope_long_sequence_sampled(attn):
         o_ref, l_ref = attention_rows(qr, kr, v[:, h // 2:h // 2 + 1], rows, True, D ** -0.5)
         idx = [r[2] for r in rows]
         assert_fwd_close(o[0, h, idx], lse[0, h, idx], o_ref, l_ref, f"long rope head {h}")
+
+
+# ------------------------------------------------------------------ the backward of the rotation
+
+def _pair_norm(x):
+    """Per element, the norm of its rotation pair (x_d, x_{d+D/2})."""
+    h = x.shape[-1] // 2
+    n = np.sqrt(x[..., :h] ** 2 + x[..., h:] ** 2)
+    return np.concatenate([n, n], axis=-1)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,base", [
+    (1, 2, 1, 300, 128, 10000.0), (2, 4, 4, 129, 64, 10000.0), (1, 3, 1, 77, 96, 500.0), (1, 2, 2, 1, 32, 10000.0),
+])
+def test_rope_inverse(attn, B, Hq, Hkv, N, D, base):
+    """attn_rope_qk_inverse against the oracle's transpose R^T (the same one-rounding bound as the
+    rotation), and rope followed by rope_inverse returning the inputs within the two roundings
+    (each at most half a bf16 step of its pair's norm)."""
+    q, k, _ = make_qkv(B, Hq, Hkv, N, D, 4100 + N)
+    cos_t, sin_t = attn.rope_tables(N, D, base, device="cuda")
+    gq, gk = attn.rope_inverse(q.cuda(), k.cuda(), cos_t, sin_t)
+    qr, kr = attn.rope(q.cuda(), k.cuda(), cos_t, sin_t)
+    q2, k2 = attn.rope_inverse(qr, kr, cos_t, sin_t)
+    torch.cuda.synchronize()
+    for got, back, x in ((gq, q2, q), (gk, k2, k)):
+        ref = rope_rotate_transpose(x, base)
+        g = got.float().cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6), float(np.max(np.abs(g - ref)))
+        xf = x.float().numpy().astype(np.float64)
+        b = back.float().cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(b - xf) <= 2.0 ** -7 * _pair_norm(xf) + 1e-6), float(np.max(np.abs(b - xf)))
+
+
+def _bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,causal", [
+    (1, 2, 2, 256, 128, False), (1, 2, 1, 200, 128, True), (2, 4, 1, 384, 64, True), (1, 2, 2, 130, 96, False),
+    (1, 2, 1, 300, 32, True), (1, 1, 1, 1, 64, False),
+])
+def test_backward_rope(attn, B, Hq, Hkv, N, D, causal):
+    """backward_rope (attn_bwd_rope) against the oracle: the rotation in fp64 rounded to bf16
+    (the operand type the backward kernels read), the fp64 attention backward, then R^T; held to
+    the backward's tolerance bars."""
+    from test_parity_bwd import assert_grad_close
+
+    q, k, v = make_qkv(B, Hq, Hkv, N, D, 4200 + N + D)
+    do = make_dout(B, Hq, N, D, 4300 + N + D)
+    scale = D ** -0.5
+    cos_t, sin_t = attn.rope_tables(N, D, device="cuda")
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    o, lse = attn.forward_rope(qd, kd, vd, cos_t, sin_t, causal=causal)
+    dq, dk, dv = attn.backward_rope(qd, kd, vd, cos_t, sin_t, o, lse, dod, causal=causal)
+    torch.cuda.synchronize()
+    st, site = attn.device_status()
+    assert st == attn.ATTN_OK, f"kernel wait gave up at site {site}"
+    qr, kr = _bf16(rope_rotate(q)), _bf16(rope_rotate(k))
+    rq, rk, rv = attention_backward(qr, kr, v, do, causal, scale)
+    ref = (rope_rotate_transpose(rq), rope_rotate_transpose(rk), rv)
+    for name, a, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        assert_grad_close(a.float().cpu().numpy().astype(np.float64), r, f"rope backward {name}")
+
+
+def test_backward_rope_is_rotate_backward_then_inverse(attn):
+    """attn_bwd_rope equals its three steps called one by one (bit for bit)."""
+    B, Hq, Hkv, N, D, causal = 2, 4, 2, 700, 128, True
+    q, k, v = (x.cuda() for x in make_qkv(B, Hq, Hkv, N, D, 4400))
+    do = make_dout(B, Hq, N, D, 4401).cuda()
+    cos_t, sin_t = attn.rope_tables(N, D, device="cuda")
+    o, lse = attn.forward_rope(q, k, v, cos_t, sin_t, causal=causal)
+    got = attn.backward_rope(q, k, v, cos_t, sin_t, o, lse, do, causal=causal)
+    qr, kr = attn.rope(q, k, cos_t, sin_t)
+    dqr, dkr, dv = attn.backward(qr, kr, v, o, lse, do, causal=causal)
+    dq, dk = attn.rope_inverse(dqr, dkr, cos_t, sin_t)
+    torch.cuda.synchronize()
+    for a, b in zip(got, (dq, dk, dv)):
+        assert torch.equal(a, b)

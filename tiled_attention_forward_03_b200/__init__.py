@@ -9,6 +9,7 @@ cannot be loaded, importing this package raises.
     dq, dk, dv = attn.backward(q, k, v, o, lse, do, causal=True)
     cos_t, sin_t = attn.rope_tables(N, D, device="cuda")
     o, lse = attn.forward_rope(q, k, v, cos_t, sin_t, causal=True)   # attention of RoPE(q), RoPE(k)
+    dq, dk, dv = attn.backward_rope(q, k, v, cos_t, sin_t, o, lse, do, causal=True)
 """
 from __future__ import annotations
 
@@ -27,7 +28,8 @@ __all__ = [
     "attn_version", "attn_selftest_exp2_poly", "attn_selftest_wait_timeout", "forward",
     "forward_from_host", "device_status", "attn_bwd", "attn_bwd_workspace_bytes", "backward",
     "backward_from_host", "attn_rope_qk", "attn_fwd_rope", "attn_fwd_rope_workspace_bytes", "rope_tables",
-    "rope", "forward_rope", "attn_fwd_fp8", "forward_fp8",
+    "rope", "forward_rope", "attn_fwd_fp8", "forward_fp8", "attn_rope_qk_inverse", "attn_bwd_rope",
+    "attn_bwd_rope_workspace_bytes", "rope_inverse", "backward_rope",
 ]
 
 ATTN_OK = 0
@@ -76,6 +78,12 @@ def _load() -> ctypes.CDLL:
     L.attn_fwd_rope.restype = i
     L.attn_fwd_rope_workspace_bytes.argtypes = [i, i, i, i, i]
     L.attn_fwd_rope_workspace_bytes.restype = ctypes.c_longlong
+    L.attn_rope_qk_inverse.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    L.attn_rope_qk_inverse.restype = i
+    L.attn_bwd_rope.argtypes = [vp] * 11 + [i, i, i, i, i, i, f, vp, ctypes.c_size_t, vp]
+    L.attn_bwd_rope.restype = i
+    L.attn_bwd_rope_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.attn_bwd_rope_workspace_bytes.restype = ctypes.c_longlong
     L.attn_fwd_ws.restype = i
     L.attn_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
     L.attn_fwd_workspace_bytes.restype = ctypes.c_longlong
@@ -184,6 +192,22 @@ def attn_fwd_rope_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> 
     return lib.attn_fwd_rope_workspace_bytes(B, Hq, Hkv, N, D)
 
 
+def attn_rope_qk_inverse(dq_rot, dk_rot, cos_t, sin_t, dq, dk, B, Hq, Hkv, N, D, stream) -> int:
+    """Direct call of the inverse RoPE entry point (pointers and stream as integers)."""
+    return lib.attn_rope_qk_inverse(dq_rot, dk_rot, cos_t, sin_t, dq, dk, B, Hq, Hkv, N, D, stream)
+
+
+def attn_bwd_rope(q, k, v, cos_t, sin_t, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, causal, scale, workspace,
+                  workspace_bytes, stream) -> int:
+    """Direct call of the RoPE backward entry point."""
+    return lib.attn_bwd_rope(q, k, v, cos_t, sin_t, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D,
+                             int(bool(causal)), float(scale), workspace, workspace_bytes, stream)
+
+
+def attn_bwd_rope_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, D: int) -> int:
+    return lib.attn_bwd_rope_workspace_bytes(B, Hq, Hkv, N, D)
+
+
 def attn_fwd_noalloc_scratch_bytes() -> int:
     return lib.attn_fwd_noalloc_scratch_bytes()
 
@@ -248,7 +272,8 @@ _workspaces: dict = {}
 
 def _workspace(device, nbytes: int, purpose: str, stream):
     """A cached device buffer of at least nbytes, per device, purpose ("fwd": the split-tail
-    schedule, "bwd": the backward pass's per-row delta and LSE, "rope": the rotated q and k)
+    schedule, "bwd": the backward pass's per-row delta and LSE, "rope": the rotated q and k,
+    "bwd_rope": the rotated q and k and the backward's per-row data)
     and stream.  Calls on one stream run in order, so they may share a buffer; calls on
     different streams get different buffers and may overlap on the GPU.  The buffer is marked
     as used on ``stream``, so that when a larger one replaces it, torch's allocator does not
@@ -584,6 +609,72 @@ def rope(q, k, cos_t, sin_t, q_out=None, k_out=None, stream=None):
     if st != ATTN_OK:
         raise AttnError(st, "attn_rope_qk")
     return q_out, k_out
+
+
+def rope_inverse(dq_rot, dk_rot, cos_t, sin_t, dq=None, dk=None, stream=None):
+    """The inverse (= transpose) of rope(): rotates by -theta.  Maps gradients with respect to
+    RoPE(q), RoPE(k) to gradients with respect to q, k; returns (dq, dk).  Pass dq=dq_rot,
+    dk=dk_rot to work in place."""
+    import torch
+
+    B, Hq, N, D = dq_rot.shape
+    Hkv = dk_rot.shape[1]
+    _check(dq_rot, "dq_rot", torch.bfloat16, (B, Hq, N, D))
+    _check(dk_rot, "dk_rot", torch.bfloat16, (B, Hkv, N, D))
+    _check(cos_t, "cos_t", torch.float32, (N, D // 2))
+    _check(sin_t, "sin_t", torch.float32, (N, D // 2))
+    dq = torch.empty_like(dq_rot) if dq is None else dq
+    dk = torch.empty_like(dk_rot) if dk is None else dk
+    _check(dq, "dq", torch.bfloat16, (B, Hq, N, D))
+    _check(dk, "dk", torch.bfloat16, (B, Hkv, N, D))
+    s = stream if stream is not None else torch.cuda.current_stream(dq_rot.device)
+    with torch.cuda.device(dq_rot.device):
+        st = attn_rope_qk_inverse(dq_rot.data_ptr(), dk_rot.data_ptr(), cos_t.data_ptr(), sin_t.data_ptr(),
+                                  dq.data_ptr(), dk.data_ptr(), B, Hq, Hkv, N, D, s.cuda_stream)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_rope_qk_inverse")
+    return dq, dk
+
+
+def backward_rope(q, k, v, cos_t, sin_t, o, lse, dout, causal: bool = False, scale: float | None = None,
+                  dq=None, dk=None, dv=None, stream=None):
+    """Backward of forward_rope (attn_bwd_rope): gradients (dq, dk, dv) with respect to the
+    unrotated q, k and v, given the forward's o and lse and dout.  The workspace (rotated q and k,
+    the backward's per-row data) is cached per device and stream."""
+    import torch
+
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, N, D]")
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    _check(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _check(k, "k", torch.bfloat16, (B, Hkv, N, D))
+    _check(v, "v", torch.bfloat16, (B, Hkv, N, D))
+    _check(cos_t, "cos_t", torch.float32, (N, D // 2))
+    _check(sin_t, "sin_t", torch.float32, (N, D // 2))
+    _check(o, "o", torch.bfloat16, (B, Hq, N, D))
+    _check(lse, "lse", torch.float32, (B, Hq, N))
+    _check(dout, "dout", torch.bfloat16, (B, Hq, N, D))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(dq, "dq", torch.bfloat16, (B, Hq, N, D))
+    _check(dk, "dk", torch.bfloat16, (B, Hkv, N, D))
+    _check(dv, "dv", torch.bfloat16, (B, Hkv, N, D))
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        ws_bytes = attn_bwd_rope_workspace_bytes(B, Hq, Hkv, N, D)
+        if ws_bytes < 0:
+            raise AttnError(ATTN_ERR_UNSUPPORTED, "attn_bwd_rope_workspace_bytes")
+        ws = _workspace(q.device, max(ws_bytes, 256), "bwd_rope", s)
+        st = attn_bwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), cos_t.data_ptr(), sin_t.data_ptr(),
+                           o.data_ptr(), lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                           dv.data_ptr(), B, Hq, Hkv, N, D, causal, scale, ws.data_ptr(), ws.numel(), s.cuda_stream)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_rope")
+    return dq, dk, dv
 
 
 def forward_rope(q, k, v, cos_t, sin_t, causal: bool = False, scale: float | None = None, out=None, lse=None,

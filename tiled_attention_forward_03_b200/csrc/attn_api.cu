@@ -804,15 +804,16 @@ int rope_checks(const void* q, const void* k, const float* cos_t, const float* s
   return ATTN_OK;
 }
 
+// sgn = +1: the rotation; -1: its inverse (= transpose), for gradients.
 int launch_rope(const void* q, const void* k, const float* cos_t, const float* sin_t, void* q_out, void* k_out,
-                int B, int Hq, int Hkv, int N, int D, cudaStream_t s) {
+                int B, int Hq, int Hkv, int N, int D, cudaStream_t s, float sgn = 1.0f) {
   const long long q_rows = (long long)B * Hq * N, k_rows = (long long)B * Hkv * N;
   const long long items = (q_rows + k_rows) * (D / 16);
   const int threads = 256;
   const long long per_block = (long long)threads * attn::kRopeItems;
   attn::attn_rope_qk<<<(unsigned)((items + per_block - 1) / per_block), threads, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k), cos_t, sin_t,
-      reinterpret_cast<__nv_bfloat16*>(q_out), reinterpret_cast<__nv_bfloat16*>(k_out), q_rows, k_rows, N, D);
+      reinterpret_cast<__nv_bfloat16*>(q_out), reinterpret_cast<__nv_bfloat16*>(k_out), q_rows, k_rows, N, D, sgn);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     record_cuda_error("rope kernel launch", e);
@@ -832,6 +833,54 @@ int attn_rope_qk(const void* q, const void* k, const float* cos_t, const float* 
   if (!q_out || !k_out) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q_out, 16) || !aligned(k_out, 16)) return ATTN_ERR_MISALIGNED;
   return launch_rope(q, k, cos_t, sin_t, q_out, k_out, B, Hq, Hkv, N, D, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_rope_qk_inverse(const void* dq_rot, const void* dk_rot, const float* cos_t, const float* sin_t, void* dq,
+                         void* dk, int B, int Hq, int Hkv, int N, int D, void* stream) {
+  int st = rope_checks(dq_rot, dk_rot, cos_t, sin_t, B, Hq, Hkv, N, D);
+  if (st != ATTN_OK || B == 0 || N == 0) return st;
+  if (!dq || !dk) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(dq, 16) || !aligned(dk, 16)) return ATTN_ERR_MISALIGNED;
+  return launch_rope(dq_rot, dk_rot, cos_t, sin_t, dq, dk, B, Hq, Hkv, N, D, reinterpret_cast<cudaStream_t>(stream),
+                     -1.0f);
+}
+
+long long attn_bwd_rope_workspace_bytes(int B, int Hq, int Hkv, int N, int D) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || N < 0 || !narrow_head_dim(D)) return -1;
+  if (B == 0 || N == 0) return 0;
+  const long long bwd = attn_bwd_workspace_bytes(B, Hq, N);
+  if (bwd < 0) return -1;
+  return (long long)(round256((size_t)B * Hq * N * D * 2) + round256((size_t)B * Hkv * N * D * 2)) + bwd;
+}
+
+int attn_bwd_rope(const void* q, const void* k, const void* v, const float* cos_t, const float* sin_t, const void* o,
+                  const float* lse, const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
+                  int D, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = rope_checks(q, k, cos_t, sin_t, B, Hq, Hkv, N, D);
+  if (st != ATTN_OK) return st;
+  if (!narrow_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * Hq * (((long long)N + attn::kBlockN - 1) / attn::kBlockN) > (1LL << 30))
+    return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return ATTN_OK;
+  // every argument of the three steps is checked before the first launch
+  if (!v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 256))
+    return ATTN_ERR_MISALIGNED;
+  const size_t q_part = round256((size_t)B * Hq * N * D * 2), k_part = round256((size_t)B * Hkv * N * D * 2);
+  const long long need = attn_bwd_workspace_bytes(B, Hq, N);
+  if (need < 0 || workspace_bytes < q_part + k_part + (size_t)need) return ATTN_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // RoPE(q), RoPE(k) into the workspace; the attention backward on them gives the gradients with
+  // respect to the rotated tensors, which the inverse rotation (the rotation's transpose) maps to
+  // q and k, in place
+  if ((st = launch_rope(q, k, cos_t, sin_t, ws, ws + q_part, B, Hq, Hkv, N, D, s)) != ATTN_OK) return st;
+  if ((st = attn_bwd(ws, ws + q_part, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, D, causal, scale,
+                     ws + q_part + k_part, workspace_bytes - q_part - k_part, stream)) != ATTN_OK)
+    return st;
+  return launch_rope(dq, dk, cos_t, sin_t, dq, dk, B, Hq, Hkv, N, D, s, -1.0f);
 }
 
 long long attn_fwd_rope_workspace_bytes(int B, int Hq, int Hkv, int N, int D) {

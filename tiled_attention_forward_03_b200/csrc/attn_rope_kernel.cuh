@@ -15,6 +15,10 @@
 // in fp32 arithmetic rounded to bf16 (nearest even).  A thread turns 8 pairs: one 16-byte
 // piece of each half of its row and the matching 32 bytes of each table row (the tables
 // stay in L2: every head reads them).  The output may alias the input.
+//
+// With sgn = -1 the kernel applies the inverse rotation (by -theta), which is also its
+// transpose: it maps gradients with respect to RoPE(q), RoPE(k) to gradients with respect to
+// q, k (the backward of the rotation; sgn = +1 multiplies sin by exactly 1).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -31,7 +35,7 @@ __global__ void __launch_bounds__(256) attn_rope_qk(const __nv_bfloat16* q, cons
                                                     const float* __restrict__ cos_t,
                                                     const float* __restrict__ sin_t, __nv_bfloat16* q_out,
                                                     __nv_bfloat16* k_out, long long q_rows, long long k_rows,
-                                                    int N, int D) {
+                                                    int N, int D, float sgn) {
   const int pieces = D / 16;  // 8-pair pieces per row
   const int half = D / 2;
   const long long q_items = q_rows * pieces;
@@ -77,7 +81,7 @@ __global__ void __launch_bounds__(256) attn_rope_qk(const __nv_bfloat16* q, cons
     for (int e = 0; e < 4; ++e) {
       const float2 a = __bfloat1622float2(pa[e]);
       const float2 b = __bfloat1622float2(pb[e]);
-      const float c_lo = cs[2 * e], c_hi = cs[2 * e + 1], s_lo = sn[2 * e], s_hi = sn[2 * e + 1];
+      const float c_lo = cs[2 * e], c_hi = cs[2 * e + 1], s_lo = sgn * sn[2 * e], s_hi = sgn * sn[2 * e + 1];
       oa[e] = pack_bf16x2(fmaf(a.x, c_lo, -b.x * s_lo), fmaf(a.y, c_hi, -b.y * s_hi));
       ob[e] = pack_bf16x2(fmaf(b.x, c_lo, a.x * s_lo), fmaf(b.y, c_hi, a.y * s_hi));
     }
