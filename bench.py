@@ -2,7 +2,7 @@
 """Benchmark of the B200 bf16 attention forward (TFLOP/s, % of the dense BF16 peak).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all] [--impl ours|reference]
-                    [--pass fwd|bwd]
+                    [--pass fwd|bwd|rope|fp8|bwd_rope]
 
 One step = one attention forward pass over the workload's batch (one kernel
 launch).  Default workload: the largest configuration, GQA B=8, Hq=32, Hkv=8,
@@ -27,6 +27,10 @@ forward's FLOP count, and adds the rotary kernel alone against the HBM roofline.
 
 `--pass fp8` times attn_fwd_fp8 on E4M3 inputs (N(0,1) x 16 rounded to E4M3, descale 1/16) with
 the forward's FLOP count, against the measured bf16 peak x 2 (the nominal E4M3/bf16 ratio).
+
+`--pass bwd_rope` times attn_bwd_rope (the rotary kernel on Q and K, the backward on the
+rotated tensors, the inverse rotation of dQ and dK) on the outputs of attn_fwd_rope, with the
+backward's FLOP count.
 
 `--impl reference` times the fp64 CPU oracle instead (the only other
 implementation of this path): each step is a bounded sample of the workload's
@@ -56,7 +60,11 @@ METRIC_FP8 = "attention fwd E4M3 (FP8) TFLOP/s (1 B200) and % of dense FP8 tenso
 FP8_OVER_BF16 = 2.0  # nominal dense E4M3 / bf16 tensor rate (4.5 / 2.25 PFLOP/s)
 METRIC_ROPE = "attention fwd with RoPE of Q and K TFLOP/s (bf16, 1 B200; forward FLOP count) and % of dense BF16 tensor peak"
 METRIC_BWD = "attention bwd TFLOP/s (bf16, 1 B200; 2.5x the forward FLOP count) and % of dense BF16 tensor peak"
-PASS_NAMES = {"fwd": "forward", "bwd": "backward", "rope": "forward with RoPE", "fp8": "forward, E4M3 inputs"}
+METRIC_BWD_ROPE = ("attention bwd through RoPE of Q and K TFLOP/s (bf16, 1 B200; 2.5x the forward FLOP count) "
+                   "and % of dense BF16 tensor peak")
+PASS_NAMES = {"fwd": "forward", "bwd": "backward", "rope": "forward with RoPE", "fp8": "forward, E4M3 inputs",
+              "bwd_rope": "backward through RoPE"}
+METRICS = {"fwd": METRIC, "bwd": METRIC_BWD, "rope": METRIC_ROPE, "fp8": METRIC_FP8, "bwd_rope": METRIC_BWD_ROPE}
 BWD_FLOP_RATIO = 2.5      # counted backward FLOPs / forward FLOPs (five matmuls against two)
 BWD_EXECUTED_RATIO = 7 / 5  # matmuls the kernels execute / matmuls counted (S and dP run twice)
 L2_FLUSH_BYTES = 512 << 20
@@ -230,7 +238,7 @@ def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = Fa
     query head.
 
     Returns (TFLOP/s, FLOPs done, seconds, heads done, sample description)."""
-    from oracle import head_backward, head_forward, rope_rotate
+    from oracle import head_backward, head_forward, rope_rotate, rope_rotate_transpose
     from attn_inputs import make_dout, make_qkv, make_qkv_e4m3
 
     q, k, v = make_qkv(1, w.Hq, w.Hkv, w.N, w.D, w.seed)  # one batch row holds all heads
@@ -241,7 +249,11 @@ def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = Fa
     t0 = time.perf_counter()
     while True:
         h = done % w.Hq
-        if backward:
+        if backward and rope:
+            dq, dk, _ = head_backward(rope_rotate(q[0, h]), rope_rotate(k[0, h // g]), v[0, h // g], do[0, h],
+                                      w.causal, w.softmax_scale)
+            rope_rotate_transpose(dq), rope_rotate_transpose(dk)
+        elif backward:
             head_backward(q[0, h], k[0, h // g], v[0, h // g], do[0, h], w.causal, w.softmax_scale)
         elif rope:
             head_forward(rope_rotate(q[0, h]), rope_rotate(k[0, h // g]), v[0, h // g], w.causal, w.softmax_scale)
@@ -254,7 +266,7 @@ def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = Fa
         if heads is None and el >= seconds:
             break
     tflops = per_head * done / el / 1e12
-    what = "gradients" if backward else ("RoPE + forward" if rope else "forward")
+    what = ("gradients through RoPE" if rope else "gradients") if backward else ("RoPE + forward" if rope else "forward")
     sample = (f"{what} of {done} heads, cycling over the {w.Hq} query heads of one batch row of {w.name} "
               f"(each head's full {w.N}x{w.N} fp64 score matrix), {el:.1f} s")
     return tflops, per_head * done, el, done, sample
@@ -265,7 +277,8 @@ def time_oracle(w, seconds: float, heads: int | None = None, backward: bool = Fa
 def run_ours(args, w):
     import torch
 
-    backward = args.pass_ == "bwd"
+    backward = args.pass_ in ("bwd", "bwd_rope")
+    bwd_rope = args.pass_ == "bwd_rope"
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
@@ -290,12 +303,20 @@ def run_ours(args, w):
         # the backward consumes the forward's saved o and lse: computed once, untimed
         do = make_dout(w.B, w.Hq, w.N, w.D, rank_seed(w.seed + 500, rank))
         dod = do.to(device)
-        attn.forward(qd, kd, vd, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
         dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+        if bwd_rope:
+            cos_t, sin_t = attn.rope_tables(w.N, w.D, device=device)
+            attn.forward_rope(qd, kd, vd, cos_t, sin_t, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
 
-        def step():
-            attn.backward(qd, kd, vd, o, lse, dod, causal=w.causal, scale=scale, dq=dq, dk=dk, dv=dv,
-                          stream=stream)
+            def step():
+                attn.backward_rope(qd, kd, vd, cos_t, sin_t, o, lse, dod, causal=w.causal, scale=scale, dq=dq,
+                                   dk=dk, dv=dv, stream=stream)
+        else:
+            attn.forward(qd, kd, vd, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
+
+            def step():
+                attn.backward(qd, kd, vd, o, lse, dod, causal=w.causal, scale=scale, dq=dq, dk=dk, dv=dv,
+                              stream=stream)
     elif fp8:
         def step():
             attn.forward_fp8(qd, kd, vd, ds, ds, ds, causal=w.causal, scale=scale, out=o, lse=lse, stream=stream)
@@ -345,11 +366,12 @@ def run_ours(args, w):
 
         def e2e_call():
             attn.backward_from_host(*host_in, causal=w.causal, scale=scale, device=device, out_host=host_out,
-                                    stream=stream)
+                                    stream=stream, rope_tables=(cos_t, sin_t) if bwd_rope else None)
         h2d = sum(x.numel() * x.element_size() for x in host_in)
         d2h = sum(x.numel() * x.element_size() for x in host_out)
-        e2e_path = ("backward_from_host: pinned host q,k,v,o,lse,dO -> device, attn_bwd, "
-                    "dq,dk,dv -> pinned host; in 4 pieces (batch rows), copies overlapping the kernels")
+        e2e_path = ("backward_from_host: pinned host q,k,v,o,lse,dO -> device, "
+                    + ("attn_bwd_rope (device-resident cos/sin tables)" if bwd_rope else "attn_bwd")
+                    + ", dq,dk,dv -> pinned host; in 4 pieces (batch rows), copies overlapping the kernels")
     else:
         qh, kh, vh = (x.pin_memory() for x in (q, k, v))
         oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -423,6 +445,9 @@ def run_ours(args, w):
     if backward:
         kernel = (f"attn_bwd call: attn_bwd_prep + attn_bwd_sm100<{w.D}, dK/dV> + attn_bwd_sm100<{w.D}, dQ>, "
                   f"timed together")
+        if bwd_rope:
+            kernel = (f"attn_bwd_rope call: attn_rope_qk + attn_bwd_prep + attn_bwd_sm100<{w.D}, dK/dV> + "
+                      f"attn_bwd_sm100<{w.D}, dQ> + attn_rope_qk_inverse, timed together")
         # read q, o, dO (query heads), k, v (KV heads), lse; write dq, dk, dv; all bf16 but lse
         q_side = w.B * w.Hq * w.N * w.D * 2
         kv_side = w.B * w.Hkv * w.N * w.D * 2
@@ -447,7 +472,7 @@ def run_ours(args, w):
         algo_bytes = w.algorithmic_bytes
 
     line = {
-        "metric": {"fwd": METRIC, "bwd": METRIC_BWD, "rope": METRIC_ROPE, "fp8": METRIC_FP8}[args.pass_],
+        "metric": METRICS[args.pass_],
         "value": round(value, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -467,7 +492,7 @@ def run_ours(args, w):
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "path": e2e_path},
-        "gpu_launches": args.steps * {"fwd": 1, "bwd": 3, "rope": 2, "fp8": 1}[args.pass_],
+        "gpu_launches": args.steps * {"fwd": 1, "bwd": 3, "rope": 2, "fp8": 1, "bwd_rope": 5}[args.pass_],
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": f"{peak_kind} bf16 matmul, {peak_regime}",
@@ -486,7 +511,8 @@ def run_ours(args, w):
                                "algorithmic_bytes": rope_bytes, "kernel": "attn_rope_qk",
                                "peak_kind": "measured HBM copy bandwidth"}
     if world == 1 and not args.no_cpu_baseline:
-        tf, _, el, done, sample = time_oracle(w, CPU_SAMPLE_SECONDS, backward=backward, rope=args.pass_ == "rope")
+        tf, _, el, done, sample = time_oracle(w, CPU_SAMPLE_SECONDS, backward=backward,
+                                              rope=args.pass_ in ("rope", "bwd_rope"))
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                                 "sample": sample}
     if dist is not None:
@@ -500,10 +526,11 @@ def run_reference(args, w):
     world, rank, _ = dist_env()
     if rank != 0:
         return None
-    backward = args.pass_ == "bwd"
+    backward = args.pass_ in ("bwd", "bwd_rope")
     per_step = []
     for i in range(args.warmup + args.steps):
-        tf, flops, el, done, sample = time_oracle(w, 0.0, heads=1, backward=backward, rope=args.pass_ == "rope")
+        tf, flops, el, done, sample = time_oracle(w, 0.0, heads=1, backward=backward,
+                                                  rope=args.pass_ in ("rope", "bwd_rope"))
         if i >= args.warmup:
             per_step.append((flops, el))
     flops = sum(f for f, _ in per_step)
@@ -514,7 +541,7 @@ def run_reference(args, w):
     sample = f"{what} of {w.name} per step (full {w.N}x{w.N} fp64 score matrix), {args.steps} steps"
     return {
         "impl": "reference",
-        "metric": {"fwd": METRIC, "bwd": METRIC_BWD, "rope": METRIC_ROPE, "fp8": METRIC_FP8}[args.pass_],
+        "metric": METRICS[args.pass_],
         "value": value,
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -541,7 +568,7 @@ def main(argv=None):
                     help="cfg1..cfg4, a sweep point name (e.g. sweep_D128_N8192_causal), or 'all'")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "rope", "fp8"], default="fwd",
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "rope", "fp8", "bwd_rope"], default="fwd",
                     help="fwd: the attention forward (default); bwd: the backward pass (attn_bwd); "
                          "rope: RoPE of Q and K then the forward (attn_fwd_rope); fp8: the E4M3 forward "
                          "(attn_fwd_fp8)")

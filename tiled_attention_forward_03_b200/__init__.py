@@ -503,12 +503,14 @@ def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
 
 
 def backward_from_host(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None, device=None,
-                       out_host=None, stream=None, pieces: int = 4):
+                       out_host=None, stream=None, pieces: int = 4, rope_tables=None):
     """End-to-end backward on host (ideally pinned) tensors: copy q, k, v, o, lse and dout in,
     run attn_bwd, copy dq, dk, dv out.  Returns host tensors (dq, dk, dv); ``out_host`` may
     hold three preallocated host tensors for them.  Pipelined in up to ``pieces`` independent
     parts as forward_from_host (batch rows, or whole KV-head groups when B == 1, so that each
-    KV head's gradient is complete within one part).  Returns after the last download."""
+    KV head's gradient is complete within one part).  With ``rope_tables`` = (cos_t, sin_t)
+    (device tables from rope_tables()) the gradients are those through RoPE (backward_rope;
+    o and lse from forward_rope).  Returns after the last download."""
     import torch
 
     dev = torch.device(device if device is not None else "cuda")
@@ -527,8 +529,12 @@ def backward_from_host(q, k, v, o, lse, dout, causal: bool = False, scale: float
 
     def compute(pc):
         qd, kd, vd, od, ld, dd = (x[f(pc)] for x, f in zip(dev_in, in_idx))
-        backward(qd, kd, vd, od, ld, dd, causal=causal, scale=scale, dq=grads[0][qi(pc)], dk=grads[1][ki(pc)],
-                 dv=grads[2][ki(pc)], stream=s)
+        if rope_tables is not None:
+            backward_rope(qd, kd, vd, rope_tables[0], rope_tables[1], od, ld, dd, causal=causal, scale=scale,
+                          dq=grads[0][qi(pc)], dk=grads[1][ki(pc)], dv=grads[2][ki(pc)], stream=s)
+        else:
+            backward(qd, kd, vd, od, ld, dd, causal=causal, scale=scale, dq=grads[0][qi(pc)], dk=grads[1][ki(pc)],
+                     dv=grads[2][ki(pc)], stream=s)
 
     _pipelined(dev, s, _pieces(B, Hq, Hkv, pieces), list(zip(host_in, dev_in, in_idx)),
                list(zip(out_host, grads, (qi, ki, ki))), compute)
