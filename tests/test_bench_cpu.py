@@ -16,7 +16,7 @@ def run_bench(*args, timeout=600):
     return proc
 
 
-@pytest.mark.parametrize("pass_", ["fwd", "bwd", "rope", "fp8"])
+@pytest.mark.parametrize("pass_", ["fwd", "bwd", "rope", "fp8", "bwd_rope"])
 def test_reference_arm_prints_one_json_line(pass_):
     proc = run_bench("--impl", "reference", "--pass", pass_, "--workload", "cfg1", "--steps", "2", "--warmup", "3")
     assert proc.returncode == 0, proc.stderr
