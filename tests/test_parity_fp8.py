@@ -54,6 +54,9 @@ def assert_close(o, lse, o_ref, lse_ref, what):
 @pytest.mark.parametrize("B,Hq,Hkv,N,D,causal", [
     (1, 2, 2, 256, 128, False), (1, 2, 2, 256, 128, True), (1, 4, 1, 513, 128, True), (2, 2, 2, 384, 64, False),
     (1, 4, 2, 300, 64, True), (1, 2, 2, 1, 128, False), (1, 2, 1, 1000, 128, False), (1, 2, 2, 2048, 128, True),
+    # head dims 32 and 96 (one 128-byte row chunk, partly used and zero-filled by TMA)
+    (1, 2, 2, 512, 32, True), (2, 4, 2, 1000, 32, False), (1, 2, 2, 1, 32, True),
+    (1, 2, 2, 1024, 96, True), (1, 4, 1, 777, 96, False), (2, 2, 2, 2048, 96, False),
 ])
 def test_fp8_small_shapes(attn, B, Hq, Hkv, N, D, causal):
     q8, k8, v8, ds = make_qkv_e4m3(B, Hq, Hkv, N, D, 5000 + N + D)

@@ -87,7 +87,9 @@ bool device_setup(int dev, int* num_sms) {
     setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<128>), attn::CsPlan<128>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<32, false, true>), attn::SmemPlan<32>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, false, true>), attn::SmemPlan<64>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<32, true>), attn::SmemPlan<32, true>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, true>), attn::SmemPlan<64, true>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<96, true>), attn::SmemPlan<96, true>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<128, true>), attn::SmemPlan<128, true>::kAlloc);
     // the wide-head kernel has no register split: dynamic shared memory opt-in only
     if (e == cudaSuccess)
@@ -298,7 +300,7 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   // ---- host-side validation (no CUDA call before this block passes)
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
     return ATTN_ERR_INVALID_ARG;
-  if (!supported_head_dim(D) || (e4m3 && D != 64 && D != 128)) return ATTN_ERR_UNSUPPORTED;
+  if (!supported_head_dim(D) || (e4m3 && D > 128)) return ATTN_ERR_UNSUPPORTED;
   if (e4m3 && (!std::isfinite(qk_descale) || !std::isfinite(o_scale) || qk_descale == 0.f)) return ATTN_ERR_INVALID_ARG;
   if ((long long)B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   // the scheduler indexes work units (256 query rows of one head) in 32 bits
@@ -457,8 +459,14 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   CUtensorMap mo;
   if ((st = encode_map(&mo, o, (long long)B * Hq, N, D, 2)) != ATTN_OK) return st;
   if (e4m3) {
-    if (D == 64)
+    if (D == 32)
+      attn::attn_fwd_sm100<32, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32, true>::kAlloc, s>>>(
+          mq, mk, mv, mo, p);
+    else if (D == 64)
       attn::attn_fwd_sm100<64, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64, true>::kAlloc, s>>>(
+          mq, mk, mv, mo, p);
+    else if (D == 96)
+      attn::attn_fwd_sm100<96, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<96, true>::kAlloc, s>>>(
           mq, mk, mv, mo, p);
     else
       attn::attn_fwd_sm100<128, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<128, true>::kAlloc, s>>>(

@@ -94,7 +94,6 @@ __device__ unsigned int g_attn_fault_site = 0;
 template <int D, bool kF8 = false>
 struct SmemPlan {
   static_assert(D == 32 || D == 64 || D == 96 || D == 128, "head dim must be 32, 64, 96 or 128");
-  static_assert(!kF8 || D == 64 || D == 128, "E4M3 head dim must be 64 or 128");
   static constexpr int kElemBytes = kF8 ? 1 : 2;
   static constexpr int kRowElems = 128 / kElemBytes;        // columns per 128-byte swizzle row
   static constexpr int kChunks = (D + kRowElems - 1) / kRowElems;  // 128-byte swizzle chunks per row
