@@ -444,3 +444,48 @@ def test_host_buffer_entry_point(attn, B, Hq, Hkv, N, D, causal, pieces):
     torch.cuda.synchronize()
     assert torch.equal(od.cpu(), oh) and torch.equal(ld.cpu(), lh)
     assert attn.device_status() == (attn.ATTN_OK, 0)
+
+
+def test_calls_from_several_host_threads(attn):
+    """Four host threads, each on its own stream, call forward() (split last wave: a cached
+    workspace per stream) and backward() on different inputs, several times and at once; every
+    result equals the one computed beforehand on a single thread, bit for bit (the kernels are
+    deterministic).  (attn_fwd_noalloc is left out: its one static array must not be used by
+    kernels that overlap.)"""
+    import threading
+
+    B, Hq, Hkv, N, D = 2, 8, 4, 1100, 128        # non-causal: the last wave is split
+    cases = [make_qkv(B, Hq, Hkv, N, D, seed=7000 + i) for i in range(4)]
+    dev = [tuple(x.cuda() for x in c) for c in cases]
+    dos = [torch.randn(B, Hq, N, D, generator=torch.Generator().manual_seed(7100 + i)).to(torch.bfloat16).cuda()
+           for i in range(4)]
+    expect = []
+    for (q, k, v), do in zip(dev, dos):
+        o, lse = attn.forward(q, k, v, causal=False)
+        expect.append((o, lse, attn.backward(q, k, v, o, lse, do, causal=False)))
+    torch.cuda.synchronize()
+    errors = []
+
+    def worker(i):
+        try:
+            q, k, v = dev[i]
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                for _ in range(4):
+                    o, lse = attn.forward(q, k, v, causal=False, stream=s)
+                    grads = attn.backward(q, k, v, o, lse, dos[i], causal=False, stream=s)
+                    s.synchronize()
+                    eo, el, eg = expect[i]
+                    assert torch.equal(o, eo) and torch.equal(lse, el), f"thread {i}: forward differs"
+                    assert all(torch.equal(a, b) for a, b in zip(grads, eg)), f"thread {i}: backward differs"
+        except Exception as exc:   # reported by the main thread
+            errors.append(repr(exc))
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(4)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not any(t.is_alive() for t in threads), "a worker thread did not finish"
+    assert not errors, errors
+    assert attn.device_status() == (attn.ATTN_OK, 0)
