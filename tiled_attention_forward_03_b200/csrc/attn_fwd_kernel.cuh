@@ -12,7 +12,7 @@
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp  8    TMA producer: Q tiles once per unit, K_j / V_j through a smem ring
 //   warp  9    MMA issuer (one elected lane): S_t = Q_t K_j^T and O_t += P_t V_j on tcgen05
-//   warp  10   output store (bf16 D = 128): TMA tensor stores of each tile's O, staged in shared memory
+//   warp  10   output store (D = 128): TMA tensor stores of each tile's O, staged in shared memory
 //   warp  11   idle (completes the third warpgroup, which gives up registers)
 //
 // Non-causal bf16 D <= 64 (kSepP): P gets tensor-memory columns of its own beside O, and each
@@ -103,11 +103,11 @@ struct SmemPlan {
   static constexpr int kStages = (kChunks == 2) ? 4 : 8;    // K/V ring depth
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
-  // bf16 D = 128: one tile's O (bf16) staged for the TMA store: 64-column chunks of 128-byte rows,
-  // 128-byte swizzle, the two tiles using it in turn (measured 1-3 % faster than 16-byte stores
-  // from the softmax warps at D = 128, and 6-10 % slower at D = 64, where the softmax warps bound
-  // the kernel; other instances store O directly)
-  static constexpr bool kStagedStore = !kF8 && D == 128;
+  // D = 128: one tile's O (bf16) staged for the TMA store: 64-column chunks of 128-byte rows,
+  // 128-byte swizzle, the two tiles using it in turn (measured against 16-byte stores from the
+  // softmax warps: 1-3 % faster for bf16 and 5-8 % for E4M3 inputs at D = 128, 6-10 % slower for
+  // bf16 at D = 64, where the softmax warps bound the kernel; other instances store O directly)
+  static constexpr bool kStagedStore = D == 128;
   static constexpr int kOChunks = (D + 63) / 64;
   static constexpr int kOStageOff = kKVOff + kStages * kTileBytes;
   static constexpr int kBarOff = kOStageOff + (kStagedStore ? kOChunks * kChunkBytes : 0);
@@ -936,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __nv_bfloat16* orow = p.o + ((size_t)head_o * p.N + (row_ok ? row : 0)) * D;
       if (w.parts == 1 && Plan::kStagedStore) {
         // O / l -> bf16 pairs in registers; O's tensor memory is then free for the next unit.
-        const float inv_l = 1.f / l;
+        const float inv_l = (kF8 ? p.o_scale : 1.f) / l;
         uint32_t packed[D / 2];
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
