@@ -85,8 +85,8 @@ bool device_setup(int dev, int* num_sms) {
     setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<64>), attn::CsPlan<64>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<96>), attn::CsPlan<96>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_colsplit_sm100<128>), attn::CsPlan<128>::kAlloc);
-    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<32, false, true>), attn::SmemPlan<32>::kAlloc);
-    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, false, true>), attn::SmemPlan<64>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<32, false, true>), attn::SmemPlan<32, false, true>::kAlloc);
+    setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, false, true>), attn::SmemPlan<64, false, true>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<32, true>), attn::SmemPlan<32, true>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<64, true>), attn::SmemPlan<64, true>::kAlloc);
     setup(reinterpret_cast<const void*>(attn::attn_fwd_sm100<96, true>), attn::SmemPlan<96, true>::kAlloc);
@@ -476,14 +476,14 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
     // are short, and there it measured 0 to 8 % slower)
     case 32:
       if (!p.causal)
-        attn::attn_fwd_sm100<32, false, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32>::kAlloc, s>>>(
+        attn::attn_fwd_sm100<32, false, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32, false, true>::kAlloc, s>>>(
             mq, mk, mv, mo, p);
       else
         attn::attn_fwd_sm100<32><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<32>::kAlloc, s>>>(mq, mk, mv, mo, p);
       break;
     case 64:
       if (!p.causal)
-        attn::attn_fwd_sm100<64, false, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(
+        attn::attn_fwd_sm100<64, false, true><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64, false, true>::kAlloc, s>>>(
             mq, mk, mv, mo, p);
       else
         attn::attn_fwd_sm100<64><<<(unsigned)grid, attn::kThreads, attn::SmemPlan<64>::kAlloc, s>>>(mq, mk, mv, mo, p);

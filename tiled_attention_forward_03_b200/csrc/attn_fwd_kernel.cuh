@@ -91,7 +91,7 @@ enum : unsigned {
 __device__ unsigned int g_attn_fault_site = 0;
 
 // kF8: Q, K, V are E4M3 bytes (one 128-byte swizzle chunk holds 128 columns) instead of bf16.
-template <int D, bool kF8 = false>
+template <int D, bool kF8 = false, bool kSepP = false>
 struct SmemPlan {
   static_assert(D == 32 || D == 64 || D == 96 || D == 128, "head dim must be 32, 64, 96 or 128");
   static constexpr int kElemBytes = kF8 ? 1 : 2;
@@ -103,11 +103,13 @@ struct SmemPlan {
   static constexpr int kStages = (kChunks == 2) ? 4 : 8;    // K/V ring depth
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
-  // D = 128: one tile's O (bf16) staged for the TMA store: 64-column chunks of 128-byte rows,
-  // 128-byte swizzle, the two tiles using it in turn (measured against 16-byte stores from the
-  // softmax warps: 1-3 % faster for bf16 and 5-8 % for E4M3 inputs at D = 128, 6-10 % slower for
-  // bf16 at D = 64, where the softmax warps bound the kernel; other instances store O directly)
-  static constexpr bool kStagedStore = D == 128;
+  // D = 128, and bf16 D = 64 in the separate-P form: one tile's O (bf16) staged for the TMA
+  // store: 64-column chunks of 128-byte rows, 128-byte swizzle, the two tiles using it in turn
+  // (measured against 16-byte stores from the softmax warps: 1-3 % faster for bf16 and 5-8 % for
+  // E4M3 inputs at D = 128, 1-4 % in the separate-P form; 6-10 % slower for the bf16 D = 64 form
+  // with P in S, where the softmax warps bound the kernel, and up to 7 % slower for E4M3 at D = 64;
+  // the other instances store O directly)
+  static constexpr bool kStagedStore = D == 128 || (D == 64 && kSepP && !kF8);
   static constexpr int kOChunks = (D + 63) / 64;
   static constexpr int kOStageOff = kKVOff + kStages * kTileBytes;
   static constexpr int kBarOff = kOStageOff + (kStagedStore ? kOChunks * kChunkBytes : 0);
@@ -361,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
                    const FwdParams p) {
-  using Plan = SmemPlan<D, kF8>;
+  using Plan = SmemPlan<D, kF8, kSepP>;
   static_assert(!kSepP || (D <= 64 && !kF8), "P beside O needs D <= 64 (bf16)");
   // 32-byte K steps of the tensor-core instructions: 16 bf16 or 32 E4M3 elements each
   constexpr int kSSteps = D * Plan::kElemBytes / 32;
