@@ -456,7 +456,7 @@ def run_ours(args, w):
         kernel = f"attn_fwd_rope call: attn_rope_qk on Q and K + the forward kernel, timed together"
         algo_bytes = w.algorithmic_bytes
     elif fp8:
-        kernel = f"attn_fwd_sm100<{w.D}, E4M3>"
+        kernel = f"attn_fwd_sm100<{w.D}, E4M3>" if w.D <= 128 else f"attn_fwd_wide_sm100<{w.D}, E4M3>"
         # q, k, v one byte per element; o bf16, lse fp32
         algo_bytes = (w.B * w.Hq + 2 * w.B * w.Hkv) * w.N * w.D + 2 * w.B * w.Hq * w.N * w.D + 4 * w.B * w.Hq * w.N
         peak_burst = peak_burst * FP8_OVER_BF16

@@ -355,8 +355,10 @@ long long attn_bwd_rope_workspace_bytes(int B, int Hq, int Hkv, int N, int D);
  *                [B, Hq, N, D] / [B, Hkv, N, D], contiguous, 16-byte aligned.       read
  *   o, lse       bf16 [B, Hq, N, D] and fp32 [B, Hq, N], as attn_fwd.              written
  *   q_descale, k_descale, v_descale   per-tensor factors (finite; q and k non-zero).
- *   D            32, 64, 96 or 128 (ATTN_ERR_UNSUPPORTED otherwise).
- *   workspace, workspace_bytes   optional split-tail workspace, as attn_fwd_ws.
+ *   D            32, 64, 96, 128, 192 or 256 (ATTN_ERR_UNSUPPORTED otherwise; 192 and 256 run
+ *                on the wide-head kernel, one CTA per 128-row query tile, as attn_fwd does).
+ *   workspace, workspace_bytes   optional split-tail workspace, as attn_fwd_ws (never used at
+ *                D = 192 and 256).
  * Numerics: Q K^T on the E4M3 tensor cores (kind::f8f6f4) with fp32 accumulation; base-2 online
  * softmax in fp32; probabilities rounded to E4M3 (nearest even; p <= 2^8 by the lazy rescale,
  * inside E4M3's range) for P V, also E4M3 with fp32 accumulation; row sums of the fp32

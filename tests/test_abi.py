@@ -260,7 +260,7 @@ def call_fp8(**kw):
 @pytest.mark.parametrize("kw,expected", [
     (dict(q=None), INVALID), (dict(o=None), INVALID), (dict(qd=0.0), INVALID), (dict(kd=math.nan), INVALID),
     (dict(vd=math.inf), INVALID), (dict(scale=math.nan), INVALID), (dict(Hq=3, Hkv=2), INVALID),
-    (dict(D=192), UNSUPPORTED), (dict(D=80), UNSUPPORTED), (dict(D=256), UNSUPPORTED),
+    (dict(D=160), UNSUPPORTED), (dict(D=80), UNSUPPORTED), (dict(D=512), UNSUPPORTED),
     (dict(v=P + 8), MISALIGNED), (dict(ws=P + 64, nbytes=4096), MISALIGNED), (dict(ws=None, nbytes=64), INVALID),
 ])
 def test_fp8_rejected_before_any_cuda_call(kw, expected):

@@ -4,8 +4,8 @@ The oracle is the plain definition (attention_forward) on the dequantized inputs
 descale * stored value, which are exact in fp64.  The kernel's scores are exact fp32 sums of
 E4M3 products, so LSE keeps the forward's bound (max |dLSE| <= 1e-3); the probabilities are
 rounded to E4M3 (3 mantissa bits) before P V.  Tolerance (derived): emulating that rounding
-on the CPU (fp32 row sums, bf16 output) gives max |dO| up to 3.9e-2 (causal rows with few
-keys) and mean |dO| up to 2.2e-3 at N = 512..2048, D = 64/128; the bar is
+on the CPU (fp32 row sums, bf16 output) gives max |dO| up to 4e-2 (causal rows with few
+keys) and mean |dO| up to 2.2e-3 at N = 512..2048, D = 32..256; the bar is
 
     max |dO| <= 1e-1,   mean |dO| <= 6e-3,   max |dLSE| <= 1e-3.
 """
@@ -57,6 +57,9 @@ def assert_close(o, lse, o_ref, lse_ref, what):
     # head dims 32 and 96 (one 128-byte row chunk, partly used and zero-filled by TMA)
     (1, 2, 2, 512, 32, True), (2, 4, 2, 1000, 32, False), (1, 2, 2, 1, 32, True),
     (1, 2, 2, 1024, 96, True), (1, 4, 1, 777, 96, False), (2, 2, 2, 2048, 96, False),
+    # head dims 192 and 256 on the wide-head kernel (192: a second 128-byte chunk, half zero-filled)
+    (1, 2, 2, 256, 192, True), (1, 4, 1, 513, 192, False), (1, 2, 2, 1, 192, False), (2, 2, 2, 1000, 192, True),
+    (1, 2, 2, 384, 256, False), (1, 4, 2, 777, 256, True), (1, 2, 2, 1, 256, True), (1, 2, 2, 2048, 256, False),
 ])
 def test_fp8_small_shapes(attn, B, Hq, Hkv, N, D, causal):
     q8, k8, v8, ds = make_qkv_e4m3(B, Hq, Hkv, N, D, 5000 + N + D)
@@ -99,7 +102,8 @@ def test_fp8_cfg2_sampled(attn):
 
 
 @pytest.mark.parametrize("name", ["cfg3", "sweep_D128_N8192_noncausal", "sweep_D64_N4096_noncausal",
-                                  "sweep_D64_N4096_causal"])
+                                  "sweep_D64_N4096_causal", "wide_D192_N8192_noncausal", "wide_D256_N8192_noncausal",
+                                  "wide_D256_N8192_causal", "wide_D192_N2048_causal"])
 def test_fp8_benchmark_workloads_sampled(attn, name):
     """Every workload the E4M3 pass is benchmarked on, at full size: seeded sampled rows (every
     128-row tile edge of one head plus uniform draws), each computed by the oracle on its own

@@ -77,7 +77,8 @@ def emulate_fp8_head(q8, k8, v8, qd, kd, vd, causal, scale):
 
 
 FP8_SHAPES = [(512, 64, True), (1024, 128, True), (2048, 128, True), (2048, 128, False), (1024, 64, False),
-              (512, 32, True), (1024, 32, False), (1024, 96, True), (2048, 96, False)]
+              (512, 32, True), (1024, 32, False), (1024, 96, True), (2048, 96, False), (1024, 192, True),
+              (1024, 256, False)]
 
 
 @pytest.fixture(scope="module")

@@ -98,6 +98,12 @@ bool device_setup(int dev, int* num_sms) {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_fwd_wide_sm100<256>),
                                cudaFuncAttributeMaxDynamicSharedMemorySize, attn::WidePlan<256>::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_fwd_wide_sm100<192, true>),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, attn::WidePlan<192, true>::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_fwd_wide_sm100<256, true>),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, attn::WidePlan<256, true>::kAlloc);
     d.err = e;
     d.attrs_ok = (e == cudaSuccess);
     if (d.attrs_ok && !regs_ok) {
@@ -300,7 +306,7 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   // ---- host-side validation (no CUDA call before this block passes)
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0 || !std::isfinite(scale))
     return ATTN_ERR_INVALID_ARG;
-  if (!supported_head_dim(D) || (e4m3 && D > 128)) return ATTN_ERR_UNSUPPORTED;
+  if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
   if (e4m3 && (!std::isfinite(qk_descale) || !std::isfinite(o_scale) || qk_descale == 0.f)) return ATTN_ERR_INVALID_ARG;
   if ((long long)B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   // the scheduler indexes work units (256 query rows of one head) in 32 bits
@@ -337,12 +343,23 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
     wp.N = N;
     wp.num_blocks = (int)(((long long)N + attn::kBlockN - 1) / attn::kBlockN);
     wp.causal = causal ? 1 : 0;
-    wp.c = std::fmax(std::fabs(scale) * 1.44269504088896340736f, 1e-30f);
-    wp.idesc_s = attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, scale < 0.f);
-    wp.idesc_pv = attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
+    // (E4M3: the scores carry the product of the Q and K descales; its sign joins scale's.)
+    const float ws_eff = scale * qk_descale;
+    wp.c = std::fmax(std::fabs(ws_eff) * 1.44269504088896340736f, 1e-30f);
+    wp.o_scale = o_scale;
+    wp.idesc_s = e4m3 ? attn::idesc_e4m3_f32(attn::kBlockM, attn::kBlockN, false, false, ws_eff < 0.f)
+                      : attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, ws_eff < 0.f);
+    wp.idesc_pv = e4m3 ? attn::idesc_e4m3_f32(attn::kBlockM, D, false, true, false)
+                       : attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
     const long long grid = (long long)B * Hq * wp.num_blocks;
     if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-    if (D == 192)
+    if (e4m3 && D == 192)
+      attn::attn_fwd_wide_sm100<192, true><<<(unsigned)grid, attn::kWideThreads, attn::WidePlan<192, true>::kAlloc,
+                                             s>>>(mq, mk, mv, wp);
+    else if (e4m3)
+      attn::attn_fwd_wide_sm100<256, true><<<(unsigned)grid, attn::kWideThreads, attn::WidePlan<256, true>::kAlloc,
+                                             s>>>(mq, mk, mv, wp);
+    else if (D == 192)
       attn::attn_fwd_wide_sm100<192><<<(unsigned)grid, attn::kWideThreads, attn::WidePlan<192>::kAlloc, s>>>(
           mq, mk, mv, wp);
     else

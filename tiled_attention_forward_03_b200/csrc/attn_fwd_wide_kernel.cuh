@@ -20,6 +20,11 @@
 //   warps 6-7  idle
 // One CTA per 128-row Q tile (grid = B * Hq * ceil(N/128)), heaviest tiles first when causal.
 // Every wait is bounded, as in the other kernels.
+//
+// kF8: Q, K, V are E4M3 bytes with per-tensor descales, as in the narrow kernel's E4M3 form:
+// 128-byte swizzle rows hold 128 columns (D = 192 uses a second chunk half zero-filled by TMA),
+// the MMAs are kind::f8f6f4 with K = 32 per instruction, P is packed four E4M3 values per TMEM
+// column, the Q and K descales join the exponent constant and the V descale joins 1/l.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -36,13 +41,15 @@ enum : unsigned {
   kSiteWideSoftmax = 23,
 };
 
-template <int D>
+template <int D, bool kF8 = false>
 struct WidePlan {
   static_assert(D == 192 || D == 256, "wide head dim must be 192 or 256");
-  static constexpr int kChunks = D / 64;                 // 64-column (128 B) swizzle chunks per row
+  static constexpr int kElemBytes = kF8 ? 1 : 2;
+  static constexpr int kRowElems = 128 / kElemBytes;     // columns per 128-byte swizzle row
+  static constexpr int kChunks = (D + kRowElems - 1) / kRowElems;  // 128 B swizzle chunks per row
   static constexpr int kChunkBytes = kBlockM * 128;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = D == 256 ? 2 : 3;       // K/V ring depth (tiles)
+  static constexpr int kStages = kF8 ? 4 : (D == 256 ? 2 : 3);  // K/V ring depth (tiles)
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
@@ -59,17 +66,21 @@ struct WideParams {
   float* lse;
   int Hq, group, N, num_blocks;
   int causal;
-  float c;            // |scale| * log2(e)
+  float c;            // |scale| * log2(e) (E4M3: times the Q and K descales)
+  float o_scale;      // E4M3: the V descale (1 for bf16)
   uint32_t idesc_s;   // 128 x 128 x D
   uint32_t idesc_pv;  // 128 x D x 128
 };
 
-template <int D>
+template <int D, bool kF8 = false>
 __global__ void __launch_bounds__(kWideThreads, 1)
     attn_fwd_wide_sm100(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const WideParams p) {
-  using Plan = WidePlan<D>;
+  using Plan = WidePlan<D, kF8>;
   constexpr int S = Plan::kStages;
+  constexpr int kSSteps = D * Plan::kElemBytes / 32;                 // 32-byte K steps of S = Q K^T
+  constexpr int kPVSteps = kBlockN * Plan::kElemBytes / 32;          // 32-byte K steps of P V
+  constexpr uint32_t kPVStepBytes = (32 / Plan::kElemBytes) * 128;   // K rows of V per step x 128 B
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -136,7 +147,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int row, int head, uint64_t pol) {
 #pragma unroll
         for (int ch = 0; ch < Plan::kChunks; ++ch)
-          tma_load_3d(dst + ch * Plan::kChunkBytes, map, bar, ch * 64, row, head, pol);
+          tma_load_3d(dst + ch * Plan::kChunkBytes, map, bar, ch * Plan::kRowElems, row, head, pol);
       };
       mbar_arrive_expect_tx(q_full, Plan::kTileBytes);
       load_tile(&tmap_q, sQ, q_full, qt * kBlockM, head_q, pol_q);
@@ -202,9 +213,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       const uint64_t db = adv(desc_k, st * Plan::kTileBytes);
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < kSSteps; ++kk) {
           const uint32_t off = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
-          mma_ss(tmem + b * 128, adv(desc_q, off), adv(db, off), p.idesc_s, kk > 0 ? 1u : 0u);
+          if constexpr (kF8)
+            mma_ss_f8(tmem + b * 128, adv(desc_q, off), adv(db, off), p.idesc_s, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tmem + b * 128, adv(desc_q, off), adv(db, off), p.idesc_s, kk > 0 ? 1u : 0u);
         }
       }
       __syncwarp();
@@ -213,8 +227,14 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       const uint64_t dv = adv(desc_v, st * Plan::kTileBytes);
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk)
-          mma_ts(tmem + 256, tmem + b * 128 + kk * 8, adv(dv, kk * 2048), p.idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kPVSteps; ++kk) {
+          if constexpr (kF8)
+            mma_ts_f8(tmem + 256, tmem + b * 128 + kk * 8, adv(dv, kk * kPVStepBytes), p.idesc_pv,
+                      (accumulate || kk > 0) ? 1u : 0u);
+          else
+            mma_ts(tmem + 256, tmem + b * 128 + kk * 8, adv(dv, kk * kPVStepBytes), p.idesc_pv,
+                   (accumulate || kk > 0) ? 1u : 0u);
+        }
       }
       __syncwarp();
     };
@@ -341,7 +361,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           tmem_st32(t_o + ch * 32, ov);
         }
       }
-      // P = 2^(s c - m) -> bf16 pairs over the first 64 columns of S; row sum in fp32.
+      // P = 2^(s c - m) -> bf16 pairs over the first 64 columns of S (E4M3: four per column over
+      // the first 32); row sum in fp32.
       {
         const float2 c2 = make_float2(c, c);
         const float2 nm2 = make_float2(-m, -m);
@@ -350,6 +371,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
+          float prev = 0.f, prev2 = 0.f;  // E4M3: the first pair of a group of four
 #pragma unroll
           for (int i = 0; i < 64; i += 2) {
             const int col = half * 64 + i;
@@ -362,9 +384,25 @@ __global__ void __launch_bounds__(kWideThreads, 1)
               pr.y = ex2_approx(x.y);
             }
             acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], pr);
-            pk[i >> 1] = pack_bf16x2(pr.x, pr.y);
+            if constexpr (kF8) {
+              if ((i & 2) == 0) {
+                prev = pr.x;
+                prev2 = pr.y;
+              } else {
+                pk[i >> 2] = pack_e4m3x4(prev, prev2, pr.x, pr.y);
+              }
+            } else {
+              pk[i >> 1] = pack_bf16x2(pr.x, pr.y);
+            }
           }
-          tmem_st32(t_s + half * 32, pk);
+          if constexpr (kF8) {
+            uint32_t pk16[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk16[i] = pk[i];
+            tmem_st16(t_s + half * 16, pk16);
+          } else {
+            tmem_st32(t_s + half * 32, pk);
+          }
         }
         const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
         l += a.x + a.y;
@@ -378,7 +416,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       tc_fence_after();
       const bool row_ok = row < p.N;
       __nv_bfloat16* orow = p.o + ((size_t)head_q * p.N + (row_ok ? row : 0)) * D;
-      const float inv_l = 1.f / l;
+      const float inv_l = (kF8 ? p.o_scale : 1.f) / l;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t ov[32];
