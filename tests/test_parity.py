@@ -247,6 +247,27 @@ def test_large_magnitude_inputs(attn):
     check_full(attn, q, k, v, True, 0.125, "large magnitude")
 
 
+@pytest.mark.parametrize("D,N,causal", [(32, 300, False), (64, 300, False), (64, 300, True), (96, 300, False),
+                                        (128, 300, True), (128, 300, False), (128, 2200, True), (192, 300, True),
+                                        (256, 300, False)])
+def test_one_dominant_key_per_row_at_every_column(attn, D, N, causal):
+    """Row i's query is a * e_(i mod D) and key k's component k mod D is a, so row i's largest
+    scores (all equal, ~300 above the others in log2 units) sit at the keys congruent to i modulo
+    D.  Across a tile's rows every column of a key block then holds some row's maximum: a row
+    maximum that skipped a column would leave 2^300 in that row's sum and a non-finite output.
+    Covers the two-tile kernel (P over S and P beside O), the column-split and the wide kernels."""
+    _, k, v = make_qkv(1, 2, 1, N, D, seed=4100 + N + D)
+    scale = 1.0 / math.sqrt(D)
+    a = float(torch.tensor(math.sqrt(300.0 / (scale * math.log2(math.e)))).to(torch.bfloat16))
+    idx = torch.arange(N)
+    qf = torch.zeros(1, 2, N, D)
+    qf[:, :, idx, idx % D] = a
+    kf = k.float().clone()
+    kf[:, :, idx, idx % D] = a
+    q, k = qf.to(torch.bfloat16), kf.to(torch.bfloat16)
+    check_full(attn, q, k, v, causal, scale, f"dominant keys D{D} N{N} causal={causal}")
+
+
 # ------------------------------------------------------------------ invariants on the GPU path
 
 def test_identical_v_rows_give_that_row(attn):

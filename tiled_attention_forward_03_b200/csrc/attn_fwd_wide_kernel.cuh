@@ -333,10 +333,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) mx[e] = max3f(s[e], s[4 + e], s[8 + e]);
 #pragma unroll
-      for (int i = 12; i < kBlockN; i += 8) {
+      for (int i = 12; i < kBlockN - 4; i += 8) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[i + e], s[i + 4 + e]);
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx[e] = fmaxf(mx[e], s[kBlockN - 4 + e]);
       const float m_new = fmaxf(m, fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]) * c);
       // Lazy rescale (as in the narrow kernel): the running max moves only when the row's
       // maximum grew by more than kRescaleLog2, and O (holding blocks < j once P(j-1) V has
