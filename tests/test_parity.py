@@ -209,6 +209,37 @@ def test_head_dims_192_and_256(attn, shape):
     check_full(attn, q, k, v, causal, 1.0 / math.sqrt(D), str(shape))
 
 
+WIDE_PERSISTENT = [
+    # (B, Hq, Hkv, N, D, causal): the wide-head kernel's persistent CTAs walking many items
+    (8, 16, 16, 2176, 192, True),    # causal tile pairs, 17 tiles per head: the middle tile is an item alone
+    (4, 20, 4, 2048, 256, True),     # causal tile pairs, GQA group 5
+    (10, 16, 16, 1920, 256, False),  # non-causal, 15 tiles per head, ~16 tiles per CTA
+    (1, 6, 2, 1500, 192, True),      # causal, fewer pairs than SMs: single tiles, heaviest first
+]
+
+
+@pytest.mark.parametrize("shape", WIDE_PERSISTENT, ids=lambda s: "B{}_Hq{}_Hkv{}_N{}_D{}_{}".format(*s[:5], "c" if s[5] else "nc"))
+def test_wide_persistent_items_sampled(attn, shape):
+    """Every item kind of the wide-head kernel's schedule, at sizes where CTAs take many items:
+    rows on both sides of the first, middle and last tiles' edges of the first and last heads,
+    plus seeded draws, each computed by the oracle on its own."""
+    B, Hq, Hkv, N, D, causal = shape
+    w = Workload(f"widep_B{B}_Hq{Hq}_N{N}_D{D}", B, Hq, Hkv, N, D, causal, 4200 + N + D)
+    q, k, v = make_workload_inputs(w)
+    T = -(-N // 128)
+    rows = set()
+    for b, h in ((0, 0), (B - 1, Hq - 1)):
+        for t in (0, T // 2, T - 1):
+            for i in (t * 128 - 1, t * 128, t * 128 + 127):
+                if 0 <= i < N:
+                    rows.add((b, h, i))
+    g = np.random.default_rng(w.seed)
+    for x in g.integers(0, B * Hq * N, 64):
+        b, rem = divmod(int(x), Hq * N)
+        rows.add((b, rem // N, rem % N))
+    check_sampled(attn, w, q, k, v, full_heads=(), rows=sorted(rows))
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_wide_head_dim_rescale_and_scales(attn, causal):
     """D = 256 with keys whose norm grows along the sequence (the lazy O rescale runs between

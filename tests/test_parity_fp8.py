@@ -101,6 +101,22 @@ def test_fp8_cfg2_sampled(attn):
     assert_close(o[idx], lse[idx], o_ref, lse_ref, "fp8 cfg2 sampled rows")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,causal", [(8, 16, 16, 2176, 256, True), (10, 16, 16, 1920, 192, False)])
+def test_fp8_wide_persistent_items_sampled(attn, B, Hq, Hkv, N, D, causal):
+    """The wide-head kernel's persistent schedule with E4M3 inputs (causal tile pairs with a
+    lone middle tile; non-causal, many tiles per CTA): seeded sampled rows."""
+    from attn_inputs import sample_rows
+
+    q8, k8, v8, ds = make_qkv_e4m3(B, Hq, Hkv, N, D, 5300 + N + D)
+    scale = D ** -0.5
+    o, lse = run(attn, q8, k8, v8, ds, causal, scale)
+    rows = sample_rows(B, Hq, N, 96, seed=5301 + N)
+    q, k, v = (x.float() * ds for x in (q8, k8, v8))
+    o_ref, lse_ref = attention_rows(q, k, v, rows, causal, scale)
+    idx = tuple(np.array(x) for x in zip(*rows))
+    assert_close(o[idx], lse[idx], o_ref, lse_ref, f"fp8 wide persistent B{B} N{N} D{D}")
+
+
 @pytest.mark.parametrize("name", ["cfg3", "sweep_D128_N8192_noncausal", "sweep_D64_N4096_noncausal",
                                   "sweep_D64_N4096_causal", "wide_D192_N8192_noncausal", "wide_D256_N8192_noncausal",
                                   "wide_D256_N8192_causal", "wide_D192_N2048_causal"])

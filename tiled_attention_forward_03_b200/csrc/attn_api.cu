@@ -351,8 +351,18 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
                       : attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, ws_eff < 0.f);
     wp.idesc_pv = e4m3 ? attn::idesc_e4m3_f32(attn::kBlockM, D, false, true, false)
                        : attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
-    const long long grid = (long long)B * Hq * wp.num_blocks;
-    if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    const long long tiles = (long long)B * Hq * wp.num_blocks;
+    if (tiles > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    // Work items: causal, a head's heaviest and lightest tiles together (equal items) when
+    // there are enough of them to fill the GPU, else single tiles.  CTAs are persistent for
+    // causal shapes and for N <= 2048 (one CTA per SM walking the items: the next tile's Q
+    // load and first scores overlap the current tile's last blocks and epilogue); longer
+    // non-causal shapes take one CTA per tile, which measured up to 2 % faster there.
+    const long long pairs = (long long)B * Hq * ((wp.num_blocks + 1) / 2);
+    wp.pair = (causal && pairs >= num_sms) ? 1 : 0;
+    wp.num_items = (int)(wp.pair ? pairs : tiles);
+    const bool persistent = causal || wp.num_blocks <= 16;
+    const long long grid = (persistent && wp.num_items > num_sms) ? num_sms : wp.num_items;
     if (e4m3 && D == 192)
       attn::attn_fwd_wide_sm100<192, true><<<(unsigned)grid, attn::kWideThreads, attn::WidePlan<192, true>::kAlloc,
                                              s>>>(mq, mk, mv, wp);
