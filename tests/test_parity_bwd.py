@@ -24,7 +24,7 @@ import pytest
 import torch
 
 from oracle import attention_backward, head_backward
-from attn_inputs import CFG2, CFG3, CFG4, make_dout, make_qkv
+from attn_inputs import Workload, CFG2, CFG3, CFG4, make_dout, make_qkv
 
 pytestmark = pytest.mark.gpu
 
@@ -187,6 +187,23 @@ def test_backward_sweep_benchmark_shapes_sampled_heads(attn, name, heads):
     """The other workloads the backward is benchmarked on, at full size: whole KV heads."""
     from attn_inputs import get_workload
     check_heads(attn, get_workload(name), heads)
+
+
+BWD_PERSISTENT = [
+    # (B, Hq, Hkv, N, D, causal): the persistent schedule's item kinds at sizes where CTAs take
+    # many units: causal block pairs with 17 blocks per head (a lone middle block); GQA group 5
+    # with the dK/dV pass unpaired (fewer pairs than SMs) and the dQ pass paired; non-causal with
+    # ~13 units per CTA
+    (8, 16, 16, 2176, 128, True),
+    (4, 20, 4, 2048, 64, True),
+    (8, 16, 16, 1920, 96, False),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,causal", BWD_PERSISTENT)
+def test_backward_persistent_items_sampled_heads(attn, B, Hq, Hkv, N, D, causal):
+    w = Workload(f"bwdp_B{B}_Hq{Hq}_Hkv{Hkv}_N{N}_D{D}", B, Hq, Hkv, N, D, causal, 4700 + N + D)
+    check_heads(attn, w, [(0, 0), (B - 1, Hkv - 1)])
 
 
 @pytest.mark.parametrize("B,Hq,Hkv", [(3, 4, 2), (1, 8, 2)])

@@ -723,11 +723,12 @@ size_t bwd_part_bytes(long long B, int Hq, int N) {
 
 template <int D>
 void launch_bwd_dim(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                    const attn::BwdParams& p, long long grid_kv, long long grid_q, cudaStream_t s) {
+                    const attn::BwdParams& pkv, const attn::BwdParams& pq, long long grid_kv, long long grid_q,
+                    cudaStream_t s) {
   attn::attn_bwd_sm100<D, true><<<(unsigned)grid_kv, attn::kBwdThreads, attn::BwdPlan<D, true>::kAlloc, s>>>(
-      mk, mv, mq, mdo, p);
+      mk, mv, mq, mdo, pkv);
   attn::attn_bwd_sm100<D, false><<<(unsigned)grid_q, attn::kBwdThreads, attn::BwdPlan<D, false>::kAlloc, s>>>(
-      mq, mdo, mk, mv, p);
+      mq, mdo, mk, mv, pq);
 }
 
 }  // namespace
@@ -802,12 +803,28 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   attn::attn_bwd_prep<<<(unsigned)prep_blocks, prep_threads, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), lse, nlse2, ndelta,
       rows, N, p.Npad, D);
-  const long long grid_kv = (long long)B * Hkv * nb, grid_q = (long long)B * Hq * nb;
+  // Persistent CTAs (at most one per SM) walk each pass's units, 128-row blocks of a head;
+  // causal units pair a head's heaviest and lightest blocks (equal items) when there are at
+  // least as many pairs as SMs.
+  int num_sms = 0;
+  e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess || num_sms < 1) {
+    record_cuda_error("cudaDeviceGetAttribute", e);
+    return ATTN_ERR_CUDA;
+  }
+  attn::BwdParams pkv = p, pq = p;
+  auto plan_pass = [&](attn::BwdParams& pp, long long heads) -> long long {
+    const long long units = heads * nb, pairs = heads * ((nb + 1) / 2);
+    pp.pair = (causal && pairs >= num_sms) ? 1 : 0;
+    pp.num_items = (int)(pp.pair ? pairs : units);
+    return pp.num_items > num_sms ? num_sms : pp.num_items;
+  };
+  const long long grid_kv = plan_pass(pkv, (long long)B * Hkv), grid_q = plan_pass(pq, (long long)B * Hq);
   switch (D) {
-    case 32: launch_bwd_dim<32>(mq, mk, mv, mdo, p, grid_kv, grid_q, s); break;
-    case 64: launch_bwd_dim<64>(mq, mk, mv, mdo, p, grid_kv, grid_q, s); break;
-    case 96: launch_bwd_dim<96>(mq, mk, mv, mdo, p, grid_kv, grid_q, s); break;
-    default: launch_bwd_dim<128>(mq, mk, mv, mdo, p, grid_kv, grid_q, s); break;
+    case 32: launch_bwd_dim<32>(mq, mk, mv, mdo, pkv, pq, grid_kv, grid_q, s); break;
+    case 64: launch_bwd_dim<64>(mq, mk, mv, mdo, pkv, pq, grid_kv, grid_q, s); break;
+    case 96: launch_bwd_dim<96>(mq, mk, mv, mdo, pkv, pq, grid_kv, grid_q, s); break;
+    default: launch_bwd_dim<128>(mq, mk, mv, mdo, pkv, pq, grid_kv, grid_q, s); break;
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) {

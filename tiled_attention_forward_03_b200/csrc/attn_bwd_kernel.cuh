@@ -15,13 +15,20 @@
 // Three launches:
 //   attn_bwd_prep   delta and LSE * log2(e) per query row, into a workspace padded to
 //                   whole 128-row tiles (pad rows hold 0)
-//   attn_bwd_sm100<D, kKV = true>   one CTA per 128-key block of a KV head: keeps K_j, V_j
+//   attn_bwd_sm100<D, kKV = true>   units of one 128-key block of a KV head: keeps K_j, V_j
 //                   in shared memory, streams the Q/dO tiles of every query head of the
 //                   group, accumulates dV_j and dK_j in tensor memory
-//   attn_bwd_sm100<D, kKV = false>  one CTA per 128-query block: keeps Q_i, dO_i, streams
+//   attn_bwd_sm100<D, kKV = false>  units of one 128-query block: keeps Q_i, dO_i, streams
 //                   the K/V tiles, accumulates dQ_i in tensor memory
-// Each CTA owns its output rows outright, so there are no atomics and the result does
-// not depend on the order CTAs run in.  The price is that the score and dP tiles are
+// Each unit owns its output rows outright, so there are no atomics and the result does
+// not depend on the order units run in.
+//
+// Persistent CTAs (at most one per SM) walk the work items with a stride of the grid; an item
+// is a unit or, causal with enough of them, a head's heaviest and lightest remaining blocks
+// (equal items).  Between units the row tiles are reloaded once the last S and dP of the
+// previous unit have read them (r_empty), the next unit's first S and dP run while the softmax
+// warps store the previous unit's gradients, and the first accumulating MMAs wait until those
+// are read (acc_free).  Per-tile barrier phases count the tiles of all units.  The price is that the score and dP tiles are
 // computed by both kernels (7 tile matmuls per (query block, key block) instead of 5).
 //
 // One kernel serves both passes.  In its own terms a CTA has "row" tiles R0, R1
@@ -113,8 +120,8 @@ struct BwdPlan {
   static constexpr int kVecOff = kC1Off + kStages1 * kTileBytes;
   static constexpr int kBarOff = kVecOff + kStages0 * kVecBytes;
   // r_full c0_full[S0] c0_empty[S0] c1_full[S1] c1_empty[S1] s_full s_free dp_full[2] p_ready
-  // ds_ready acc_full drain
-  static constexpr int kNumBars = 1 + 2 * kStages0 + 2 * kStages1 + 8;
+  // ds_ready acc_full drain r_empty acc_free
+  static constexpr int kNumBars = 1 + 2 * kStages0 + 2 * kStages1 + 10;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -132,6 +139,8 @@ struct BwdParams {
   float scale;
   uint32_t idesc_s;     // 128 x 128 x D, both operands K-major
   uint32_t idesc_acc;   // 128 x D x 128, A from TMEM, B MN-major
+  int pair;             // causal: an item is a row head's heaviest and lightest remaining row blocks
+  int num_items;        // items of the pass being launched
 };
 
 // -delta_i = -sum_d dO_id O_id (fp32 sums of the bf16 products) and -lse2_i = -LSE_i log2(e)
@@ -197,13 +206,25 @@ struct BwdUnit {
   int c0;         // first column block
 };
 
+// Unit `which` (0 or 1) of work item `item`; false if the item has no such unit.  Items are
+// numbered row head by row head; a causal item pairs the heaviest and the lightest remaining
+// row blocks of a head (equal items) when p.pair is set, else an item is one row block,
+// heaviest first.
 template <bool kKV>
-__device__ __forceinline__ BwdUnit bwd_unit(const BwdParams& p) {
-  BwdUnit w;
+__device__ __forceinline__ bool bwd_unit(const BwdParams& p, int item, int which, BwdUnit& w) {
   const int nb = p.num_blocks;
-  const long long u = blockIdx.x;
-  w.row_head = (int)(u / nb);
-  const int k = (int)(u - (long long)w.row_head * nb);
+  int k;
+  if (p.pair) {
+    const int sph = (nb + 1) >> 1;
+    w.row_head = item / sph;
+    const int s = item - w.row_head * sph;
+    if (which == 1 && s >= nb - 1 - s) return false;
+    k = which ? nb - 1 - s : s;   // k = 0 is the heaviest block in both passes
+  } else {
+    if (which) return false;
+    w.row_head = item / nb;
+    k = item - w.row_head * nb;
+  }
   if (kKV) {
     // key block rb sees query blocks rb..nb-1 (causal): heaviest (rb = 0) first
     w.rb = k;
@@ -217,7 +238,7 @@ __device__ __forceinline__ BwdUnit bwd_unit(const BwdParams& p) {
     w.cpb = p.causal ? w.rb + 1 : nb;
     w.n = w.cpb;
   }
-  return w;
+  return true;
 }
 
 // Column tile `it` of a unit: its block index and head.
@@ -262,6 +283,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* ds_ready = s_full + 5;
   uint64_t* acc_full = s_full + 6;
   uint64_t* drain = s_full + 7;
+  uint64_t* r_empty = s_full + 8;    // the unit's last S and dP have read R0, R1
+  uint64_t* acc_free = s_full + 9;   // the epilogue has read the accumulators (256 arrivals)
   // At D <= 64 tensor memory has room for a second dP buffer (S 128 + dP 2 x 128 + two
   // accumulators of D <= 64 columns): dP(t+1) then goes into the other buffer as soon as S(t+1)
   // is issued, instead of waiting for the MMAs that read P(t) and dS(t).
@@ -276,7 +299,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const BwdUnit w = bwd_unit<kKV>(p);
 
   if (threadIdx.x == 0) {
     mbar_init(r_full, 1);
@@ -296,6 +318,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(ds_ready, 256);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
+    mbar_init(r_empty, 1);
+    mbar_init(acc_free, 256);
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -326,15 +350,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int ch = 0; ch < Plan::kChunks; ++ch)
           tma_load_3d(dst + ch * Plan::kChunkBytes, map, bar, ch * 64, row, head, pol);
       };
+      Ring r0, r1;
+      uint32_t filled0 = 0u, par0 = 0u, filled1 = 0u, par1 = 0u;  // per stage: ever filled / parity of last fill
+      uint32_t units = 0u;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x)
+      for (int which = 0; which < 2 && ok; ++which) {
+      BwdUnit w;
+      if (!bwd_unit<kKV>(p, item, which, w)) continue;
+      // the row tiles once the previous unit's last S and dP have read them
+      if (units > 0u && !(ok = wait_phase(r_empty, (units - 1u) & 1u, abort_flag, kSiteBwdProducer))) break;
       mbar_arrive_expect_tx(r_full, 2 * Plan::kTileBytes);
       load_tile(&tmap_r0, sR, r_full, w.rb * kBlockM, w.row_head, pol_once);
       load_tile(&tmap_r1, sR + Plan::kTileBytes, r_full, w.rb * kBlockM, w.row_head, pol_once);
-      Ring r0, r1;
-      uint32_t filled0 = 0u, par0 = 0u, filled1 = 0u, par1 = 0u;  // per stage: ever filled / parity of last fill
+      ++units;
       for (int it = 0; it < w.n; ++it) {
         int cb, chead;
         bwd_col<kKV>(p, w, it, cb, chead);
-        if (!wait_phase(&c0_empty[r0.stage], r0.phase ^ 1u, abort_flag, kSiteBwdProducer)) break;
+        if (!(ok = wait_phase(&c0_empty[r0.stage], r0.phase ^ 1u, abort_flag, kSiteBwdProducer))) break;
         uint64_t* bar0 = &c0_full[r0.stage];
         mbar_arrive_expect_tx(bar0, Plan::kTileBytes + Plan::kVecBytes);
         load_tile(&tmap_c0, sC0 + r0.stage * Plan::kTileBytes, bar0, cb * kBlockN, chead, pol_shared);
@@ -347,7 +380,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         filled0 |= 1u << r0.stage;
         par0 = (par0 & ~(1u << r0.stage)) | (r0.phase << r0.stage);
         r0.advance<S0>();
-        if (!wait_phase(&c1_empty[r1.stage], r1.phase ^ 1u, abort_flag, kSiteBwdProducer)) break;
+        if (!(ok = wait_phase(&c1_empty[r1.stage], r1.phase ^ 1u, abort_flag, kSiteBwdProducer))) break;
         uint64_t* bar1 = &c1_full[r1.stage];
         mbar_arrive_expect_tx(bar1, Plan::kTileBytes);
         load_tile(&tmap_c1, sC1 + r1.stage * Plan::kTileBytes, bar1, cb * kBlockN, chead, pol_shared);
@@ -355,8 +388,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         par1 = (par1 & ~(1u << r1.stage)) | (r1.phase << r1.stage);
         r1.advance<S1>();
       }
+      }
       // Drain: every issued copy lands before the CTA may exit.
-      drain_phase(r_full, 0u, abort_flag);
+      if (units > 0u) drain_phase(r_full, (units - 1u) & 1u, abort_flag);
       for (int s = 0; s < S0; ++s)
         if (filled0 & (1u << s)) drain_phase(&c0_full[s], (par0 >> s) & 1u, abort_flag);
       for (int s = 0; s < S1; ++s)
@@ -411,23 +445,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     };
     auto st_bytes = [](uint32_t st) -> uint32_t { return st * Plan::kTileBytes; };
 
-    bool ok = wait_all(r_full, 0u, kSiteBwdMmaRow);
     Ring r0, r1;  // ring positions of the current tile's C0 and C1
-    if (ok && w.n > 0) ok = wait_all(&c0_full[0], 0u, kSiteBwdMmaCol);
-    if (ok && w.n > 0) {
-      tc_fence_after();
-      issue_rc(0, desc_r0, desc_c0_k);
-      commit(s_full);
-      ok = wait_all(&c1_full[0], 0u, kSiteBwdMmaCol);
-    }
-    if (ok && w.n > 0) {
-      tc_fence_after();
-      issue_rc(dp_col(0), desc_r1, desc_c1_k);
-      commit(&dp_full[dp_bar(0)]);
-      if (!kKV) commit(&c1_empty[0]);
-    }
+    uint32_t T = 0u;      // column tiles of earlier units: tile it of this unit is T + it
+    uint32_t units = 0u;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x)
+    for (int which = 0; which < 2 && ok; ++which) {
+    BwdUnit w;
+    if (!bwd_unit<kKV>(p, item, which, w)) continue;
+    if (!(ok = wait_all(r_full, units & 1u, kSiteBwdMmaRow))) break;
+    // First tile's S and dP.  S's columns were read by the softmax (s_free of the previous unit's
+    // last tile was waited for); dP's buffer was last read by MMAs issued before these.
+    if (!(ok = wait_all(&c0_full[r0.stage], r0.phase, kSiteBwdMmaCol))) break;
+    tc_fence_after();
+    issue_rc(0, desc_r0, adv(desc_c0_k, st_bytes(r0.stage)));
+    commit(s_full);
+    if (!(ok = wait_all(&c1_full[r1.stage], r1.phase, kSiteBwdMmaCol))) break;
+    tc_fence_after();
+    issue_rc(dp_col((int)T), desc_r1, adv(desc_c1_k, st_bytes(r1.stage)));
+    commit(&dp_full[dp_bar((int)T)]);
+    if (!kKV) commit(&c1_empty[r1.stage]);
+    if (w.n == 1) commit(r_empty);
     for (int it = 0; it < w.n && ok; ++it) {
-      const uint32_t par = (uint32_t)it & 1u;
+      const int t = (int)T + it;          // tile index over all units (barrier phases)
+      const uint32_t par = (uint32_t)t & 1u;
       Ring n0 = r0, n1 = r1;  // the next tile's
       n0.advance<S0>();
       n1.advance<S1>();
@@ -442,19 +483,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // dP(t+1) into the other buffer, whose P(t-1) / dS(t-1) the previous MMAs have read
           if (!(ok = wait_all(&c1_full[n1.stage], n1.phase, kSiteBwdMmaCol))) break;
           tc_fence_after();
-          issue_rc(dp_col(it + 1), desc_r1, adv(desc_c1_k, st_bytes(n1.stage)));
-          commit(&dp_full[dp_bar(it + 1)]);
+          issue_rc(dp_col(t + 1), desc_r1, adv(desc_c1_k, st_bytes(n1.stage)));
+          commit(&dp_full[dp_bar(t + 1)]);
           if (!kKV) commit(&c1_empty[n1.stage]);
+          if (it + 2 == w.n) commit(r_empty);
         }
       }
+      // the first accumulating MMAs of a unit overwrite the accumulators: the previous unit's
+      // epilogue must have read them
+      if (it == 0 && units > 0u && !(ok = wait_all(acc_free, (units - 1u) & 1u, kSiteBwdMmaDS))) break;
       if (!(ok = wait_all(ds_ready, par, kSiteBwdMmaDS))) break;
       tc_fence_after();
-      issue_acc(kAccDS, dp_col(it) + 32, adv(desc_c0_mn, st_bytes(r0.stage)), it > 0);
+      issue_acc(kAccDS, dp_col(t) + 32, adv(desc_c0_mn, st_bytes(r0.stage)), it > 0);
       commit(&c0_empty[r0.stage]);
       if (kKV) {
         if (!(ok = wait_all(p_ready, par, kSiteBwdMmaP))) break;
         tc_fence_after();
-        issue_acc(kAccP, dp_col(it), adv(desc_c1_mn, st_bytes(r1.stage)), it > 0);
+        issue_acc(kAccP, dp_col(t), adv(desc_c1_mn, st_bytes(r1.stage)), it > 0);
         commit(&c1_empty[r1.stage]);
       }
       if (!kDualDP && has_next) {
@@ -463,11 +508,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_rc(128, desc_r1, adv(desc_c1_k, st_bytes(n1.stage)));
         commit(&dp_full[0]);
         if (!kKV) commit(&c1_empty[n1.stage]);
+        if (it + 2 == w.n) commit(r_empty);
       }
       r0 = n0;
       r1 = n1;
     }
-    if (ok) commit(acc_full);
+    if (!ok) break;
+    commit(acc_full);
+    T += (uint32_t)w.n;
+    ++units;
+    }
     // Drain: all MMAs issued by this warp complete before TMEM is released.
     commit(drain);
     drain_phase(drain, 0u, abort_flag);
@@ -480,6 +530,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_s = tmem_base + lane_off + 64 * h;
     const uint32_t t_dp0 = tmem_base + lane_off + 64 * h;   // + dp_col(t): this thread's dP columns
     const float c = p.c;
+    bool ok = true;
+    Ring ring;  // position of the current tile's C0 (and per-query vectors)
+    // bits 0-1: column tiles of earlier units mod 4 (the per-tile barrier phases need no more);
+    // bit 2: earlier units mod 2 (the accumulator barrier's phase)
+    uint32_t st = 0u;
+    for (int q = 0; ok; ++q) {
+    const int item = (int)blockIdx.x + (q >> 1) * (int)gridDim.x;
+    if (item >= p.num_items) break;
+    BwdUnit w;
+    if (!bwd_unit<kKV>(p, item, q & 1, w)) continue;
     const int row = w.rb * kBlockM + r;         // global index of this thread's tile row
     // Q pass: the row's -lse2 and -delta are fixed for the whole unit.
     float row_nlse2 = 0.f, row_ndelta = 0.f;
@@ -488,11 +548,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       row_nlse2 = p.nlse2[off];
       row_ndelta = p.ndelta[off];
     }
-    bool ok = true;
-    Ring ring;  // position of the current tile's C0 (and per-query vectors)
-    for (int it = 0; it < w.n && ok; ++it) {
-      int cb, chead;
-      bwd_col<kKV>(p, w, it, cb, chead);
+    int cb = w.c0;                              // column block of the current tile
+    for (int it0 = 0; it0 < w.n && ok; ++it0) {
+      const int it = (int)(st & 3u) + it0;      // tile index over all units, mod 4 (barrier phases)
       const uint32_t par = (uint32_t)it & 1u;
       const float* vec = sVec + ring.stage * 2 * kBlockN + 64 * h;
       if (!(ok = wait_phase(s_full, par, abort_flag, kSiteBwdSoftS))) break;
@@ -618,11 +676,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(p_ready);
       }
       ring.advance<S0>();
+      if (++cb == p.num_blocks) cb = w.c0;     // the next query head of the group (KV pass)
     }
 
+    if (!ok) break;
     // Epilogue: this thread's row of acc_p / acc_ds, 32-column chunks alternating between
     // the two warpgroups, scaled (dK, dQ) and rounded to bf16.
-    if (ok && w.n > 0 && wait_phase(acc_full, 0u, abort_flag, kSiteBwdSoftAcc)) {
+    if (!(ok = wait_phase(acc_full, (st >> 2) & 1u, abort_flag, kSiteBwdSoftAcc))) break;
+    {
       tc_fence_after();
       const bool row_ok = row < p.N;
       auto store_acc = [&](uint32_t col, float mul, __nv_bfloat16* out) {
@@ -648,6 +709,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       } else {
         store_acc(kAccDS, p.scale, p.dq);
       }
+      // the accumulators are read: the next unit's first accumulating MMAs may overwrite them
+      tc_fence_before();
+      mbar_arrive(acc_free);
+    }
+    st = ((st + (uint32_t)w.n) & 3u) | ((st ^ 4u) & 4u);
     }
   }
 
