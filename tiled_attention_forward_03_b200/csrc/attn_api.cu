@@ -694,6 +694,14 @@ cudaError_t bwd_setup_dim() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn::attn_bwd_sm100<D, false>),
                              cudaFuncAttributeMaxDynamicSharedMemorySize, attn::BwdPlan<D, false>::kAlloc);
+  // the register split (setmaxnreg) needs exactly the launch allocation it was sized for
+  if (attn::BwdCfg<D>::kSplit) {
+    cudaFuncAttributes fa{};
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(attn::attn_bwd_sm100<D, true>));
+    if (e == cudaSuccess && fa.numRegs != attn::kRegsAtLaunch) e = cudaErrorInvalidDeviceFunction;
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(attn::attn_bwd_sm100<D, false>));
+    if (e == cudaSuccess && fa.numRegs != attn::kRegsAtLaunch) e = cudaErrorInvalidDeviceFunction;
+  }
   return e;
 }
 
@@ -725,9 +733,9 @@ template <int D>
 void launch_bwd_dim(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                     const attn::BwdParams& pkv, const attn::BwdParams& pq, long long grid_kv, long long grid_q,
                     cudaStream_t s) {
-  attn::attn_bwd_sm100<D, true><<<(unsigned)grid_kv, attn::kBwdThreads, attn::BwdPlan<D, true>::kAlloc, s>>>(
+  attn::attn_bwd_sm100<D, true><<<(unsigned)grid_kv, attn::BwdCfg<D>::kThreads, attn::BwdPlan<D, true>::kAlloc, s>>>(
       mk, mv, mq, mdo, pkv);
-  attn::attn_bwd_sm100<D, false><<<(unsigned)grid_q, attn::kBwdThreads, attn::BwdPlan<D, false>::kAlloc, s>>>(
+  attn::attn_bwd_sm100<D, false><<<(unsigned)grid_q, attn::BwdCfg<D>::kThreads, attn::BwdPlan<D, false>::kAlloc, s>>>(
       mq, mdo, mk, mv, pq);
 }
 

@@ -39,11 +39,12 @@
 //   P  = 2^(S c - lse2),  dS = P o (dP - delta)         (lse2, delta per query)
 //   acc_p  += P  C1   (KV pass: dV)          acc_ds += dS C0   (dK or dQ)
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, or 320 at D = 96):
 //   warps 0-7  softmax: TMEM lane = tile row (warp % 4 picks the 32-lane slice), warps 0-3
 //              take columns 0-63 and warps 4-7 columns 64-127 of each tile
 //   warp  8    TMA producer
 //   warp  9    MMA issuer (one elected lane)
+//   warps 10-11 idle (complete the third warpgroup for the register split)
 //
 // Tensor memory (512 columns):
 //   [  0,128) S fp32 (released to the next tile's S as soon as the softmax has loaded it)
@@ -72,7 +73,18 @@
 
 namespace attn {
 
-constexpr int kBwdThreads = 320;
+// Threads per CTA.  D = 32, 64, 128: three warpgroups (softmax warps 0-7, producer 8, MMA 9, idle
+// 10-11) with the forward kernel's register split, the softmax warpgroups at kRegsSoftmax and the
+// third at kRegsControl (launch: 384 x kRegsAtLaunch; removes the spills of a 320-thread CTA's
+// 168-register ceiling; interleaved A/B +1 to +3 %).  D = 96 keeps 320 threads without the split
+// (the split measured -7 % there).
+template <int D>
+struct BwdCfg {
+  static constexpr bool kSplit = D != 96;
+  static constexpr int kThreads = kSplit ? 384 : 320;
+};
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= 384 * kRegsAtLaunch,
+              "backward register split exceeds the launch allocation");
 constexpr float kLog2e = 1.4426950408889634f;
 // Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial (exp2_poly2)
 // instead of the special-function unit.  Measured on B200 (interleaved A/B): at D = 64 the
@@ -255,7 +267,7 @@ __device__ __forceinline__ void bwd_col(const BwdParams& p, const BwdUnit& w, in
 }
 
 template <int D, bool kKV>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     attn_bwd_sm100(const __grid_constant__ CUtensorMap tmap_r0, const __grid_constant__ CUtensorMap tmap_r1,
                    const __grid_constant__ CUtensorMap tmap_c0, const __grid_constant__ CUtensorMap tmap_c1,
                    const BwdParams p) {
@@ -340,6 +352,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
+    if constexpr (BwdCfg<D>::kSplit) regs_decrease<kRegsControl>();
     // Two rings of S stages: C0 tiles (with the KV pass's per-query vectors) and C1 tiles,
     // each refilled as soon as the MMAs that read it have completed.
     if (lane == 0) {
@@ -399,6 +412,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    if constexpr (BwdCfg<D>::kSplit) regs_decrease<kRegsControl>();
     // Per column tile t (tcgen05 MMAs of one CTA run in issue order):
     //   S(t+1) once the softmax has S(t) in registers;
     //   acc_ds(t) once dS(t) is in TMEM, then C0(t) is released;
@@ -522,8 +536,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     commit(drain);
     drain_phase(drain, 0u, abort_flag);
     __syncwarp();
+  } else if (warp >= 10) {
+    // idle: completes the third warpgroup, whose registers go to the softmax warps
+    if constexpr (BwdCfg<D>::kSplit) regs_decrease<kRegsControl>();
   } else {
     // ------------------------------------------------------------ softmax warps 0-7
+    if constexpr (BwdCfg<D>::kSplit) regs_increase<kRegsSoftmax>();
     const int r = threadIdx.x & 127;            // tile row == TMEM lane
     const int h = warp >> 2;                    // column half
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
