@@ -173,6 +173,8 @@ def call_rope(**kw):
     (dict(D=80), UNSUPPORTED), (dict(D=384), UNSUPPORTED), (dict(q=P + 8), MISALIGNED),
     (dict(c=P + 4), MISALIGNED), (dict(ko=P + 2), MISALIGNED),
     (dict(B=1 << 20, Hq=1 << 10, Hkv=1 << 10, N=1 << 20), UNSUPPORTED),
+    # rows of Q and K together at 2^32 (the kernel's 32-bit row index) and one below
+    (dict(B=1, Hq=1 << 15, Hkv=1 << 15, N=1 << 16, D=32), UNSUPPORTED),
 ])
 def test_rope_rejected_before_any_cuda_call(kw, expected):
     assert call_rope(**kw) == expected

@@ -32,7 +32,7 @@ def attn():
 
 @pytest.mark.parametrize("B,Hq,Hkv,N,D,base", [
     (1, 2, 1, 300, 128, 10000.0), (2, 4, 4, 129, 64, 10000.0), (1, 3, 1, 77, 96, 500.0), (1, 2, 2, 1, 32, 10000.0),
-    (1, 2, 1, 16384, 128, 10000.0),
+    (1, 2, 1, 16384, 128, 10000.0), (1, 2, 1, 300, 192, 10000.0), (2, 2, 2, 129, 256, 500.0),
 ])
 def test_rope_rotation(attn, B, Hq, Hkv, N, D, base):
     q, k, _ = make_qkv(B, Hq, Hkv, N, D, 4000 + N)

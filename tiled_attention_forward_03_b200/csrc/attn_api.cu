@@ -856,8 +856,9 @@ int rope_checks(const void* q, const void* k, const float* cos_t, const float* s
                 int N, int D) {
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0) return ATTN_ERR_INVALID_ARG;
   if (!supported_head_dim(D)) return ATTN_ERR_UNSUPPORTED;
-  // one thread per 8 rotation pairs, 256 per block, on a 1-D grid (< 2^31 blocks)
-  if ((long long)B * (Hq + Hkv) * (long long)N * (D / 16) > (1LL << 38)) return ATTN_ERR_UNSUPPORTED;
+  // rows of Q and K together below 2^32 (the kernel indexes rows in 32 bits; a bf16 tensor of
+  // 2^32 rows of D >= 32 would take 256 GB): one thread per 8 rotation pairs, < 2^31 blocks
+  if ((long long)B * (Hq + Hkv) * (long long)N >= (1LL << 32)) return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return ATTN_OK;
   if (!q || !k || !cos_t || !sin_t) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(cos_t, 16) || !aligned(sin_t, 16)) return ATTN_ERR_MISALIGNED;
@@ -870,10 +871,21 @@ int launch_rope(const void* q, const void* k, const float* cos_t, const float* s
   const long long q_rows = (long long)B * Hq * N, k_rows = (long long)B * Hkv * N;
   const long long items = (q_rows + k_rows) * (D / 16);
   const int threads = 256;
-  const long long per_block = (long long)threads * attn::kRopeItems;
-  attn::attn_rope_qk<<<(unsigned)((items + per_block - 1) / per_block), threads, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k), cos_t, sin_t,
-      reinterpret_cast<__nv_bfloat16*>(q_out), reinterpret_cast<__nv_bfloat16*>(k_out), q_rows, k_rows, N, D, sgn);
+  const unsigned grid = (unsigned)((items + threads - 1) / threads);
+  const attn::FastDiv div_n = attn::make_fast_div((uint32_t)N);
+  const auto qb = reinterpret_cast<const __nv_bfloat16*>(q);
+  const auto kb = reinterpret_cast<const __nv_bfloat16*>(k);
+  const auto qo = reinterpret_cast<__nv_bfloat16*>(q_out);
+  const auto ko = reinterpret_cast<__nv_bfloat16*>(k_out);
+  const uint32_t qr = (uint32_t)q_rows, kr = (uint32_t)k_rows, n = (uint32_t)N;
+  switch (D) {
+    case 32: attn::attn_rope_qk<32><<<grid, threads, 0, s>>>(qb, kb, cos_t, sin_t, qo, ko, qr, kr, n, div_n, sgn); break;
+    case 64: attn::attn_rope_qk<64><<<grid, threads, 0, s>>>(qb, kb, cos_t, sin_t, qo, ko, qr, kr, n, div_n, sgn); break;
+    case 96: attn::attn_rope_qk<96><<<grid, threads, 0, s>>>(qb, kb, cos_t, sin_t, qo, ko, qr, kr, n, div_n, sgn); break;
+    case 128: attn::attn_rope_qk<128><<<grid, threads, 0, s>>>(qb, kb, cos_t, sin_t, qo, ko, qr, kr, n, div_n, sgn); break;
+    case 192: attn::attn_rope_qk<192><<<grid, threads, 0, s>>>(qb, kb, cos_t, sin_t, qo, ko, qr, kr, n, div_n, sgn); break;
+    default: attn::attn_rope_qk<256><<<grid, threads, 0, s>>>(qb, kb, cos_t, sin_t, qo, ko, qr, kr, n, div_n, sgn); break;
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     record_cuda_error("rope kernel launch", e);

@@ -23,71 +23,54 @@
 
 #include <cuda_bf16.h>
 
-#include "sm100_ptx.cuh"
+#include "attn_fwd_kernel.cuh"  // FastDiv, and the PTX wrappers
 
 namespace attn {
 
-// Work item = one 8-pair piece of one row; each thread takes kRopeItems items (grid-strided
-// by the thread count, so a warp's accesses stay contiguous) and issues all their loads first.
-// Measured on B200 (B4 H16 N2048 D128): one item per thread 4.7 TB/s, two 4.0 TB/s.
-constexpr int kRopeItems = 1;
+// Work item = one 8-pair piece of one row, one per thread (all loads issued before any use).
+// The row and the piece come from the item by a division by the compile-time piece count, the
+// position in the sequence from the row by a multiply-high division by N (rows < 2^32, checked
+// on the host).  Measured on B200 (B4 H16 N2048 D128): 4.96 TB/s, against 4.7 TB/s with 64-bit
+// divisions by runtime values here; two items per thread measured 4.0 TB/s.
+template <int D>
 __global__ void __launch_bounds__(256) attn_rope_qk(const __nv_bfloat16* q, const __nv_bfloat16* k,
                                                     const float* __restrict__ cos_t,
                                                     const float* __restrict__ sin_t, __nv_bfloat16* q_out,
-                                                    __nv_bfloat16* k_out, long long q_rows, long long k_rows,
-                                                    int N, int D, float sgn) {
-  const int pieces = D / 16;  // 8-pair pieces per row
-  const int half = D / 2;
-  const long long q_items = q_rows * pieces;
-  const long long total = q_items + k_rows * pieces;
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  const long long first = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  uint4 ua[kRopeItems], ub[kRopeItems];
-  float4 cv[kRopeItems][2], sv[kRopeItems][2];
+                                                    __nv_bfloat16* k_out, uint32_t q_rows, uint32_t k_rows,
+                                                    uint32_t N, FastDiv div_n, float sgn) {
+  constexpr int kPieces = D / 16;  // 8-pair pieces per row
+  constexpr int kHalf = D / 2;
+  const unsigned long long q_items = (unsigned long long)q_rows * kPieces;
+  const unsigned long long total = q_items + (unsigned long long)k_rows * kPieces;
+  const unsigned long long item = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (item >= total) return;
+  const bool is_q = item < q_items;
+  const unsigned long long it = is_q ? item : item - q_items;
+  const uint32_t row = (uint32_t)(it / kPieces);
+  const int d = (int)(it - (unsigned long long)row * kPieces) * 8;
+  const uint32_t pos = row - fast_div(row, div_n) * N;
+  const __nv_bfloat16* src = (is_q ? q : k) + (size_t)row * D;
+  const uint4 ua = *reinterpret_cast<const uint4*>(src + d);
+  const uint4 ub = *reinterpret_cast<const uint4*>(src + kHalf + d);
+  const float4* ct = reinterpret_cast<const float4*>(cos_t + (size_t)pos * kHalf + d);
+  const float4* st = reinterpret_cast<const float4*>(sin_t + (size_t)pos * kHalf + d);
+  const float4 c0 = ct[0], c1 = ct[1], s0 = st[0], s1 = st[1];
+  __nv_bfloat16* dst = (is_q ? q_out : k_out) + (size_t)row * D;
+  const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&ua);
+  const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&ub);
+  uint32_t oa[4], ob[4];
 #pragma unroll
-  for (int u = 0; u < kRopeItems; ++u) {
-    const long long item = first + u * stride;
-    if (item >= total) continue;
-    const bool is_q = item < q_items;
-    const long long it = is_q ? item : item - q_items;
-    const long long row = it / pieces;
-    const int d = (int)(it - row * pieces) * 8;
-    const int pos = (int)(row % N);
-    const __nv_bfloat16* src = (is_q ? q : k) + row * D;
-    ua[u] = *reinterpret_cast<const uint4*>(src + d);
-    ub[u] = *reinterpret_cast<const uint4*>(src + half + d);
-    const float4* ct = reinterpret_cast<const float4*>(cos_t + (size_t)pos * half + d);
-    const float4* st = reinterpret_cast<const float4*>(sin_t + (size_t)pos * half + d);
-    cv[u][0] = ct[0];
-    cv[u][1] = ct[1];
-    sv[u][0] = st[0];
-    sv[u][1] = st[1];
+  for (int e = 0; e < 4; ++e) {
+    const float2 a = __bfloat1622float2(pa[e]);
+    const float2 b = __bfloat1622float2(pb[e]);
+    const float c_lo = cs[2 * e], c_hi = cs[2 * e + 1], s_lo = sgn * sn[2 * e], s_hi = sgn * sn[2 * e + 1];
+    oa[e] = pack_bf16x2(fmaf(a.x, c_lo, -b.x * s_lo), fmaf(a.y, c_hi, -b.y * s_hi));
+    ob[e] = pack_bf16x2(fmaf(b.x, c_lo, a.x * s_lo), fmaf(b.y, c_hi, a.y * s_hi));
   }
-#pragma unroll
-  for (int u = 0; u < kRopeItems; ++u) {
-    const long long item = first + u * stride;
-    if (item >= total) continue;
-    const bool is_q = item < q_items;
-    const long long it = is_q ? item : item - q_items;
-    const long long row = it / pieces;
-    const int d = (int)(it - row * pieces) * 8;
-    __nv_bfloat16* dst = (is_q ? q_out : k_out) + row * D;
-    const float cs[8] = {cv[u][0].x, cv[u][0].y, cv[u][0].z, cv[u][0].w, cv[u][1].x, cv[u][1].y, cv[u][1].z, cv[u][1].w};
-    const float sn[8] = {sv[u][0].x, sv[u][0].y, sv[u][0].z, sv[u][0].w, sv[u][1].x, sv[u][1].y, sv[u][1].z, sv[u][1].w};
-    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&ua[u]);
-    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&ub[u]);
-    uint32_t oa[4], ob[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 a = __bfloat1622float2(pa[e]);
-      const float2 b = __bfloat1622float2(pb[e]);
-      const float c_lo = cs[2 * e], c_hi = cs[2 * e + 1], s_lo = sgn * sn[2 * e], s_hi = sgn * sn[2 * e + 1];
-      oa[e] = pack_bf16x2(fmaf(a.x, c_lo, -b.x * s_lo), fmaf(a.y, c_hi, -b.y * s_hi));
-      ob[e] = pack_bf16x2(fmaf(b.x, c_lo, a.x * s_lo), fmaf(b.y, c_hi, a.y * s_hi));
-    }
-    *reinterpret_cast<uint4*>(dst + d) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-    *reinterpret_cast<uint4*>(dst + half + d) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-  }
+  *reinterpret_cast<uint4*>(dst + d) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+  *reinterpret_cast<uint4*>(dst + kHalf + d) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
 }
 
 }  // namespace attn
