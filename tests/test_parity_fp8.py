@@ -117,7 +117,7 @@ def test_fp8_wide_persistent_items_sampled(attn, B, Hq, Hkv, N, D, causal):
     assert_close(o[idx], lse[idx], o_ref, lse_ref, f"fp8 wide persistent B{B} N{N} D{D}")
 
 
-@pytest.mark.parametrize("name", ["cfg3", "sweep_D128_N8192_noncausal", "sweep_D64_N4096_noncausal",
+@pytest.mark.parametrize("name", ["cfg3", "cfg4", "sweep_D128_N8192_noncausal", "sweep_D64_N4096_noncausal",
                                   "sweep_D64_N4096_causal", "wide_D192_N8192_noncausal", "wide_D256_N8192_noncausal",
                                   "wide_D256_N8192_causal", "wide_D192_N2048_causal"])
 def test_fp8_benchmark_workloads_sampled(attn, name):

@@ -224,9 +224,18 @@ def test_backward_rope(attn, B, Hq, Hkv, N, D, causal):
         assert_grad_close(a.float().cpu().numpy().astype(np.float64), r, f"rope backward {name}")
 
 
-def test_backward_rope_is_rotate_backward_then_inverse(attn):
-    """attn_bwd_rope equals its three steps called one by one (bit for bit)."""
-    B, Hq, Hkv, N, D, causal = 2, 4, 2, 700, 128, True
+@pytest.mark.parametrize("shape", [(2, 4, 2, 700, 128, True), "cfg2", "cfg3"], ids=str)
+def test_backward_rope_is_rotate_backward_then_inverse(attn, shape):
+    """attn_bwd_rope equals its three steps called one by one (bit for bit), also at the sizes
+    the backward through RoPE is benchmarked on (cfg2, cfg3), where the plain backward's own
+    parity is checked on sampled heads."""
+    from attn_inputs import get_workload
+
+    if isinstance(shape, str):
+        w = get_workload(shape)
+        B, Hq, Hkv, N, D, causal = w.B, w.Hq, w.Hkv, w.N, w.D, w.causal
+    else:
+        B, Hq, Hkv, N, D, causal = shape
     q, k, v = (x.cuda() for x in make_qkv(B, Hq, Hkv, N, D, 4400))
     do = make_dout(B, Hq, N, D, 4401).cuda()
     cos_t, sin_t = attn.rope_tables(N, D, device="cuda")
