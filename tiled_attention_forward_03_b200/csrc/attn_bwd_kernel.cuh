@@ -132,8 +132,8 @@ struct BwdPlan {
   static constexpr int kVecOff = kC1Off + kStages1 * kTileBytes;
   static constexpr int kBarOff = kVecOff + kStages0 * kVecBytes;
   // r_full c0_full[S0] c0_empty[S0] c1_full[S1] c1_empty[S1] s_full s_free dp_full[2] p_ready
-  // ds_ready acc_full drain r_empty acc_free
-  static constexpr int kNumBars = 1 + 2 * kStages0 + 2 * kStages1 + 10;
+  // ds_ready acc_full drain r_empty acc_free p_ready' ds_ready' (the last two: second dP buffer)
+  static constexpr int kNumBars = 1 + 2 * kStages0 + 2 * kStages1 + 12;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -306,6 +306,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   auto dp_col = [](int t) -> uint32_t { return 128u + (kDualDP ? 128u * (uint32_t)(t & 1) : 0u); };
   auto dp_bar = [](int t) -> int { return kDualDP ? (t & 1) : 0; };
   auto dp_par = [](int t) -> uint32_t { return kDualDP ? (((uint32_t)t >> 1) & 1u) : ((uint32_t)t & 1u); };
+  // dS and P of tile t are ready: one barrier per dP buffer, like dp_full.  With two buffers the
+  // softmax can finish tile t+1 (its S and dP are issued early) before the MMA warp has waited for
+  // tile t; a single barrier would then complete twice and its parity wait for t would stall.
+  auto ds_ready_bar = [&](int t) -> uint64_t* { return (kDualDP && (t & 1)) ? s_full + 11 : s_full + 5; };
+  auto p_ready_bar = [&](int t) -> uint64_t* { return (kDualDP && (t & 1)) ? s_full + 10 : s_full + 4; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Plan::kMiscOff);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Plan::kMiscOff + 4);
 
@@ -328,6 +333,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     mbar_init(&dp_full[1], 1);
     mbar_init(p_ready, 256);
     mbar_init(ds_ready, 256);
+    mbar_init(s_full + 10, 256);
+    mbar_init(s_full + 11, 256);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     mbar_init(r_empty, 1);
@@ -506,12 +513,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       // the first accumulating MMAs of a unit overwrite the accumulators: the previous unit's
       // epilogue must have read them
       if (it == 0 && units > 0u && !(ok = wait_all(acc_free, (units - 1u) & 1u, kSiteBwdMmaDS))) break;
-      if (!(ok = wait_all(ds_ready, par, kSiteBwdMmaDS))) break;
+      if (!(ok = wait_all(ds_ready_bar(t), dp_par(t), kSiteBwdMmaDS))) break;
       tc_fence_after();
       issue_acc(kAccDS, dp_col(t) + 32, adv(desc_c0_mn, st_bytes(r0.stage)), it > 0);
       commit(&c0_empty[r0.stage]);
       if (kKV) {
-        if (!(ok = wait_all(p_ready, par, kSiteBwdMmaP))) break;
+        if (!(ok = wait_all(p_ready_bar(t), dp_par(t), kSiteBwdMmaP))) break;
         tc_fence_after();
         issue_acc(kAccP, dp_col(t), adv(desc_c1_mn, st_bytes(r1.stage)), it > 0);
         commit(&c1_empty[r1.stage]);
@@ -680,7 +687,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(ds_ready);
+      mbar_arrive(ds_ready_bar(it));
       if (kKV) {
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
@@ -691,7 +698,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(p_ready);
+        mbar_arrive(p_ready_bar(it));
       }
       ring.advance<S0>();
       if (++cb == p.num_blocks) cb = w.c0;     // the next query head of the group (KV pass)
