@@ -55,7 +55,8 @@ typedef enum {
  *         is an empty problem: ATTN_OK is returned and nothing is launched
  *         (pointers may then be null).  Limits: B*Hq <= 2^31-1, N <= 2^31-1 and
  *         B*Hq*ceil(N/256) <= 2^31-1 (work units of 256 query rows, indexed in 32 bits
- *         by the scheduler); beyond them ATTN_ERR_UNSUPPORTED.
+ *         by the scheduler), and at D = 192, 256 B*Hq*ceil(N/128) <= 2^30 (query tiles of the
+ *         wide-head kernel); beyond them ATTN_ERR_UNSUPPORTED.
  *   D     head dim of q, k, v and o: 32, 64, 96, 128, 192 or 256.  D <= 128 runs on the two-tile
  *         kernel (two 128-row Q tiles per CTA ping-pong on the tensor core); 192 and 256 run on a
  *         one-tile kernel that ping-pongs two score buffers instead (2 x (128 + D) tensor-memory

@@ -64,6 +64,8 @@ def call(**kw):
     (dict(D=80), UNSUPPORTED), (dict(D=384), UNSUPPORTED), (dict(D=0), UNSUPPORTED), (dict(D=48), UNSUPPORTED),
     (dict(D=160), UNSUPPORTED), (dict(q=P + 8), MISALIGNED), (dict(k=P + 2), MISALIGNED), (dict(v=P + 4), MISALIGNED),
     (dict(o=P + 1), MISALIGNED), (dict(lse=P + 2), MISALIGNED),
+    # D = 192, 256: more than 2^30 query tiles (the wide-head kernel steps through them in 32 bits)
+    (dict(B=1 << 10, Hq=1 << 10, Hkv=1 << 10, N=(1 << 17) + 1, D=256), UNSUPPORTED),
 ])
 def test_rejected_before_any_cuda_call(kw, expected):
     assert call(**kw) == expected

@@ -311,6 +311,9 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
   if ((long long)B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   // the scheduler indexes work units (256 query rows of one head) in 32 bits
   if (attn_num_units(B, Hq, N) > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  // D = 192, 256: the wide-head kernel's CTAs step through its tiles in 32 bits
+  if (!narrow_head_dim(D) && (long long)B * Hq * (((long long)N + attn::kBlockN - 1) / attn::kBlockN) > (1LL << 30))
+    return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return ATTN_OK;  // empty problem: nothing to compute or write
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
@@ -351,8 +354,7 @@ int launch_forward(const void* q, const void* k, const void* v, void* o, float* 
                       : attn::idesc_bf16_f32(attn::kBlockM, attn::kBlockN, false, false, ws_eff < 0.f);
     wp.idesc_pv = e4m3 ? attn::idesc_e4m3_f32(attn::kBlockM, D, false, true, false)
                        : attn::idesc_bf16_f32(attn::kBlockM, D, false, true, false);
-    const long long tiles = (long long)B * Hq * wp.num_blocks;
-    if (tiles > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    const long long tiles = (long long)B * Hq * wp.num_blocks;   // <= 2^30, checked above
     // Work items: causal, a head's heaviest and lightest tiles together (equal items) when
     // there are enough of them to fill the GPU, else single tiles.  CTAs are persistent for
     // causal shapes and for N <= 2048 (one CTA per SM walking the items: the next tile's Q
